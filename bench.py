@@ -1,0 +1,353 @@
+"""Benchmark of the VSA block-sparse attention forward on B200.
+
+One step = one VSA attention call on the 1344x768 5 s shape (133,696 tokens:
+4,672 conditioning + 32x48x84 video, H=24, d=128, keep 10%, exact_kv), i.e.
+vsa_coarse_select + vsa_sparse_attn_fwd on inputs resident in HBM; the
+geometry map is built and uploaded once per shape, outside the timed region.
+
+Metric: effective TFLOP/s of the fine branch's valid work (4 * 128 FLOP per
+attended (query, key) pair, x heads), and ms per call. Inputs (2.5 GB) are
+larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun), every rank runs its own copy of the workload (weak
+scaling, no collective on the data path); timing is the max over ranks.
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per VSA attention call and effective TFLOP/s (% bf16 peak) at 129k tokens"
+WORKLOAD = "5s"
+
+
+def valid_flop_fast(counts, n_cond, idx, cnt, sink_rows):
+    """Valid fine-branch FLOP of one call: 4 * 128 per attended (valid query,
+    valid key) pair; keys of a query tile = conditioning tokens + tokens of its
+    selected video tiles (all tokens for dense conditioning rows)."""
+    counts = counts.astype(np.float64)
+    vid = counts[n_cond:]
+    B, H, Nt, kmax = idx.shape
+    mask = np.arange(kmax)[None, None, None, :] < cnt[..., None]
+    keys = np.where(mask, vid[np.clip(idx, 0, len(vid) - 1)], 0.0).sum(-1) + counts[:n_cond].sum()
+    if sink_rows:
+        keys[:, :, :n_cond] = counts.sum()
+    return 4.0 * 128.0 * float((keys * counts[None, None, :]).sum())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, bits, lay, head, n_tiles, rng_seed=0):
+    """Times the oracle on one head: its whole selection and the fine branch of
+    n_tiles query tiles. Returns (seconds, valid FLOP of the sampled fine work,
+    seconds extrapolated to one whole call)."""
+    from oracle import vsa_oracle as O
+    f = O.bf16_bits_to_f64
+    q, k, v, g = bits
+    t0 = time.perf_counter()
+    qh, kh, vh, gh = f(q[0, :, head]), f(k[0, :, head]), f(v[0, :, head]), f(g[0, :, head])
+    p = O.Params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink)
+    qb, kb, vb, sc, sel, thr, oc, scale = O.selection_for_head(qh, kh, vh, lay, p)
+    t_sel = time.perf_counter() - t0
+    tiles = np.random.default_rng(rng_seed).choice(lay.n_tiles, n_tiles, replace=False)
+    flop = 0.0
+    counts = (lay.perm >= 0).sum(1)
+    t1 = time.perf_counter()
+    for qt in tiles:
+        keys = O.key_tokens_for_tile(lay, int(qt), sel[qt], p.sink)
+        O.output_rows_for_tile(qh, kh, vh, gh, lay, p, int(qt), sel[qt], oc, scale)
+        flop += 4.0 * 128 * counts[qt] * keys.size
+    t_fine = time.perf_counter() - t1
+    secs = t_sel * n_tiles / lay.n_tiles + t_fine
+    per_call = (t_sel + t_fine * lay.n_tiles / n_tiles) * wl.H
+    return secs, flop, per_call
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(n[0]) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from block_sparse_video_geometry_b200 import workloads as W
+    from oracle import vsa_oracle as O
+    wl = W.WORKLOADS[args.workload]
+    lay = O.build_layout([O.Segment(k, s, n, gr) for (k, s, n, gr) in wl.segments()], wl.seq_len)
+    bits = W.make_inputs(wl, lay.inv // O.TILE)
+    n_tiles = args.ref_tiles
+    for i in range(args.warmup):
+        oracle_sample(wl, bits, lay, head=i % wl.H, n_tiles=max(2, n_tiles // 4), rng_seed=i)
+    secs, flops = 0.0, 0.0
+    per_call = []
+    for i in range(args.steps):
+        s, fl, pc = oracle_sample(wl, bits, lay, head=(i * 7) % wl.H, n_tiles=n_tiles, rng_seed=100 + i)
+        secs += s
+        flops += fl
+        per_call.append(pc)
+    tflops = flops / secs / 1e12
+    ms_call = 1e3 * statistics.mean(per_call)
+    sample = ("one head per step: its whole selection (pool, scores, top-k, coarse) pro rata plus the fine "
+              "branch of %d random query tiles; ms_per_step extrapolated to a whole call (24 heads)" % n_tiles)
+    line = {"impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "1344x768 5 s: 4672 conditioning + 32x48x84 video tokens, H=24, d=128, "
+                                   "keep 10%, exact_kv", "B": wl.B, "seq_len": wl.seq_len,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    from block_sparse_video_geometry_b200 import vsa, workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = W.WORKLOADS[args.workload].with_(seed=W.WORKLOADS[args.workload].seed + rank)
+    lay = vsa.Layout(wl.segments(), wl.seq_len)
+    perm, inv, counts, kinds = lay.tables()
+    bits = W.make_inputs(wl, inv // vsa.TILE)
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v, g = (to_dev(x) for x in bits)
+    stream = torch.cuda.Stream(device=dev)
+    out_dtype = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
+    params = vsa.make_params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink)
+    with torch.cuda.stream(stream):
+        fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, out_dtype=out_dtype, stream=stream)
+        out = torch.empty(q.shape, dtype=out_dtype, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
+        vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
+                            fwd.ws_attn, stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = vsa.sparse_attn_status(fwd.ws_attn, stream)
+    if st != vsa.OK:
+        raise RuntimeError("kernel status %s" % vsa.status_string(st))
+    flop = valid_flop_fast(counts, lay.info.n_cond_tiles, fwd.idx.cpu().numpy(), fwd.cnt.cpu().numpy(),
+                           wl.sink == vsa.SINK_EXACT_KV_AND_ROWS)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+
+    # ---- headline: K whole steps, device-timed on the launching stream
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+
+    # ---- per-kernel split: selection call vs attention call, events on the same stream
+    sel_ms, att_ms = [], []
+    for _ in range(max(3, min(args.steps, 10))):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
+        e[1].record(stream)
+        vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
+                            fwd.ws_attn, stream)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        sel_ms.append(e[0].elapsed_time(e[1]))
+        att_ms.append(e[1].elapsed_time(e[2]))
+    sel_ms, att_ms = statistics.median(sel_ms), statistics.median(att_ms)
+
+    # ---- end to end through the public API with host buffers
+    host_in = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in bits]
+    host_out = torch.empty(out.shape, dtype=out_dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(2, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        barrier()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            for hsrc, ddst in zip(host_in, (q, k, v, g)):
+                ddst.copy_(hsrc, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+        ev1.record(stream)
+        barrier()
+    ms_e2e = ev0.elapsed_time(ev1) / e2e_steps
+
+    times = torch.tensor([ms_step, ms_e2e, att_ms, sel_ms], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    ms_step, ms_e2e, att_ms, sel_ms = times.tolist()
+
+    if rank == 0:
+        peaks, src = measured_peaks()
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        achieved = flop / (att_ms * 1e-3) / 1e12
+        info = lay.info
+        ld = (info.n_video_tiles + 63) // 64 * 64
+        sel_bytes = (3 * q.numel() * 2                                           # Q, K, V read once
+                     + 2 * wl.B * wl.H * info.n_tiles * ld * 4                    # scores written + read
+                     + 4 * wl.B * wl.H * info.n_tiles * (fwd.kmax + 1 + 128))    # idx, cnt, o_coarse
+        value = world * flop / (ms_step * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "1344x768 5 s: 4672 conditioning (512 text + 48x84 ref image + 128 "
+                                   "audio) + 32x48x84 video tokens, H=24, d=128, keep 10%, exact_kv, "
+                                   "%s output" % args.out_dtype,
+                       "B": wl.B, "seq_len": wl.seq_len, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
+                       "l2": "inputs (2.5 GB) larger than L2; no flush"},
+            "roofline": {"bound": "tensor", "kernel": "vsa_attn_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": "%s bf16_tflops_sustained" % src,
+                         "frac_of_burst": achieved / peaks["bf16_tflops"],
+                         "flop_per_launch": flop, "ms_per_launch": att_ms},
+            "selection": {"bound": "hbm", "achieved": sel_bytes / (sel_ms * 1e-3) / 1e9,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": sel_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                          "bytes_per_call": sel_bytes, "ms_per_call": sel_ms},
+            "e2e": {"value": world * flop / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "gpu_launches": 4 * wl.B * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            from oracle import vsa_oracle as O
+            olay = O.build_layout([O.Segment(k_, s_, n_, g_) for (k_, s_, n_, g_) in wl.segments()], wl.seq_len)
+            secs, fl, per_call = oracle_sample(wl, bits, olay, head=0, n_tiles=args.ref_tiles)
+            line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+                                    "kind": "oracle", "ms_per_call_extrapolated": per_call * 1e3,
+                                    "sample": "head 0: whole selection pro rata + fine branch of %d random "
+                                              "query tiles" % args.ref_tiles}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32")
+    ap.add_argument("--ref-tiles", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

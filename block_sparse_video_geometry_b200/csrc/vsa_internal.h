@@ -1,0 +1,95 @@
+// Internal definitions shared by the host layout builder and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "vsa.h"
+
+namespace vsa {
+
+constexpr int kTile = VSA_TILE;       // tokens per tile
+constexpr int kCube = 4;              // 4x4x4 video cubes
+constexpr int kHeadDim = VSA_HEAD_DIM;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Device copy of the geometry map. All arrays live in one caller-owned buffer.
+//  perm   [n_tiles*64]  token of (tile, slot), -1 for padding
+//  inv    [seq_len]     tile*64 + slot of each token
+//  valid  [n_tiles]     bit s set <=> slot s holds a token
+//  count  [n_tiles]     popcount(valid)
+//  origin [n_tiles]     conditioning tile: (first token, 0, 0, kind)
+//                       video tile:        (t0, h0, w0, VSA_SEG_VIDEO)
+struct DevLayout {
+  const int32_t* perm;
+  const int32_t* inv;
+  const unsigned long long* valid;
+  const int32_t* count;
+  const int4* origin;
+  int32_t n_cond;
+  int32_t n_video;
+  int32_t n_tiles;
+  int32_t grid_t, grid_h, grid_w;
+  int64_t video_start;
+  int64_t seq_len;
+};
+
+struct TablesOffsets {
+  size_t perm, inv, valid, count, origin, total;
+};
+
+}  // namespace vsa
+
+struct vsa_layout {
+  int64_t seq_len = 0;
+  int32_t n_cond = 0, n_video = 0, n_tiles = 0;
+  int32_t grid_t = 0, grid_h = 0, grid_w = 0;
+  int64_t video_start = 0;
+  std::vector<int32_t> perm, inv, count, kind;
+  std::vector<unsigned long long> valid;
+  std::vector<int32_t> origin;   // 4 per tile
+  vsa::TablesOffsets off{};
+  void* dev_buf = nullptr;       // caller-owned, set by vsa_layout_upload
+
+  vsa::DevLayout dev() const {
+    const char* b = static_cast<const char*>(dev_buf);
+    vsa::DevLayout d;
+    d.perm = reinterpret_cast<const int32_t*>(b + off.perm);
+    d.inv = reinterpret_cast<const int32_t*>(b + off.inv);
+    d.valid = reinterpret_cast<const unsigned long long*>(b + off.valid);
+    d.count = reinterpret_cast<const int32_t*>(b + off.count);
+    d.origin = reinterpret_cast<const int4*>(b + off.origin);
+    d.n_cond = n_cond;
+    d.n_video = n_video;
+    d.n_tiles = n_tiles;
+    d.grid_t = grid_t;
+    d.grid_h = grid_h;
+    d.grid_w = grid_w;
+    d.video_start = video_start;
+    d.seq_len = seq_len;
+    return d;
+  }
+};
+
+namespace vsa {
+
+// k for top-k selection: max(1, ceil(keep * Nv * (1 - 2^-20))), clamped to Nv.
+int32_t topk_count(float keep, int32_t n_video);
+
+// Validation shared by the entry points.
+vsa_status check_params(const vsa_params* p);
+float effective_scale(const vsa_params* p);
+vsa_status check_qkv(const void* q, const void* k, const void* v, int64_t sb, int64_t ss,
+                     int64_t sh, int32_t B, int32_t H);
+
+// Workspace layout of vsa_coarse_select.
+struct SelectWorkspace {
+  size_t pooled, scores, stats, total;
+  int32_t n_row_blocks;   // 64-query-tile blocks of the coarse kernel
+  int32_t ld_scores;      // score row stride: Nv rounded up to 64
+};
+SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H);
+
+}  // namespace vsa

@@ -1,0 +1,261 @@
+"""ctypes binding of libvsa (C ABI in include/vsa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. torch tensors are used as device buffers and torch streams as CUDA
+streams. The library is loaded on first use; if it is missing the call raises,
+there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvsa.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, ERR_TIMEOUT, ERR_NOT_UPLOADED = range(7)
+SEG_TEXT, SEG_REF_IMAGE, SEG_REF_AUDIO, SEG_OTHER_COND, SEG_VIDEO = range(5)
+SELECT_TOPK, SELECT_ADAPTIVE = 0, 1
+SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS = 0, 1
+OUT_F32, OUT_BF16 = 0, 1
+TILE, HEAD_DIM = 64, 128
+
+
+class VSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32),
+                ("grid_w", ctypes.c_int32), ("start", ctypes.c_int64), ("length", ctypes.c_int64)]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("keep", ctypes.c_float), ("tau", ctypes.c_float),
+                ("sink", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class LayoutInfo(ctypes.Structure):
+    _fields_ = [("seq_len", ctypes.c_int64), ("n_cond_tiles", ctypes.c_int32),
+                ("n_video_tiles", ctypes.c_int32), ("n_tiles", ctypes.c_int32),
+                ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("video_start", ctypes.c_int64), ("device_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32, _I64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+_SIGNATURES = {
+    "vsa_layout_build": (_I32, [ctypes.POINTER(Segment), _I32, _I64, _P, _SZ, _P, ctypes.POINTER(_P)]),
+    "vsa_layout_upload": (_I32, [_P, _P, _SZ, _P]),
+    "vsa_layout_query": (_I32, [_P, ctypes.POINTER(LayoutInfo)]),
+    "vsa_layout_copy_tables": (_I32, [_P, _P, _P, _P, _P]),
+    "vsa_layout_free": (None, [_P]),
+    "vsa_select_kmax": (_I32, [_P, ctypes.POINTER(Params), ctypes.POINTER(_I32)]),
+    "vsa_coarse_select_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
+    "vsa_coarse_select": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
+                                 _P, _P, _P, _P, _SZ, _P]),
+    "vsa_sparse_attn_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
+    "vsa_sparse_attn_fwd": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
+                                   _P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64, _I64,
+                                   _P, _SZ, _P]),
+    "vsa_sparse_attn_status": (_I32, [_P, _P]),
+    "vsa_status_string": (ctypes.c_char_p, [_I32]),
+    "vsa_version": (_I32, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libvsa.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libvsa.so is missing: build it with "
+                               "`python -m block_sparse_video_geometry_b200.build_ext`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().vsa_status_string(status).decode()
+
+
+def version() -> int:
+    return lib().vsa_version()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise VSAError(status, where)
+
+
+def make_params(mode: int = SELECT_TOPK, keep: float = 0.1, tau: float = 1.0,
+                sink: int = SINK_EXACT_KV, scale: float = 0.0) -> Params:
+    return Params(mode, keep, tau, sink, scale)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return 0
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream        # torch.cuda.Stream
+
+
+class Layout:
+    """Owned vsa_layout handle. `segments` is a list of (kind, start, length,
+    (t, h, w) or None) in sequence order."""
+
+    def __init__(self, segments, seq_len: int):
+        arr = (Segment * len(segments))()
+        for i, (kind, start, length, grid) in enumerate(segments):
+            t, h, w = grid if grid is not None else (0, 0, 0)
+            arr[i] = Segment(kind, t, h, w, start, length)
+        handle = _P()
+        _check(lib().vsa_layout_build(arr, len(segments), seq_len, None, 0, None, ctypes.byref(handle)),
+               "vsa_layout_build")
+        self._h = handle
+        self.info = LayoutInfo()
+        _check(lib().vsa_layout_query(self._h, ctypes.byref(self.info)), "vsa_layout_query")
+        self._dev = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h and _lib is not None:
+            _lib.vsa_layout_free(h)
+            self._h = None
+
+    def tables(self):
+        """Host copies: perm [n_tiles, 64], inv [S], tile_count [n_tiles], tile_kind [n_tiles]."""
+        i = self.info
+        perm = np.empty(i.n_tiles * TILE, dtype=np.int32)
+        inv = np.empty(i.seq_len, dtype=np.int32)
+        cnt = np.empty(i.n_tiles, dtype=np.int32)
+        kind = np.empty(i.n_tiles, dtype=np.int32)
+        _check(lib().vsa_layout_copy_tables(self._h, perm.ctypes.data, inv.ctypes.data, cnt.ctypes.data,
+                                            kind.ctypes.data), "vsa_layout_copy_tables")
+        return perm.reshape(-1, TILE), inv, cnt, kind
+
+    def upload(self, dev_buf, stream=None) -> None:
+        """Uploads the device tables into `dev_buf` (a torch uint8 CUDA tensor
+        of at least info.device_bytes bytes, kept alive by this object)."""
+        _check(lib().vsa_layout_upload(self._h, dev_buf.data_ptr(), dev_buf.numel() * dev_buf.element_size(),
+                                       _stream_handle(stream)), "vsa_layout_upload")
+        self._dev = dev_buf
+
+    def kmax(self, params: Params) -> int:
+        k = _I32()
+        _check(lib().vsa_select_kmax(self._h, ctypes.byref(params), ctypes.byref(k)), "vsa_select_kmax")
+        return k.value
+
+    def coarse_select_workspace_size(self, B: int, H: int, params: Params) -> int:
+        n = _SZ()
+        _check(lib().vsa_coarse_select_workspace_size(self._h, B, H, ctypes.byref(params), ctypes.byref(n)),
+               "vsa_coarse_select_workspace_size")
+        return n.value
+
+    def sparse_attn_workspace_size(self, B: int, H: int, params: Params) -> int:
+        n = _SZ()
+        _check(lib().vsa_sparse_attn_workspace_size(self._h, B, H, ctypes.byref(params), ctypes.byref(n)),
+               "vsa_sparse_attn_workspace_size")
+        return n.value
+
+
+def _qkv_strides(q, k, v):
+    if not (q.stride() == k.stride() == v.stride()):
+        raise ValueError("q, k and v must share strides")
+    if q.dim() != 4 or q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
+        raise ValueError("q, k, v must be [B, S, H, 128] with a contiguous head dim")
+    return q.stride(0), q.stride(1), q.stride(2)
+
+
+def coarse_select(layout: Layout, params: Params, q, k, v, idx, cnt, o_coarse, workspace, stream=None) -> None:
+    """vsa_coarse_select on torch tensors (bf16 q/k/v [B, S, H, 128])."""
+    B, S, H, _ = q.shape
+    sb, ss, sh = _qkv_strides(q, k, v)
+    _check(lib().vsa_coarse_select(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
+                                   v.data_ptr(), sb, ss, sh, idx.data_ptr(), cnt.data_ptr(),
+                                   o_coarse.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _stream_handle(stream)),
+           "vsa_coarse_select")
+
+
+def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: int, o_coarse, out,
+                    workspace, stream=None) -> None:
+    """vsa_sparse_attn_fwd on torch tensors; out is float32 or bfloat16 [B, S, H, 128]."""
+    import torch
+    B, S, H, _ = q.shape
+    sb, ss, sh = _qkv_strides(q, k, v)
+    if out.dtype == torch.float32:
+        od = OUT_F32
+    elif out.dtype == torch.bfloat16:
+        od = OUT_BF16
+    else:
+        raise ValueError("out must be float32 or bfloat16")
+    _check(lib().vsa_sparse_attn_fwd(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
+                                     v.data_ptr(), sb, ss, sh, g.data_ptr(), g.stride(0), g.stride(1),
+                                     g.stride(2), idx.data_ptr(), cnt.data_ptr(), kmax, o_coarse.data_ptr(),
+                                     out.data_ptr(), od, out.stride(0), out.stride(1), out.stride(2),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream)), "vsa_sparse_attn_fwd")
+
+
+def sparse_attn_status(workspace, stream=None) -> int:
+    """Synchronises the stream and returns the kernel's status word (OK or ERR_TIMEOUT)."""
+    return lib().vsa_sparse_attn_status(workspace.data_ptr(), _stream_handle(stream))
+
+
+class Forward:
+    """Holds the buffers of one shape and runs the two calls of the forward
+    pass (caller-owned torch buffers; no allocation inside the calls)."""
+
+    def __init__(self, layout: Layout, params: Params, B: int, H: int, device="cuda",
+                 out_dtype=None, stream=None):
+        import torch
+        self.layout, self.params, self.B, self.H = layout, params, B, H
+        info = layout.info
+        if layout._dev is None:
+            buf = torch.empty(info.device_bytes, dtype=torch.uint8, device=device)
+            layout.upload(buf, stream)
+        self.kmax = layout.kmax(params)
+        self.idx = torch.empty((B, H, info.n_tiles, self.kmax), dtype=torch.int32, device=device)
+        self.cnt = torch.empty((B, H, info.n_tiles), dtype=torch.int32, device=device)
+        self.o_coarse = torch.empty((B, H, info.n_tiles, HEAD_DIM), dtype=torch.float32, device=device)
+        self.ws_select = torch.empty(layout.coarse_select_workspace_size(B, H, params), dtype=torch.uint8,
+                                     device=device)
+        self.ws_attn = torch.empty(layout.sparse_attn_workspace_size(B, H, params), dtype=torch.uint8,
+                                   device=device)
+        self.out_dtype = out_dtype or torch.float32
+        self.stream = stream
+
+    def __call__(self, q, k, v, g, out=None):
+        import torch
+        if out is None:
+            out = torch.empty(q.shape, dtype=self.out_dtype, device=q.device)
+        coarse_select(self.layout, self.params, q, k, v, self.idx, self.cnt, self.o_coarse, self.ws_select,
+                      self.stream)
+        sparse_attn_fwd(self.layout, self.params, q, k, v, g, self.idx, self.cnt, self.kmax, self.o_coarse,
+                        out, self.ws_attn, self.stream)
+        return out
+
+    def pooled(self):
+        """Pooled means [3, B, H, n_tiles, 128] left in the selection workspace."""
+        import torch
+        n = 3 * self.B * self.H * self.layout.info.n_tiles * HEAD_DIM
+        return self.ws_select[: 4 * n].view(torch.float32).view(3, self.B, self.H, self.layout.info.n_tiles,
+                                                                HEAD_DIM)

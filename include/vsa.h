@@ -1,0 +1,261 @@
+/*
+ * vsa.h - C ABI of libvsa: VSA-style block-sparse video attention, forward
+ * pass, for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are web pages, cited by title and section):
+ *  - A packed sequence [conditioning prefix | generated video] is split into
+ *    64-token tiles: conditioning segments (text, reference image, reference
+ *    audio) into segment-pure runs, the video latent grid into 4x4x4 cubes.
+ *    ("Ref2VA VSA : noeud d'attention sparse pour le Ref2VA H3", section
+ *    "Le correctif d'attention a deux niveaux"; "ComfyUI-Ref2VA-VSA",
+ *    "Technical Architecture" and "The Solution: Ref2VAVSAGatePatch".)
+ *  - A coarse branch mean-pools Q/K/V per tile, scores query tiles against
+ *    video key tiles and selects, per query tile, the video key tiles to attend
+ *    exactly (fixed keep fraction or per-head adaptive threshold).
+ *    ("BSAI FastH3 Native VSA (recipe)", "The mechanism, briefly" and "The
+ *    inputs that matter"; "ComfyUI Agrega Nodo Central de Atencion Dispersa y
+ *    Compilador Comfy", section "Atencion dispersa por bloques", Sol-Attn,
+ *    top-k and VSA bullets.)
+ *  - A fine branch attends each query tile exactly to every conditioning key
+ *    token plus its selected video tiles; the output is o_fine + g * o_coarse.
+ *
+ * Conventions for every call:
+ *  - The caller owns all device memory. The library never allocates device
+ *    memory, never synchronises a stream (except vsa_sparse_attn_status, which
+ *    exists to do exactly that) and enqueues all GPU work on the given stream.
+ *  - Tensors are bf16 with head_dim 128, addressed by element strides for the
+ *    batch, sequence and head dimensions; the head_dim is contiguous.
+ *  - Errors are returned, never raised or aborted. VSA_ERR_UNSUPPORTED means
+ *    "this library does not run this case; the caller should run dense
+ *    attention" (the pages' rule that every ambiguous case runs dense, "BSAI
+ *    FastH3 Native VSA (recipe)", "The mechanism, briefly").
+ *  - On an error no GPU work has been enqueued, except where VSA_ERR_CUDA
+ *    reports a failed launch.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VSA_TILE 64
+#define VSA_HEAD_DIM 128
+#define VSA_MAX_SEGMENTS 64
+
+typedef enum {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1,          /* malformed argument: null pointer, bad size, bad descriptor */
+  VSA_ERR_UNSUPPORTED = 2,          /* valid request this library does not run: caller runs dense */
+  VSA_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes below the size query's answer */
+  VSA_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
+  VSA_ERR_TIMEOUT = 5,              /* a kernel gave up waiting (reported by vsa_sparse_attn_status) */
+  VSA_ERR_NOT_UPLOADED = 6          /* the layout has no device tables (see vsa_layout_upload) */
+} vsa_status;
+
+/* Segment kinds of the packed sequence. Every kind except VIDEO is
+ * conditioning: never pruned as keys. */
+typedef enum {
+  VSA_SEG_TEXT = 0,
+  VSA_SEG_REF_IMAGE = 1,
+  VSA_SEG_REF_AUDIO = 2,
+  VSA_SEG_OTHER_COND = 3,
+  VSA_SEG_VIDEO = 4
+} vsa_seg_kind;
+
+/* One segment of the packed-sequence descriptor: tokens [start, start+length).
+ * For VSA_SEG_VIDEO, grid_t * grid_h * grid_w == length and the tokens are the
+ * latent grid in raster order (t slowest, w fastest); other kinds ignore the
+ * grid fields. */
+typedef struct {
+  int32_t kind;
+  int32_t grid_t, grid_h, grid_w;
+  int64_t start;
+  int64_t length;
+} vsa_segment;
+
+typedef enum { VSA_SELECT_TOPK = 0, VSA_SELECT_ADAPTIVE = 1 } vsa_select_mode;
+
+/* sink_conditioning ("BSAI FastH3 Native VSA (recipe)", "The inputs that
+ * matter"): EXACT_KV = every query attends every conditioning key exactly;
+ * EXACT_KV_AND_ROWS = in addition, conditioning query rows attend the whole
+ * sequence densely (and get no coarse term). */
+typedef enum { VSA_SINK_EXACT_KV = 0, VSA_SINK_EXACT_KV_AND_ROWS = 1 } vsa_sink_mode;
+
+typedef enum { VSA_OUT_F32 = 0, VSA_OUT_BF16 = 1 } vsa_out_dtype;
+
+/* Selection parameters.
+ *  mode  : VSA_SELECT_TOPK keeps k = max(1, ceil(keep * Nv)) video key tiles
+ *          per query tile (Nv = number of video tiles; the product is taken in
+ *          double with a relative guard of 2^-20); ties go to the lower tile.
+ *          VSA_SELECT_ADAPTIVE keeps the video key tiles whose score is
+ *          >= mean + tau * std of that (batch, head)'s whole score matrix
+ *          (population std), and at least the row's argmax.
+ *  keep  : (0, 1], used by TOPK.
+ *  tau   : >= 0, used by ADAPTIVE.
+ *  sink  : vsa_sink_mode.
+ *  scale : softmax scale of both branches; <= 0 selects 1/sqrt(128). */
+typedef struct {
+  int32_t mode;
+  float keep;
+  float tau;
+  int32_t sink;
+  float scale;
+} vsa_params;
+
+typedef struct vsa_layout vsa_layout;   /* opaque; owns its host tables */
+
+typedef struct {
+  int64_t seq_len;
+  int32_t n_cond_tiles;      /* conditioning tiles: tile ids [0, n_cond_tiles) */
+  int32_t n_video_tiles;     /* video tiles: tile ids [n_cond_tiles, n_tiles) */
+  int32_t n_tiles;
+  int32_t grid_t, grid_h, grid_w;
+  int64_t video_start;       /* first token of the video segment */
+  size_t device_bytes;       /* bytes vsa_layout_upload needs */
+} vsa_layout_info;
+
+/* ------------------------------------------------------------------------ */
+/* Geometry map (token -> tile permutation)                                  */
+/* ------------------------------------------------------------------------ */
+
+/* vsa_layout_build: builds the geometry map of a packed sequence on the host
+ * ("Le correctif d'attention a deux niveaux", item 1: segment-pure tiles; 4x4x4
+ * video cubes, "ComfyUI-Ref2VA-VSA", "Technical Architecture").
+ *
+ *  segs, n_segs : descriptor, segments in sequence order covering
+ *                 [0, seq_len) contiguously, 1 <= n_segs <= VSA_MAX_SEGMENTS,
+ *                 exactly one VSA_SEG_VIDEO segment. Conditioning segments may
+ *                 come before or after the video.
+ *  dev_buf      : optional device buffer of at least info.device_bytes bytes;
+ *                 when non-NULL the device tables are uploaded into it on
+ *                 `stream` (as vsa_layout_upload does). NULL builds the host
+ *                 tables only.
+ *  out          : receives the handle; free it with vsa_layout_free. The
+ *                 caller keeps dev_buf alive while the handle is used.
+ * Tile ids: conditioning tiles first (64-token runs of each conditioning
+ * segment in descriptor order, the last run of a segment possibly partial),
+ * then the video cubes in raster order over (t/4, h/4, w/4); slots of a cube
+ * are raster order over (t, h, w), slots outside the grid are padding.
+ * Errors: INVALID_ARG for a malformed descriptor; UNSUPPORTED when there is
+ * no video segment, more than one, or seq_len >= 2^31 tokens. */
+vsa_status vsa_layout_build(const vsa_segment* segs, int32_t n_segs, int64_t seq_len,
+                            void* dev_buf, size_t dev_bytes, cudaStream_t stream,
+                            vsa_layout** out);
+
+/* Copies the device tables into dev_buf (>= info.device_bytes, 256-byte
+ * aligned) with cudaMemcpyAsync on `stream`, and records dev_buf in the
+ * handle. The source is pageable host memory: the call returns once the host
+ * tables are staged, so the handle may be freed right after; it is a set-up
+ * step and must not be issued while `stream` is being captured. */
+vsa_status vsa_layout_upload(vsa_layout* layout, void* dev_buf, size_t dev_bytes,
+                             cudaStream_t stream);
+
+vsa_status vsa_layout_query(const vsa_layout* layout, vsa_layout_info* info);
+
+/* Host copies of the tables, any pointer may be NULL:
+ *  perm       int32 [n_tiles * 64] : token of (tile, slot), -1 for padding
+ *  inv        int32 [seq_len]      : tile * 64 + slot of each token
+ *  tile_count int32 [n_tiles]      : valid tokens of each tile
+ *  tile_kind  int32 [n_tiles]      : vsa_seg_kind of each tile */
+vsa_status vsa_layout_copy_tables(const vsa_layout* layout, int32_t* perm, int32_t* inv,
+                                  int32_t* tile_count, int32_t* tile_kind);
+
+void vsa_layout_free(vsa_layout* layout);
+
+/* ------------------------------------------------------------------------ */
+/* Coarse branch + selection                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* kmax: the row length of the index list (k for TOPK, Nv for ADAPTIVE). */
+vsa_status vsa_select_kmax(const vsa_layout* layout, const vsa_params* params, int32_t* kmax);
+
+vsa_status vsa_coarse_select_workspace_size(const vsa_layout* layout, int32_t B, int32_t H,
+                                            const vsa_params* params, size_t* bytes);
+
+/* vsa_coarse_select: the coarse branch and the block selection
+ * ("BSAI FastH3 Native VSA (recipe)", "The mechanism, briefly": scores the
+ * blocks and keeps the top slice; "ComfyUI Agrega Nodo Central ...", VSA
+ * bullet: coarse compression branch; Sol-Attn bullet: adaptive threshold).
+ *
+ *  q, k, v        : bf16 [B, S, H, 128] at element strides (stride_b,
+ *                   stride_s, stride_h); 16-byte aligned, strides multiples
+ *                   of 8.
+ *  idx            : int32 [B, H, n_tiles, kmax] out: per query tile the
+ *                   selected video tiles as video ordinals in [0, Nv),
+ *                   ascending; entries past cnt are left unspecified.
+ *  cnt            : int32 [B, H, n_tiles] out: list lengths.
+ *  o_coarse       : float [B, H, n_tiles, 128] out:
+ *                   sum_v softmax_v(s[qt, v]) * mean(V of video tile v), with
+ *                   s[qt, v] = scale * <mean Q of tile qt, mean K of video tile v>.
+ *  workspace      : device scratch of vsa_coarse_select_workspace_size bytes,
+ *                   256-byte aligned. Its first 3*B*H*n_tiles*128 floats hold
+ *                   the pooled means [3 (q,k,v), B, H, n_tiles, 128] after
+ *                   the call.
+ * All query tiles are processed, conditioning tiles included (under
+ * EXACT_KV_AND_ROWS their lists are ignored by vsa_sparse_attn_fwd).
+ * Pooling, scores, thresholds and the coarse softmax are fp32 (adaptive
+ * mean/std accumulate in fp64). */
+vsa_status vsa_coarse_select(const vsa_layout* layout, const vsa_params* params,
+                             int32_t B, int32_t H,
+                             const void* q, const void* k, const void* v,
+                             int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                             int32_t* idx, int32_t* cnt, float* o_coarse,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Fine branch + gate combine                                                */
+/* ------------------------------------------------------------------------ */
+
+vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* layout, int32_t B, int32_t H,
+                                          const vsa_params* params, size_t* bytes);
+
+/* vsa_sparse_attn_fwd: exact attention of every query tile over all
+ * conditioning key tokens plus the video tiles of its list (EXACT_KV), or over
+ * the whole sequence for conditioning query tiles (EXACT_KV_AND_ROWS), then
+ * out = o_fine + g * o_coarse[tile] (no coarse term on dense conditioning rows).
+ * ("BSAI FastH3 Native VSA (recipe)", "The inputs that matter",
+ * sink_conditioning; "ComfyUI-Ref2VA-VSA", "Video-Only Sparse Attention".)
+ *
+ *  q, k, v, strides : as for vsa_coarse_select.
+ *  g                : bf16 [B, S, H] gate at element strides (g_stride_*).
+ *  idx, cnt, kmax   : lists from vsa_coarse_select (same params).
+ *  o_coarse         : float [B, H, n_tiles, 128] from vsa_coarse_select.
+ *  out              : [B, S, H, 128] of out_dtype (vsa_out_dtype) at element
+ *                     strides out_stride_*, head_dim contiguous; every valid
+ *                     token row is written.
+ *  workspace        : vsa_sparse_attn_workspace_size bytes, 256-byte aligned.
+ * Softmax statistics and accumulation are fp32; the probabilities enter the
+ * second tensor-core product as bf16. A kernel wait that runs out is recorded
+ * in the workspace and reported by vsa_sparse_attn_status. */
+vsa_status vsa_sparse_attn_fwd(const vsa_layout* layout, const vsa_params* params,
+                               int32_t B, int32_t H,
+                               const void* q, const void* k, const void* v,
+                               int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                               const void* g, int64_t g_stride_b, int64_t g_stride_s,
+                               int64_t g_stride_h,
+                               const int32_t* idx, const int32_t* cnt, int32_t kmax,
+                               const float* o_coarse,
+                               void* out, int32_t out_dtype, int64_t out_stride_b,
+                               int64_t out_stride_s, int64_t out_stride_h,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream` and reads the error word a previous
+ * vsa_sparse_attn_fwd left in `workspace`: VSA_OK, VSA_ERR_TIMEOUT (a bounded
+ * wait in the kernel ran out; the output is incomplete) or VSA_ERR_CUDA. */
+vsa_status vsa_sparse_attn_status(const void* workspace, cudaStream_t stream);
+
+const char* vsa_status_string(vsa_status status);
+
+/* Library ABI version, (major << 16) | minor. */
+int32_t vsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

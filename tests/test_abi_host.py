@@ -1,0 +1,149 @@
+"""Host-side tests of libvsa (no GPU needed): the library loads and exports
+every function include/vsa.h declares; the C++ geometry map equals the
+oracle's bit for bit; k rounding matches; malformed arguments are rejected
+with a status before any GPU work."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_video_geometry_b200 import vsa, workloads as W
+from oracle import vsa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if hdr.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", hdr)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(vsa_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert "vsa_layout_build" in names and "vsa_coarse_select" in names and "vsa_sparse_attn_fwd" in names
+    L = vsa.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert vsa.version() >> 16 == 1
+    assert vsa.status_string(vsa.ERR_UNSUPPORTED).startswith("unsupported")
+
+
+def _segments(cond, grid, after=()):
+    segs, pos = [], 0
+    for kind, n in cond:
+        segs.append((kind, pos, n, None))
+        pos += n
+    nv = grid[0] * grid[1] * grid[2]
+    segs.append((vsa.SEG_VIDEO, pos, nv, grid))
+    pos += nv
+    for kind, n in after:
+        segs.append((kind, pos, n, None))
+        pos += n
+    return segs, pos
+
+
+CASES = [
+    (((0, 32), (1, 16), (2, 16)), (8, 8, 8), ()),
+    (((0, 512), (1, 448), (2, 64)), (16, 32, 32), ()),
+    (((0, 70),), (5, 6, 7), ()),
+    ((), (3, 1, 9), ()),
+    (((0, 1), (1, 64), (2, 65)), (1, 1, 1), ()),
+    (((0, 5),), (9, 4, 13), ((2, 100),)),           # conditioning after the video
+    (((0, 512), (1, 4032), (2, 128)), (61, 48, 84), ()),
+]
+
+
+@pytest.mark.parametrize("cond,grid,after", CASES)
+def test_layout_matches_oracle_bit_exact(cond, grid, after):
+    segs, S = _segments(cond, grid, after)
+    lay = vsa.Layout(segs, S)
+    ref = O.build_layout([O.Segment(k, s, n, g) for (k, s, n, g) in segs], S)
+    perm, inv, cnt, kind = lay.tables()
+    assert lay.info.n_cond_tiles == ref.n_cond_tiles
+    assert lay.info.n_video_tiles == ref.n_video_tiles
+    assert np.array_equal(perm, ref.perm)
+    assert np.array_equal(inv, ref.inv)
+    assert np.array_equal(cnt, (ref.perm >= 0).sum(1))
+    assert np.array_equal(kind, ref.tile_kind)
+    assert lay.info.device_bytes >= perm.nbytes + inv.nbytes
+
+
+def test_topk_count_matches_oracle():
+    segs, S = _segments(((0, 64),), (8, 8, 8))
+    rng = np.random.default_rng(0)
+    for nv_grid in [(8, 8, 8), (16, 32, 32), (32, 48, 84), (61, 48, 84), (7, 5, 3)]:
+        segs, S = _segments(((0, 64),), nv_grid)
+        lay = vsa.Layout(segs, S)
+        nv = lay.info.n_video_tiles
+        for keep in list(rng.uniform(0, 1, 40)) + [0.1, 0.2, 0.5, 1.0, 1e-7, 0.25]:
+            keep = float(np.float32(keep))
+            if keep <= 0:
+                continue
+            p = vsa.make_params(keep=keep)
+            assert lay.kmax(p) == O.topk_count(keep, nv), (keep, nv)
+        assert lay.kmax(vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=1.0)) == nv
+
+
+@pytest.mark.parametrize("segs,S,status", [
+    ([(0, 0, 10, None)], 10, vsa.ERR_UNSUPPORTED),                                   # no video
+    ([(4, 0, 8, (2, 2, 2)), (4, 8, 8, (2, 2, 2))], 16, vsa.ERR_UNSUPPORTED),          # two videos
+    ([(0, 0, 4, None), (4, 5, 8, (2, 2, 2))], 13, vsa.ERR_INVALID_ARG),               # gap
+    ([(4, 0, 9, (2, 2, 2))], 9, vsa.ERR_INVALID_ARG),                                 # grid mismatch
+    ([(0, 0, 4, None), (4, 4, 8, (2, 2, 2))], 20, vsa.ERR_INVALID_ARG),               # not covering
+    ([(7, 0, 4, None), (4, 4, 8, (2, 2, 2))], 12, vsa.ERR_INVALID_ARG),               # bad kind
+    ([(0, 0, 0, None), (4, 0, 8, (2, 2, 2))], 8, vsa.ERR_INVALID_ARG),                # empty segment
+])
+def test_layout_rejects_bad_descriptors(segs, S, status):
+    with pytest.raises(vsa.VSAError) as e:
+        vsa.Layout(segs, S)
+    assert e.value.status == status
+
+
+def test_calls_validate_before_any_gpu_work():
+    segs, S = _segments(((0, 64),), (8, 8, 8))
+    lay = vsa.Layout(segs, S)
+    L = vsa.lib()
+    good = vsa.make_params(keep=0.5)
+    n = ctypes.c_size_t()
+    for bad in [vsa.make_params(keep=0.0), vsa.make_params(keep=1.5), vsa.make_params(mode=3),
+                vsa.make_params(sink=5), vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=-1.0),
+                vsa.make_params(scale=float("nan"))]:
+        assert L.vsa_coarse_select_workspace_size(lay.handle, 1, 2, ctypes.byref(bad), ctypes.byref(n)) == \
+            vsa.ERR_INVALID_ARG
+    assert L.vsa_coarse_select_workspace_size(lay.handle, 1, 2, ctypes.byref(good), ctypes.byref(n)) == vsa.OK
+    assert n.value > 0
+    fake = 1 << 20   # aligned non-null fake pointer: validation must stop before it is touched
+    args = dict(q=fake, k=fake, v=fake, sb=S * 2 * 128, ss=2 * 128, sh=128)
+    # layout not uploaded
+    st = L.vsa_coarse_select(lay.handle, ctypes.byref(good), 1, 2, args["q"], args["k"], args["v"], args["sb"],
+                             args["ss"], args["sh"], fake, fake, fake, fake, n.value, None)
+    assert st == vsa.ERR_NOT_UPLOADED
+    # misaligned q, bad strides, null outputs, small workspace
+    assert L.vsa_coarse_select(lay.handle, ctypes.byref(good), 1, 2, fake + 2, fake, fake, args["sb"], args["ss"],
+                               args["sh"], fake, fake, fake, fake, n.value, None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_coarse_select(lay.handle, ctypes.byref(good), 1, 2, fake, fake, fake, args["sb"], 3,
+                               args["sh"], fake, fake, fake, fake, n.value, None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_coarse_select(lay.handle, ctypes.byref(good), 1, 2, fake, fake, fake, args["sb"], args["ss"],
+                               args["sh"], None, fake, fake, fake, n.value, None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_coarse_select(lay.handle, ctypes.byref(good), 0, 2, fake, fake, fake, args["sb"], args["ss"],
+                               args["sh"], fake, fake, fake, fake, n.value, None) == vsa.ERR_INVALID_ARG
+    kmax = lay.kmax(good)
+    common = (lay.handle, ctypes.byref(good), 1, 2, fake, fake, fake, args["sb"], args["ss"], args["sh"],
+              fake, 2, 2 * S, 2)
+    # wrong kmax, bad out dtype, unaligned out stride, not uploaded
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, 7, S * 256, 256, 128, fake, 256,
+                                 None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_BF16, S * 256, 256, 129, fake,
+                                 256, None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
+                                 16, None) == vsa.ERR_WORKSPACE_TOO_SMALL
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
+                                 256, None) == vsa.ERR_NOT_UPLOADED

@@ -1,0 +1,157 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs. Tolerances are defined in vsa_cases."""
+
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+from block_sparse_video_geometry_b200 import vsa, workloads as W
+from oracle import vsa_oracle as O
+
+import vsa_cases as C
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+# --------------------------------------------- tcgen05 building blocks ----
+def test_tcgen05_building_blocks(cuda_ok):
+    """One S = Q K^T (3-D and 5-D TMA maps), one O = P V (swizzled P, MN-major V)."""
+    import torch
+    lib = ctypes.CDLL(os.path.join(ROOT, "tests", "native", "libmma_check.so"))
+    lib.mma_check_run.restype = ctypes.c_int
+    g = torch.Generator().manual_seed(0)
+    r = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16).cuda()
+    q, k, v, p = r(128, 128), r(64, 128), r(64, 128), r(128, 64)
+    T, Hg, Wd = 6, 5, 9
+    grid = r(T, Hg, Wd, 2, 128)
+    s1, s2, o = (torch.zeros(128, n, device="cuda") for n in (64, 64, 128))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0, h0, w0, head = 4, 4, 8, 1           # a cube cut by all three grid edges
+    rc = lib.mma_check_run(*(ctypes.c_void_p(x.data_ptr()) for x in (q, k, v, p, grid)),
+                           T, Hg, Wd, t0, h0, w0, head,
+                           *(ctypes.c_void_p(x.data_ptr()) for x in (s1, s2, o, err)))
+    assert rc == 0
+    f = lambda x: x.float().cpu()
+    assert torch.allclose(f(s1), f(q) @ f(k).T, atol=1e-2, rtol=1e-3)
+    cube = torch.zeros(4, 4, 4, 128)
+    gc = f(grid)[t0:t0 + 4, h0:h0 + 4, w0:w0 + 4, head]
+    cube[: gc.shape[0], : gc.shape[1], : gc.shape[2]] = gc
+    assert torch.allclose(f(s2), f(q) @ cube.reshape(64, 128).T, atol=1e-2, rtol=1e-3)
+    assert torch.allclose(f(o), f(p) @ f(v), atol=1e-2, rtol=1e-3)
+
+
+# --------------------------------------------------------- full checks ----
+def full_check(wl, out_dtype="f32", heads=None, out_tiles=None, **prm_over):
+    lay = C.oracle_layout(wl)
+    bits = C.inputs(wl, lay)
+    prm = C.params_of(wl, **prm_over)
+    res = C.gpu_forward(wl, bits, prm, out_dtype)
+    assert res["status"] == vsa.OK
+    C.check_lists_valid(res, lay)
+    worst = 0.0
+    for b in range(wl.B):
+        for h in (range(wl.H) if heads is None else heads):
+            ho = C.HeadOracle(wl, lay, bits, b, h, prm)
+            for t, x in enumerate((ho.qbar, ho.kbar, ho.vbar)):
+                assert np.abs(res["pooled"][t, b, h] - x).max() <= 1e-4
+            assert np.abs(res["o_coarse"][b, h] - ho.o_coarse).max() <= 1e-3
+            excl = C.compare_selection(ho, res["idx"][b, h], res["cnt"][b, h])
+            assert len(excl) <= max(2, lay.n_tiles // 20)
+            tiles = range(lay.n_tiles) if out_tiles is None else out_tiles(lay)
+            tiles = [t for t in tiles if t not in excl]
+            mx, _ = C.compare_outputs(ho, res, b, h, tiles, bf16=(out_dtype == "bf16"))
+            worst = max(worst, mx)
+    return res, worst
+
+
+def test_tiny_full(cuda_ok):
+    full_check(W.WORKLOADS["tiny"])
+
+
+def test_tiny_bf16_output(cuda_ok):
+    full_check(W.WORKLOADS["tiny"], out_dtype="bf16")
+
+
+@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS])
+@pytest.mark.parametrize("keep", [0.125, 0.5, 1.0])
+def test_tiny_keep_and_sink(cuda_ok, keep, sink):
+    full_check(W.WORKLOADS["tiny"], keep=keep, sink=sink)
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0, 1.5, 2.0])
+def test_tiny_adaptive(cuda_ok, tau):
+    full_check(W.WORKLOADS["tiny"].with_(mode=O.MODE_ADAPTIVE, tau=tau))
+
+
+EDGE_WORKLOADS = [
+    # ragged in every dimension, two batches, one conditioning segment
+    W.Workload("ragged_b2", B=2, H=3, cond=((W.SEG_TEXT, 70),), grid=(5, 6, 7), keep=0.3, seed=11),
+    # no conditioning prefix at all
+    W.Workload("video_only", B=1, H=2, cond=(), grid=(8, 8, 12), keep=0.25, seed=12),
+    # conditioning after the video, odd number of tiles, thin grid
+    W.Workload("cond_after", B=1, H=2, cond=((W.SEG_TEXT, 5),), grid=(9, 4, 13), keep=0.2, seed=13,
+               cond_after=((W.SEG_REF_AUDIO, 100),)),
+    # one video tile only, partial
+    W.Workload("one_tile", B=1, H=1, cond=((W.SEG_TEXT, 1), (W.SEG_REF_IMAGE, 64), (W.SEG_REF_AUDIO, 65)),
+               grid=(1, 1, 1), keep=1.0, seed=14),
+    # single-frame, single-row grid
+    W.Workload("thin", B=1, H=2, cond=((W.SEG_TEXT, 40),), grid=(3, 1, 9), keep=0.5, seed=15),
+]
+
+
+@pytest.mark.parametrize("wl", EDGE_WORKLOADS, ids=lambda w: w.name)
+@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS])
+def test_edge_layouts(cuda_ok, wl, sink):
+    full_check(wl, sink=sink)
+
+
+def test_k_equals_one(cuda_ok):
+    full_check(W.WORKLOADS["tiny"], keep=1e-6)
+
+
+def test_gate_zero_gives_fine_branch_and_keep_all_gives_dense(cuda_ok):
+    """keep=100% and g=0: the output is plain dense softmax attention."""
+    wl = W.WORKLOADS["tiny"]
+    lay = C.oracle_layout(wl)
+    q, k, v, g = C.inputs(wl, lay)
+    g0 = np.zeros_like(g)
+    res = C.gpu_forward(wl, (q, k, v, g0), C.params_of(wl, keep=1.0))
+    f = O.bf16_bits_to_f64
+    for h in range(wl.H):
+        dense = O.softmax_attention(f(q[0, :, h]), f(k[0, :, h]), f(v[0, :, h]), O.default_scale())
+        err = np.abs(res["out"][0, :, h] - dense)
+        assert err.max() <= C.OUT_MAX_ABS and err.mean() <= C.OUT_MEAN_ABS
+
+
+def test_deterministic_rerun(cuda_ok):
+    wl = W.WORKLOADS["tiny"]
+    lay = C.oracle_layout(wl)
+    bits = C.inputs(wl, lay)
+    a = C.gpu_forward(wl, bits, C.params_of(wl))
+    b = C.gpu_forward(wl, bits, C.params_of(wl))
+    for key in ("idx", "cnt", "o_coarse", "out"):
+        if key == "idx":
+            for x, y, n in zip(a["idx"].reshape(-1, a["kmax"]), b["idx"].reshape(-1, b["kmax"]), a["cnt"].ravel()):
+                assert np.array_equal(x[:n], y[:n])
+        else:
+            assert np.array_equal(a[key], b[key])
+
+
+def test_mid_all_heads_selection_two_heads_outputs(cuda_ok):
+    wl = W.WORKLOADS["mid"]
+    lay = C.oracle_layout(wl)
+    bits = C.inputs(wl, lay)
+    prm = C.params_of(wl)
+    res = C.gpu_forward(wl, bits, prm)
+    C.check_lists_valid(res, lay)
+    rng = np.random.default_rng(0)
+    for h in range(wl.H):
+        ho = C.HeadOracle(wl, lay, bits, 0, h, prm)
+        excl = C.compare_selection(ho, res["idx"][0, h], res["cnt"][0, h])
+        assert np.abs(res["o_coarse"][0, h] - ho.o_coarse).max() <= 1e-3
+        tiles = range(lay.n_tiles) if h in (0, 17) else rng.choice(lay.n_tiles, 6, replace=False)
+        C.compare_outputs(ho, res, 0, h, [t for t in tiles if t not in excl])

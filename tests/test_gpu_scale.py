@@ -1,0 +1,83 @@
+"""GPU parity at the full 1344x768 shapes, in the launch configuration the
+benchmark times (fp32 output, one call of each entry point). The oracle checks
+whole selection matrices of sampled heads and the outputs of sampled query
+tiles (conditioning tiles, first/last video tiles, ragged tiles, random ones)."""
+
+import numpy as np
+import pytest
+
+from block_sparse_video_geometry_b200 import vsa, workloads as W
+from oracle import vsa_oracle as O
+
+import vsa_cases as C
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_tiles(lay, rng, n_random=6):
+    nc, nt = lay.n_cond_tiles, lay.n_tiles
+    fixed = {0, nc - 1, nc, nc + 1, nt - 2, nt - 1} if nc else {0, 1, nt - 2, nt - 1}
+    partial = [t for t in range(nc, nt) if (lay.perm[t] >= 0).sum() < O.TILE]
+    if partial:
+        fixed |= {partial[0], partial[-1]}
+    return sorted(fixed | set(rng.choice(nt, n_random, replace=False).tolist()))
+
+
+def run_case(wl, heads, n_random=6, g_zero=False, **prm_over):
+    lay = C.oracle_layout(wl)
+    q, k, v, g = C.inputs(wl, lay)
+    if g_zero:
+        g = np.zeros_like(g)
+    prm = C.params_of(wl, **prm_over)
+    res = C.gpu_forward(wl, (q, k, v, g), prm)
+    assert res["status"] == vsa.OK
+    rng = np.random.default_rng(1234)
+    kept = []
+    for h in heads:
+        ho = C.HeadOracle(wl, lay, (q, k, v, g), 0, h, prm)
+        assert np.abs(res["pooled"][1, 0, h] - ho.kbar).max() <= 1e-4
+        assert np.abs(res["o_coarse"][0, h] - ho.o_coarse).max() <= 1e-3
+        excl = C.compare_selection(ho, res["idx"][0, h], res["cnt"][0, h])
+        assert len(excl) <= lay.n_tiles // 20
+        tiles = [t for t in sample_tiles(lay, rng, n_random) if t not in excl]
+        C.compare_outputs(ho, res, 0, h, tiles)
+        kept.append(res["cnt"][0, h].mean() / lay.n_video_tiles)
+    # every list is valid on every head
+    cnt = res["cnt"]
+    assert cnt.min() >= 1 and cnt.max() <= res["kmax"]
+    return lay, res, kept
+
+
+def test_5s_topk_10pct(cuda_ok):
+    lay, res, kept = run_case(W.WORKLOADS["5s"], heads=(0, 11, 23))
+    assert lay.n_video_tiles == 2016 and res["kmax"] == 202
+
+
+def test_10s_ragged_rows_dense(cuda_ok):
+    lay, res, kept = run_case(W.WORKLOADS["10s"], heads=(0, 23), n_random=4)
+    assert lay.n_video_tiles == 4032 and res["kmax"] == 404
+
+
+@pytest.mark.parametrize("tau", [1.0, 1.5, 2.0])
+def test_5s_adaptive_tau(cuda_ok, tau):
+    lay, res, kept = run_case(W.WORKLOADS["5s_adaptive"].with_(tau=tau), heads=(0, 13), n_random=4)
+    # kept fraction near the Gaussian tail above mean + tau * std
+    import math
+    tail = 0.5 * math.erfc(tau / math.sqrt(2))
+    assert abs(float(np.mean(kept)) - tail) < 0.05
+
+
+def test_5s_keep_all_equals_dense(cuda_ok):
+    wl = W.WORKLOADS["5s"].with_(keep=1.0)
+    lay = C.oracle_layout(wl)
+    q, k, v, g = C.inputs(wl, lay)
+    res = C.gpu_forward(wl, (q, k, v, np.zeros_like(g)), C.params_of(wl, keep=1.0))
+    f = O.bf16_bits_to_f64
+    rng = np.random.default_rng(7)
+    for h in (0, 19):
+        kk, vv = f(k[0, :, h]), f(v[0, :, h])
+        for qt in rng.choice(lay.n_tiles, 3, replace=False):
+            toks = lay.tile_tokens(int(qt))
+            dense = O.softmax_attention(f(q[0, toks, h]), kk, vv, O.default_scale())
+            err = np.abs(res["out"][0, toks, h] - dense)
+            assert err.max() <= C.OUT_MAX_ABS and err.mean() <= C.OUT_MEAN_ABS

@@ -1,0 +1,139 @@
+"""Shared helpers of the parity tests: seeded inputs, one GPU forward through
+the C ABI, the oracle on chosen (batch, head, query tile) samples, and the
+comparison rules.
+
+Tolerances (stated here once, used by every parity test):
+* layout and selected tile indices: bit-exact, except rows whose oracle
+  scores have a near-tie (gap < 1e-4) at the selection boundary; in such a
+  row the two sets may differ only by tiles within 1e-4 of the boundary, and
+  the row's outputs are left out of the comparison;
+* fp32 output: max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle;
+* bf16 output: the same bounds plus the bf16 rounding of the output itself
+  (half an ulp of the reference value per element, a quarter ulp on average);
+* o_coarse (fp32 path vs fp64): max-abs <= 1e-3; pooled means: max-abs <= 1e-4.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from block_sparse_video_geometry_b200 import workloads as W
+from oracle import vsa_oracle as O
+
+GAP = 1e-4
+OUT_MAX_ABS, OUT_MEAN_ABS = 2e-2, 2e-3
+
+
+def oracle_layout(wl):
+    return O.build_layout([O.Segment(k, s, n, g) for (k, s, n, g) in wl.segments()], wl.seq_len)
+
+
+def inputs(wl, lay):
+    return W.make_inputs(wl, lay.inv // O.TILE)
+
+
+def params_of(wl, **kw):
+    d = dict(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink)
+    d.update(kw)
+    return d
+
+
+def gpu_forward(wl, bits, prm: dict, out_dtype="f32", layout=None):
+    """Runs vsa_coarse_select + vsa_sparse_attn_fwd on cuda:0; returns numpy arrays."""
+    import torch
+    from block_sparse_video_geometry_b200 import vsa
+    q, k, v, g = bits
+    dev = torch.device("cuda:0")
+    t = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    tq, tk, tv, tg = t(q), t(k), t(v), t(g)
+    lay = layout or vsa.Layout(wl.segments(), wl.seq_len)
+    p = vsa.make_params(**prm)
+    fwd = vsa.Forward(lay, p, wl.B, wl.H, device=dev,
+                      out_dtype=torch.float32 if out_dtype == "f32" else torch.bfloat16)
+    out = fwd(tq, tk, tv, tg)
+    st = vsa.sparse_attn_status(fwd.ws_attn)
+    torch.cuda.synchronize()
+    res = dict(status=st, idx=fwd.idx.cpu().numpy(), cnt=fwd.cnt.cpu().numpy(),
+               o_coarse=fwd.o_coarse.cpu().numpy(), pooled=fwd.pooled().cpu().numpy(),
+               out=out.float().cpu().numpy(), kmax=fwd.kmax)
+    del fwd, tq, tk, tv, tg, out
+    torch.cuda.empty_cache()
+    return res
+
+
+class HeadOracle:
+    """Oracle state of one (batch, head): pooled means, scores, lists, coarse."""
+
+    def __init__(self, wl, lay, bits, b, h, prm: dict):
+        f = O.bf16_bits_to_f64
+        q, k, v, g = bits
+        self.q, self.k, self.v = f(q[b, :, h]), f(k[b, :, h]), f(v[b, :, h])
+        self.g = f(g[b, :, h])
+        self.lay = lay
+        self.p = O.Params(mode=prm["mode"], keep=prm["keep"], tau=prm["tau"], sink=prm["sink"])
+        (self.qbar, self.kbar, self.vbar, self.scores, self.sel, self.thr, self.o_coarse,
+         self.scale) = O.selection_for_head(self.q, self.k, self.v, lay, self.p)
+
+    def tile_out(self, qt):
+        return O.output_rows_for_tile(self.q, self.k, self.v, self.g, self.lay, self.p, qt,
+                                      self.sel[qt], self.o_coarse, self.scale)
+
+
+def check_lists_valid(res, lay):
+    """Every list is ascending, in range and as long as cnt says."""
+    idx, cnt = res["idx"], res["cnt"]
+    nv = lay.n_video_tiles
+    assert cnt.min() >= 1 and cnt.max() <= res["kmax"]
+    B, H, Nt, _ = idx.shape
+    for b in range(B):
+        for h in range(H):
+            for qt in range(Nt):
+                row = idx[b, h, qt, : cnt[b, h, qt]]
+                assert row.min() >= 0 and row.max() < nv
+                assert np.all(np.diff(row) > 0)
+
+
+def compare_selection(ho: HeadOracle, gpu_idx, gpu_cnt):
+    """Returns the set of query tiles left out for a near-tie; asserts the rest."""
+    excluded = set()
+    for qt, want in enumerate(ho.sel):
+        got = gpu_idx[qt, : gpu_cnt[qt]]
+        if got.size == want.size and np.array_equal(got, want):
+            continue
+        row = ho.scores[qt]
+        if ho.p.mode == O.MODE_TOPK:
+            srt = np.sort(row)[::-1]
+            kk = want.size
+            edge = srt[kk - 1]
+            nxt = srt[kk] if kk < srt.size else -np.inf
+            assert edge - nxt < GAP, "query tile %d: selection differs without a near-tie" % qt
+        else:
+            edge = ho.thr
+        diff = np.setxor1d(got, want)
+        assert np.all(np.abs(row[diff] - edge) < GAP), "query tile %d: differs away from the boundary" % qt
+        excluded.add(qt)
+    return excluded
+
+
+def out_error(got, want, bf16: bool):
+    """(max excess over the bound, mean-abs error, mean bound) for one block of rows."""
+    err = np.abs(got - want)
+    if not bf16:
+        return float(err.max()), float(err.mean()), OUT_MEAN_ABS
+    half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), 1e-30))) - 8)
+    return float((err - half_ulp).max()), float(err.mean()), OUT_MEAN_ABS + float((half_ulp / 2).mean())
+
+
+def compare_outputs(ho: HeadOracle, res, b, h, tiles, bf16=False):
+    """Compares the GPU output rows of the given query tiles with the oracle."""
+    errs, means, bounds = [], [], []
+    for qt in tiles:
+        toks, of, want = ho.tile_out(qt)
+        got = res["out"][b, toks, h]
+        mx, mean, bound = out_error(got, want, bf16)
+        errs.append(mx)
+        means.append(mean)
+        bounds.append(bound)
+    assert max(errs) <= OUT_MAX_ABS, "max-abs %.3g" % max(errs)
+    assert float(np.mean(means)) <= float(np.mean(bounds)), "mean-abs %.3g" % np.mean(means)
+    return max(errs), float(np.mean(means))
