@@ -106,6 +106,15 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def describe(wl) -> str:
+    names = {0: "text", 1: "ref image", 2: "ref audio", 3: "other"}
+    cond = " + ".join("%d %s" % (n, names.get(k, "cond")) for k, n in wl.cond)
+    sel = ("keep %g%%" % (100 * wl.keep)) if wl.mode == 0 else ("adaptive tau %g" % wl.tau)
+    sink = "exact_kv" if wl.sink == 0 else "exact_kv_and_rows"
+    return "%s: %s conditioning + %dx%dx%d video tokens (S=%d), B=%d, H=%d, d=%d, %s, %s" % (
+        wl.name, cond or "no", *wl.grid, wl.seq_len, wl.B, wl.H, wl.D, sel, sink)
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -177,9 +186,9 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "1344x768 5 s: 4672 conditioning + 32x48x84 video tokens, H=24, d=128, "
-                                   "keep 10%, exact_kv", "B": wl.B, "seq_len": wl.seq_len,
-                       "parallelism": "host cores"},
+            "config": {"workload": describe(wl) + ", %s output" % args.out_dtype, "B": wl.B,
+                       "seq_len": wl.seq_len, "parallelism": "host cores",
+                       "l2": "inputs (2.5 GB) larger than L2; no flush"},
             "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -298,9 +307,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "1344x768 5 s: 4672 conditioning (512 text + 48x84 ref image + 128 "
-                                   "audio) + 32x48x84 video tokens, H=24, d=128, keep 10%, exact_kv, "
-                                   "%s output" % args.out_dtype,
+            "config": {"workload": describe(wl) + ", %s output" % args.out_dtype,
                        "B": wl.B, "seq_len": wl.seq_len, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
                        "l2": "inputs (2.5 GB) larger than L2; no flush"},
             "roofline": {"bound": "tensor", "kernel": "vsa_attn_kernel", "achieved": achieved, "peak": peak,

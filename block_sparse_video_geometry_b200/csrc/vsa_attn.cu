@@ -650,7 +650,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   if (kmax != want_kmax) return VSA_ERR_INVALID_ARG;
   if (L->n_cond > kMaxCondTiles) return VSA_ERR_UNSUPPORTED;
   const int n_sm = sm_count();
-  if (n_sm <= 0) return VSA_ERR_CUDA;
+  if (n_sm <= 0) return cuda_fail("vsa_sparse_attn_fwd: no current CUDA device");
 
   const DevLayout D = L->dev();
   AttnArgs a{};
@@ -691,10 +691,11 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.err = static_cast<int*>(workspace);
 
   const size_t smem = sizeof(AttnSmem) + 1024;
-  if (cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return VSA_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, kAttnWorkspace, stream) != cudaSuccess) return VSA_ERR_CUDA;
+  cudaError_t e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
+  e = cudaMemsetAsync(workspace, 0, kAttnWorkspace, stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaMemsetAsync", e);
   const int grid = std::max(1, std::min(a.n_items, n_sm));
   const uint16_t* qq = static_cast<const uint16_t*>(q);
   const uint16_t* kk = static_cast<const uint16_t*>(k);
@@ -704,22 +705,26 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
     const int64_t vo = L->video_start * ss;
     const uint16_t* bases[3] = {qq + b * sb, kk + b * sb, vv + b * sb};
     for (int t = 0; t < 3; ++t) {
-      if (!make_cond_map(&m[2 * t], bases[t], L->seq_len, H, ss, sh)) return VSA_ERR_CUDA;
+      if (!make_cond_map(&m[2 * t], bases[t], L->seq_len, H, ss, sh))
+        return cuda_fail("vsa_sparse_attn_fwd: cuTensorMapEncodeTiled (token map)");
       if (!make_video_map(&m[2 * t + 1], bases[t] + vo, L->grid_t, L->grid_h, L->grid_w, H, ss, sh))
-        return VSA_ERR_CUDA;
+        return cuda_fail("vsa_sparse_attn_fwd: cuTensorMapEncodeTiled (video grid map)");
     }
     a.b = b;
     vsa_attn_kernel<<<grid, kThreads, smem, stream>>>(a, m[0], m[1], m[2], m[3], m[4], m[5]);
-    if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: launch", e);
   }
   return VSA_OK;
 }
 
 vsa_status vsa_sparse_attn_status(const void* workspace, cudaStream_t stream) {
   if (!workspace) return VSA_ERR_INVALID_ARG;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return VSA_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_status: cudaStreamSynchronize", e);
   int err = 0;
-  if (cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return VSA_ERR_CUDA;
+  e = cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_status: cudaMemcpy", e);
   return err == 0 ? VSA_OK : static_cast<vsa_status>(err);
 }
 

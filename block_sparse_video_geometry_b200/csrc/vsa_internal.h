@@ -78,6 +78,11 @@ namespace vsa {
 // k for top-k selection: max(1, ceil(keep * Nv * (1 - 2^-20))), clamped to Nv.
 int32_t topk_count(float keep, int32_t n_video);
 
+// Records "where: cuda error string" for vsa_last_error_detail and returns
+// VSA_ERR_CUDA; a message-only variant for failures without a cudaError_t.
+vsa_status cuda_fail(const char* where, cudaError_t e);
+vsa_status cuda_fail(const char* where);
+
 // Validation shared by the entry points.
 vsa_status check_params(const vsa_params* p);
 float effective_scale(const vsa_params* p);

@@ -10,6 +10,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <new>
 
@@ -18,6 +19,20 @@
 #include "vsa_internal.h"
 
 namespace vsa {
+
+namespace {
+thread_local char g_detail[256] = "";
+}
+
+vsa_status cuda_fail(const char* where, cudaError_t e) {
+  std::snprintf(g_detail, sizeof(g_detail), "%s: %s", where, cudaGetErrorString(e));
+  return VSA_ERR_CUDA;
+}
+
+vsa_status cuda_fail(const char* where) {
+  std::snprintf(g_detail, sizeof(g_detail), "%s", where);
+  return VSA_ERR_CUDA;
+}
 
 int32_t topk_count(float keep, int32_t n_video) {
   const double prod = static_cast<double>(keep) * static_cast<double>(n_video) *
@@ -209,8 +224,8 @@ vsa_status vsa_layout_upload(vsa_layout* L, void* dev_buf, size_t dev_bytes, cud
       {L->off.origin, L->origin.data(), L->origin.size() * sizeof(int32_t)},
   };
   for (const Piece& p : pieces) {
-    if (cudaMemcpyAsync(b + p.off, p.src, p.bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-      return VSA_ERR_CUDA;
+    const cudaError_t e = cudaMemcpyAsync(b + p.off, p.src, p.bytes, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail("vsa_layout_upload: cudaMemcpyAsync", e);
   }
   L->dev_buf = dev_buf;
   return VSA_OK;
@@ -264,5 +279,7 @@ const char* vsa_status_string(vsa_status s) {
 }
 
 int32_t vsa_version(void) { return (1 << 16) | 0; }
+
+const char* vsa_last_error_detail(void) { return g_detail; }
 
 }  // extern "C"

@@ -56,7 +56,7 @@ pool_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restr
   const int tile = blockIdx.x, b = blockIdx.y, which = blockIdx.z;
   const uint16_t* x = which == 0 ? q : (which == 1 ? k : v);
   __shared__ int tok[kTile];
-  if (threadIdx.x < kTile) tok[threadIdx.x] = L.perm[tile * kTile + threadIdx.x];
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
   __syncthreads();
   const float n = static_cast<float>(L.count[tile]);
   const int nchunks = H * 16;
@@ -456,22 +456,23 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
 
   const size_t coarse_smem = sizeof(CoarseSmem);
   auto ck = adaptive ? coarse_kernel<true> : coarse_kernel<false>;
-  if (cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(coarse_smem)) != cudaSuccess)
-    return VSA_ERR_CUDA;
+  cudaError_t e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(coarse_smem));
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: cudaFuncSetAttribute(coarse)", e);
   ck<<<dim3(ws.n_row_blocks, H, B), kCoarseThreads, coarse_smem, stream>>>(
       L->n_tiles, L->n_cond, L->n_video, H, B, pooled, scale, scores, ld, o_coarse, stats);
 
   const size_t sel_smem = rows_per_block * row_bytes + rows_per_block * 256 * sizeof(uint32_t);
   auto sk = adaptive ? select_kernel<true> : select_kernel<false>;
-  if (cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sel_smem)) != cudaSuccess)
-    return VSA_ERR_CUDA;
+  e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sel_smem));
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: cudaFuncSetAttribute(select)", e);
   sk<<<dim3((L->n_tiles + rows_per_block - 1) / rows_per_block, H, B), 32 * rows_per_block, sel_smem,
        stream>>>(L->n_tiles, L->n_video, H, scores, ld, kmax, p->tau, stats, ws.n_row_blocks, idx,
                  kmax, cnt);
-  if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: launch", e);
   return VSA_OK;
 }
 
 }  // extern "C"
+

@@ -27,7 +27,10 @@ TILE, HEAD_DIM = 64, 128
 class VSAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+        msg = "%s: %s (status %d)" % (where, status_string(status), status)
+        if status == ERR_CUDA:
+            msg += ": " + lib().vsa_last_error_detail().decode()
+        super().__init__(msg)
 
 
 class Segment(ctypes.Structure):
@@ -68,6 +71,7 @@ _SIGNATURES = {
     "vsa_sparse_attn_status": (_I32, [_P, _P]),
     "vsa_status_string": (ctypes.c_char_p, [_I32]),
     "vsa_version": (_I32, []),
+    "vsa_last_error_detail": (ctypes.c_char_p, []),
 }
 
 

@@ -251,6 +251,11 @@ vsa_status vsa_sparse_attn_status(const void* workspace, cudaStream_t stream);
 
 const char* vsa_status_string(vsa_status status);
 
+/* Text of the most recent VSA_ERR_CUDA returned on the calling thread: the
+ * failing runtime call and CUDA's error string ("" if none yet). The pointer
+ * stays valid until the thread's next failing call. */
+const char* vsa_last_error_detail(void);
+
 /* Library ABI version, (major << 16) | minor. */
 int32_t vsa_version(void);
 
