@@ -82,6 +82,8 @@ int32_t topk_count(float keep, int32_t n_video);
 // VSA_ERR_CUDA; a message-only variant for failures without a cudaError_t.
 vsa_status cuda_fail(const char* where, cudaError_t e);
 vsa_status cuda_fail(const char* where);
+// Records a message for vsa_last_error_detail without a CUDA error.
+void set_detail(const char* msg);
 
 // Validation shared by the entry points.
 vsa_status check_params(const vsa_params* p);

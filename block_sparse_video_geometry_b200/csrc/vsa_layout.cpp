@@ -34,6 +34,8 @@ vsa_status cuda_fail(const char* where) {
   return VSA_ERR_CUDA;
 }
 
+void set_detail(const char* msg) { std::snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+
 int32_t topk_count(float keep, int32_t n_video) {
   const double prod = static_cast<double>(keep) * static_cast<double>(n_video) *
                       (1.0 - 1.0 / 1048576.0);

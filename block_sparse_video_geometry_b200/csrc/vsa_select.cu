@@ -476,3 +476,73 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
 
 }  // extern "C"
 
+// -------------------------------------------------------------------------
+// Allocation-free variant of vsa_coarse_select.
+//
+// Some callers cannot hand this library a workspace: code running inside a
+// host framework that plans every device allocation ahead of time and forbids
+// allocations outside its plan, or callers that must not pay the device-wide
+// synchronisation and latency of cudaMalloc in the middle of a step. For them
+// the selection scratch (pooled means, score matrix, adaptive partial sums)
+// lives in the fixed buffer below, which is part of the library's device
+// image: every GPU that loads libvsa holds these 32 MiB until the process
+// exits. Workloads whose scratch does not fit are refused, not truncated.
+// -------------------------------------------------------------------------
+#include <cstdio>
+#include <mutex>
+
+namespace vsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+}  // namespace vsa
+
+extern "C" vsa_status vsa_coarse_select_noalloc(const vsa_layout* L, const vsa_params* p, int32_t B,
+                                                int32_t H, const void* q, const void* k, const void* v,
+                                                int64_t sb, int64_t ss, int64_t sh, int32_t* idx,
+                                                int32_t* cnt, float* o_coarse, cudaStream_t stream) {
+  if (!L || B <= 0 || H <= 0) return VSA_ERR_INVALID_ARG;
+  vsa_status st = check_params(p);
+  if (st != VSA_OK) return st;
+  const size_t need = select_workspace(L, B, H).total;
+  if (need > kNoAllocScratchBytes) {
+    char msg[160];
+    std::snprintf(msg, sizeof(msg),
+                  "vsa_coarse_select_noalloc: this shape needs %zu bytes of scratch, the built-in buffer "
+                  "holds %zu",
+                  need, kNoAllocScratchBytes);
+    set_detail(msg);
+    return VSA_ERR_UNSUPPORTED;
+  }
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_noalloc: cudaGetDevice", e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) {
+    set_detail("vsa_coarse_select_noalloc: device ordinal beyond 63");
+    return VSA_ERR_UNSUPPORTED;
+  }
+  void* scratch = nullptr;
+  {
+    // Host code must not use the array's name as a device address: the
+    // address is looked up once per device, with that device current.
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+      if (e != cudaSuccess) {
+        g_noalloc_ptr[dev] = nullptr;
+        return cuda_fail("vsa_coarse_select_noalloc: cudaGetSymbolAddress", e);
+      }
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return vsa_coarse_select(L, p, B, H, q, k, v, sb, ss, sh, idx, cnt, o_coarse, scratch,
+                           kNoAllocScratchBytes, stream);
+}

@@ -64,6 +64,8 @@ _SIGNATURES = {
     "vsa_coarse_select_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
     "vsa_coarse_select": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
                                  _P, _P, _P, _P, _SZ, _P]),
+    "vsa_coarse_select_noalloc": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
+                                         _P, _P, _P, _P]),
     "vsa_sparse_attn_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
     "vsa_sparse_attn_fwd": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
                                    _P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64, _I64,
@@ -197,6 +199,17 @@ def coarse_select(layout: Layout, params: Params, q, k, v, idx, cnt, o_coarse, w
                                    o_coarse.data_ptr(), workspace.data_ptr(),
                                    workspace.numel() * workspace.element_size(), _stream_handle(stream)),
            "vsa_coarse_select")
+
+
+def coarse_select_noalloc(layout: Layout, params: Params, q, k, v, idx, cnt, o_coarse, stream=None) -> None:
+    """vsa_coarse_select_noalloc: the selection call for callers that cannot
+    provide scratch memory (the library's built-in 32 MiB buffer is used)."""
+    B, S, H, _ = q.shape
+    sb, ss, sh = _qkv_strides(q, k, v)
+    _check(lib().vsa_coarse_select_noalloc(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
+                                           v.data_ptr(), sb, ss, sh, idx.data_ptr(), cnt.data_ptr(),
+                                           o_coarse.data_ptr(), _stream_handle(stream)),
+           "vsa_coarse_select_noalloc")
 
 
 def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: int, o_coarse, out,

@@ -207,6 +207,33 @@ vsa_status vsa_coarse_select(const vsa_layout* layout, const vsa_params* params,
                              int32_t* idx, int32_t* cnt, float* o_coarse,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* vsa_coarse_select_noalloc: vsa_coarse_select without a workspace argument.
+ * The web pages describe no such call; it exists for callers that cannot give
+ * this library scratch memory: a host framework that plans every device
+ * allocation in advance and allows none outside its plan, or a caller that
+ * cannot afford the synchronisation and latency of cudaMalloc inside a step.
+ *
+ * Same arguments, outputs and results as vsa_coarse_select, minus workspace.
+ * The scratch (pooled means, score matrix, adaptive sums) is a fixed 32 MiB
+ * buffer inside the library's device image, held by every GPU that loads the
+ * library until the process exits. Shapes whose scratch exceeds 32 MiB
+ * (roughly: B * H * n_tiles * (1536 + 4 * round_up(n_video_tiles, 64)) bytes;
+ * the 17k-token, 24-head workload fits, the 1344x768 shapes do not) are
+ * refused with VSA_ERR_UNSUPPORTED and a message in vsa_last_error_detail.
+ * The first call on a device looks up the buffer's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. Every call on a device shares the one buffer and leaves its
+ * contents behind; each call writes every scratch byte it later reads, so
+ * nothing needs clearing, but calls that overlap on the GPU (different
+ * streams, or concurrent host threads) race on the buffer. Allocates no
+ * memory of any kind. */
+vsa_status vsa_coarse_select_noalloc(const vsa_layout* layout, const vsa_params* params,
+                                     int32_t B, int32_t H,
+                                     const void* q, const void* k, const void* v,
+                                     int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                                     int32_t* idx, int32_t* cnt, float* o_coarse,
+                                     cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Fine branch + gate combine                                                */
 /* ------------------------------------------------------------------------ */
@@ -251,9 +278,10 @@ vsa_status vsa_sparse_attn_status(const void* workspace, cudaStream_t stream);
 
 const char* vsa_status_string(vsa_status status);
 
-/* Text of the most recent VSA_ERR_CUDA returned on the calling thread: the
- * failing runtime call and CUDA's error string ("" if none yet). The pointer
- * stays valid until the thread's next failing call. */
+/* Text of the most recent VSA_ERR_CUDA returned on the calling thread (the
+ * failing runtime call and CUDA's error string), or of a shape refused by
+ * vsa_coarse_select_noalloc; "" if none yet. The pointer stays valid until
+ * the thread's next failing call. */
 const char* vsa_last_error_detail(void);
 
 /* Library ABI version, (major << 16) | minor. */
