@@ -13,17 +13,22 @@
 //    tiles' key lists; each 128x64 score block is masked per 64-row half for
 //    key tiles that only one of the two tiles selected. Conditioning key tiles
 //    are shared by every query tile, so they run at full M = 128 efficiency.
-//  * Q, K, V are read straight from the natural [B, S, H, 128] layout by TMA:
-//    a 3-D map (d, head, token) for 64-token conditioning runs and a 5-D map
-//    (d, head, w, h, t) over the video latent grid whose 4x4x4 box lands a
-//    video cube in shared memory in slot order; cubes cut by the grid edge are
-//    zero-filled by the TMA unit and masked in the softmax.
-//  * Warp roles: warp 0 streams the merged key list and issues TMA loads into
-//    a 4-stage ring; warp 1 owns TMEM and issues tcgen05.mma (S = Q K^T into
-//    one of two TMEM score buffers, O += P V into a TMEM accumulator); warps
-//    2-5 run the online softmax (fp32, exp2, lazy rescale of O in TMEM when
-//    the running max grows by more than 2^8), write P as bf16 into swizzled
-//    shared memory, and run the epilogue.
+//  * Q, K, V are read straight from the natural [B, S, H, 128] layout by TMA
+//    (no multicast): a 3-D map (d, head, token) for 64-token conditioning runs
+//    and a 5-D map (d, head, w, h, t) over the video latent grid whose 4x4x4
+//    box lands a video cube in shared memory in slot order; cubes cut by the
+//    grid edge are zero-filled by the TMA unit and masked in the softmax. Each
+//    64-key step gathers 256 rows of 128 B; a TMA issue occupies its warp for
+//    a few hundred cycles, so K and V have a producer warp each, and two CTAs
+//    per SM keep the TMA unit busy.
+//  * Warp roles per CTA: warp 0 walks the merged key list, loads Q and K and
+//    publishes per-step tile info; warp 1 loads V; warp 2 owns TMEM and issues
+//    tcgen05.mma (S = Q K^T into one of two TMEM score buffers; O += P V with P
+//    read from TMEM); warps 3-6 run the fp32 online softmax (exp2, lazy rescale
+//    of O in TMEM when the running max grows by more than 2^8), write P as bf16
+//    over the score buffer with tcgen05.st, and run the epilogue. About 100 KB
+//    of shared memory and 256 TMEM columns per CTA: two CTAs share an SM so
+//    that one's softmax overlaps the other's tensor work.
 //  * Every wait is bounded: a wait that runs out sets an error word in the
 //    workspace, raises an abort flag that ends the other roles' loops, drains
 //    in-flight TMA and MMA work and frees TMEM before the block exits.
@@ -45,12 +50,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
+static_assert(kKStages == kVStages, "the producers share one stage counter");
+constexpr int kInfoSlots = 4;
+constexpr int kThreads = 224;
+constexpr int kWarpK = 0, kWarpV = 1, kWarpMma = 2;   // warps 3..6: softmax / epilogue
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;
+constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;   // P (bf16) overwrites S columns 0..31
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kMaxCondTiles = 2048;
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);    // S = Q K^T, both K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // O = P V, V is MN-major
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -65,17 +73,21 @@ struct StageInfo {
 };
 
 struct AttnSmem {
-  uint8_t q[2][128 * 128];            // [d half][128 rows x 128 B], SW128
-  uint8_t k[kStages][2][64 * 128];    // [stage][d half][64 keys x 128 B], SW128
-  uint8_t v[kStages][2][64 * 128];
-  uint8_t p[2][128 * 128];            // [buffer][128 rows x 64 keys bf16], SW128
-  int2 cond[kMaxCondTiles];           // conditioning tiles: (first token, count)
-  StageInfo info[kStages];
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint8_t q[2][128 * 128];             // [d half][128 rows x 128 B], SW128
+  uint8_t k[kKStages][2][64 * 128];    // [stage][d half][64 keys x 128 B], SW128
+  uint8_t v[kVStages][2][64 * 128];
+  StageInfo info[kInfoSlots];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t info_full[kInfoSlots];
   uint64_t q_full, q_empty, s_full[2], p_full[2], o_done, o_full, o_empty, drain;
   uint32_t tmem_base;
   int abort;
+  int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
 };
+
+size_t attn_smem_bytes(int n_cond) {
+  return sizeof(AttnSmem) + sizeof(int2) * static_cast<size_t>(std::max(0, n_cond - 1)) + 1024;
+}
 
 struct Geom {
   int32_t n_cond, n_video, n_tiles;
@@ -224,7 +236,19 @@ __device__ __forceinline__ bool warp_wait(AttnSmem& sm, uint64_t& bar, uint32_t 
   return ok != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Pairwise tree reductions over 64 values: short dependency chains.
+__device__ __forceinline__ float tree_max64(const float (&x)[64]) {
+  float t[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) t[i] = fmaxf(x[i], x[i + 32]);
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  return t[0];
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tq_c,
                 const __grid_constant__ CUtensorMap tq_v, const __grid_constant__ CUtensorMap tk_c,
                 const __grid_constant__ CUtensorMap tk_v, const __grid_constant__ CUtensorMap tv_c,
@@ -238,27 +262,36 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
   for (int i = threadIdx.x; i < G.n_cond; i += kThreads)
     sm.cond[i] = make_int2(a.origin[i].x, a.count[i]);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.kv_full[s]), 1);
-      mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(smem_u32(&sm.k_full[s]), 1);
+      mbar_init(smem_u32(&sm.k_empty[s]), 1);
     }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(smem_u32(&sm.v_full[s]), 1);
+      mbar_init(smem_u32(&sm.v_empty[s]), 1);
+    }
+    for (int s = 0; s < kInfoSlots; ++s) mbar_init(smem_u32(&sm.info_full[s]), 1);
     mbar_init(smem_u32(&sm.q_full), 1);
     mbar_init(smem_u32(&sm.q_empty), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.p_full[i]), 128);
+      mbar_init(smem_u32(&sm.p_full[i]), 4);     // one arrival per softmax warp
     }
     mbar_init(smem_u32(&sm.o_done), 1);
     mbar_init(smem_u32(&sm.o_full), 1);
-    mbar_init(smem_u32(&sm.o_empty), 128);
+    mbar_init(smem_u32(&sm.o_empty), 4);
     mbar_init(smem_u32(&sm.drain), 1);
     sm.abort = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    for (const CUtensorMap* m : {&tq_c, &tq_v, &tk_c, &tk_v, &tv_c, &tv_v}) tma_prefetch_desc(m);
+    for (const CUtensorMap* m : {&tq_c, &tq_v, &tk_c, &tk_v}) tma_prefetch_desc(m);
   }
-  if (warp == 1) {
+  if (warp == kWarpV && lane == 0) {
+    tma_prefetch_desc(&tv_c);
+    tma_prefetch_desc(&tv_v);
+  }
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -267,24 +300,32 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    uint32_t step = 0;
-    int it_n = 0;
+  if (warp == kWarpK || warp == kWarpV) {
+    // ----------------------------------------------------------- producers
+    // Both producer warps walk the same key list; the K warp also loads Q and
+    // publishes the per-step tile info.
+    const bool is_k = warp == kWarpK;
+    const CUtensorMap* mc = is_k ? &tk_c : &tv_c;
+    const CUtensorMap* mv = is_k ? &tk_v : &tv_v;
+    uint64_t* full = is_k ? sm.k_full : sm.v_full;
+    uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
+    uint32_t step = 0, issued = 0;
+    int it_n = 0, q_loads = 0;
     bool ok = true;
-    int q_loads = 0;
     for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
       const Item it = decode_item(a, item);
-      if (!(ok = warp_wait(sm, sm.q_empty, (it_n & 1) ^ 1, lane, a.err))) break;
-      if (lane == 0) {
-        const uint32_t bar = smem_u32(&sm.q_full);
-        mbar_arrive_expect_tx(bar, (it.qb >= 0 ? 2u : 1u) * 16384u);
-        load_tile(sm, G, &tq_c, &tq_v, it.qa, it.h, smem_u32(sm.q[0]), smem_u32(sm.q[1]), bar);
-        if (it.qb >= 0)
-          load_tile(sm, G, &tq_c, &tq_v, it.qb, it.h, smem_u32(sm.q[0] + 8192),
-                    smem_u32(sm.q[1] + 8192), bar);
+      if (is_k) {
+        if (!(ok = warp_wait(sm, sm.q_empty, (it_n & 1) ^ 1, lane, a.err))) break;
+        if (lane == 0) {
+          const uint32_t bar = smem_u32(&sm.q_full);
+          mbar_arrive_expect_tx(bar, (it.qb >= 0 ? 2u : 1u) * 16384u);
+          load_tile(sm, G, &tq_c, &tq_v, it.qa, it.h, smem_u32(sm.q[0]), smem_u32(sm.q[1]), bar);
+          if (it.qb >= 0)
+            load_tile(sm, G, &tq_c, &tq_v, it.qb, it.h, smem_u32(sm.q[0] + 8192),
+                      smem_u32(sm.q[1] + 8192), bar);
+        }
+        ++q_loads;
       }
-      ++q_loads;
       const int both = it.qb >= 0 ? 3 : 1;
       const int n_dense = it.dense ? G.n_tiles : G.n_cond;
       ListReader la, lb;
@@ -301,12 +342,12 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
           mask = both;
           return true;
         }
-        const int32_t x = la.peek(), y = lb.peek();
-        if (x == INT_MAX && y == INT_MAX) return false;
-        const int32_t t = min(x, y);
-        mask = (x == t ? 1 : 0) | (y == t ? 2 : 0);
-        if (x == t) la.pop(lane);
-        if (y == t) lb.pop(lane);
+        const int32_t x0 = la.peek(), y0 = lb.peek();
+        if (x0 == INT_MAX && y0 == INT_MAX) return false;
+        const int32_t t = min(x0, y0);
+        mask = (x0 == t ? 1 : 0) | (y0 == t ? 2 : 0);
+        if (x0 == t) la.pop(lane);
+        if (y0 == t) lb.pop(lane);
         tile = G.n_cond + t;
         return true;
       };
@@ -314,20 +355,23 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
       bool have = next(tile, mask);
       while (have) {
         const bool more = next(ntile, nmask);
-        const int s = step % kStages;
-        if (!(ok = warp_wait(sm, sm.kv_empty[s], ((step / kStages) & 1) ^ 1, lane, a.err))) break;
-        if (lane == 0) {
-          StageInfo& inf = sm.info[s];
+        const int st = step % kKStages;
+        if (!(ok = warp_wait(sm, empty[st], ((step / kKStages) & 1) ^ 1, lane, a.err))) break;
+        if (is_k && lane == 0) {
+          StageInfo& inf = sm.info[step % kInfoSlots];
           inf.tile = tile;
           inf.mask = mask;
           inf.last = more ? 0 : 1;
           inf.valid = tile_mask(sm, G, tile);
-          const uint32_t bar = smem_u32(&sm.kv_full[s]);
-          mbar_arrive_expect_tx(bar, 32768u);
-          load_tile(sm, G, &tk_c, &tk_v, tile, it.h, smem_u32(sm.k[s][0]), smem_u32(sm.k[s][1]), bar);
-          load_tile(sm, G, &tv_c, &tv_v, tile, it.h, smem_u32(sm.v[s][0]), smem_u32(sm.v[s][1]), bar);
+          mbar_arrive(smem_u32(&sm.info_full[step % kInfoSlots]));
+        }
+        if (lane == 0) {
+          uint8_t (*buf)[64 * 128] = is_k ? sm.k[st] : sm.v[st];
+          mbar_arrive_expect_tx(smem_u32(&full[st]), 16384u);
+          load_tile(sm, G, mc, mv, tile, it.h, smem_u32(buf[0]), smem_u32(buf[1]), smem_u32(&full[st]));
         }
         __syncwarp();
+        ++issued;
         ++step;
         tile = ntile;
         mask = nmask;
@@ -337,11 +381,11 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
     if (!ok && lane == 0) {
       // let every issued TMA load land before the block can exit: the last
       // fill of each stage, and the last Q load
-      for (uint32_t st = (step > kStages ? step - kStages : 0); st < step; ++st)
-        mbar_wait(smem_u32(&sm.kv_full[st % kStages]), (st / kStages) & 1, nullptr, kDrainNs);
-      if (q_loads > 0) mbar_wait(smem_u32(&sm.q_full), (q_loads - 1) & 1, nullptr, kDrainNs);
+      for (uint32_t i = (issued > kKStages ? issued - kKStages : 0); i < issued; ++i)
+        mbar_wait(smem_u32(&full[i % kKStages]), (i / kKStages) & 1, nullptr, kDrainNs);
+      if (is_k && q_loads > 0) mbar_wait(smem_u32(&sm.q_full), (q_loads - 1) & 1, nullptr, kDrainNs);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ----------------------------------------------------------------- MMA
     bool ok = true;
     if (lane == 0) {
@@ -350,17 +394,17 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
       auto pv = [&](uint32_t st, bool first) -> bool {
         if (!mbar_wait(smem_u32(&sm.p_full[st & 1]), (st >> 1) & 1, &sm.abort, kTimeoutNs)) return false;
         if (first && !mbar_wait(smem_u32(&sm.o_empty), (it_n & 1) ^ 1, &sm.abort, kTimeoutNs)) return false;
+        const int vs = st % kVStages;
+        if (!mbar_wait(smem_u32(&sm.v_full[vs]), (st / kVStages) & 1, &sm.abort, kTimeoutNs)) return false;
         tc_fence_after();
-        const int s = st % kStages;
-        const uint32_t pbase = smem_u32(sm.p[st & 1]);
-        const uint32_t vbase = smem_u32(sm.v[s][0]);
+        const uint32_t pcol = tmem + ((st & 1) ? kColS1 : kColS0);
+        const uint32_t vbase = smem_u32(sm.v[vs][0]);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = smem_desc_sw128(pbase + kk * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
-          umma_ss(tmem + kColO, ad, bd, kIdescPV, (first && kk == 0) ? 0u : 1u);
+          umma_ts(tmem + kColO, pcol + kk * 8, bd, kIdescPV, (first && kk == 0) ? 0u : 1u);
         }
-        umma_commit(smem_u32(&sm.kv_empty[s]));
+        umma_commit(smem_u32(&sm.v_empty[vs]));
         umma_commit(smem_u32(&sm.o_done));
         return true;
       };
@@ -369,12 +413,12 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
         int j = 0;
         bool last = false;
         while (!last) {
-          const int s = step % kStages;
-          if (!(ok = mbar_wait(smem_u32(&sm.kv_full[s]), (step / kStages) & 1, &sm.abort, kTimeoutNs))) break;
+          const int ks = step % kKStages;
+          if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (step / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
           tc_fence_after();
-          last = sm.info[s].last != 0;
+          last = sm.info[step % kInfoSlots].last != 0;
           const uint32_t qbase = smem_u32(sm.q[0]);
-          const uint32_t kbase = smem_u32(sm.k[s][0]);
+          const uint32_t kbase = smem_u32(sm.k[ks][0]);
           const uint32_t dS = tmem + ((step & 1) ? kColS1 : kColS0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -383,6 +427,7 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
             const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * 8192 + off, 16, 1024);
             umma_ss(dS, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
           }
+          umma_commit(smem_u32(&sm.k_empty[ks]));
           umma_commit(smem_u32(&sm.s_full[step & 1]));
           if (last) umma_commit(smem_u32(&sm.q_empty));
           if (j > 0 && !(ok = pv(step - 1, j == 1))) break;
@@ -405,84 +450,84 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
     const int r = quad * 32 + lane;         // row of the 128-row tile
     const int half = r >> 6;                // 0: first query tile, 1: second
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c = a.scale_log2;
     uint32_t step = 0;
     int it_n = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
       const Item it = decode_item(a, item);
-      float m_ref = -INFINITY, l = 0.f;
+      float ms = -INFINITY, l = 0.f;        // running max (scaled, log2 domain) and sum
       bool last = false;
       while (!last) {
-        const int s = step % kStages;
-        if (!(ok = warp_wait(sm, sm.s_full[step & 1], (step >> 1) & 1, lane, a.err))) break;
-        if (!(ok = warp_wait(sm, sm.kv_full[s], (step / kStages) & 1, lane, a.err))) break;
-        tc_fence_after();
-        const StageInfo inf = sm.info[s];
+        if (!(ok = warp_wait(sm, sm.info_full[step % kInfoSlots], (step / kInfoSlots) & 1, lane, a.err))) break;
+        const StageInfo inf = sm.info[step % kInfoSlots];
         last = inf.last != 0;
-        uint8_t* prow = sm.p[step & 1] + r * 128;
+        if (!(ok = warp_wait(sm, sm.s_full[step & 1], (step >> 1) & 1, lane, a.err))) break;
+        tc_fence_after();
+        const uint32_t scol = lane_addr + ((step & 1) ? kColS1 : kColS0);
+        uint32_t pw[32];
         if ((inf.mask >> half) & 1) {
           float x[64];
           {
-            uint32_t u[32];
-            const uint32_t col = (step & 1) ? kColS1 : kColS0;
-            tmem_ld32(lane_addr + col, u);
+            uint32_t u0[32], u1[32];
+            tmem_ld32(scol, u0);
+            tmem_ld32(scol + 32, u1);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(u[c]);
-            tmem_ld32(lane_addr + col + 32, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) x[32 + c] = __uint_as_float(u[c]);
+            for (int i = 0; i < 32; ++i) {
+              x[i] = __uint_as_float(u0[i]);
+              x[32 + i] = __uint_as_float(u1[i]);
+            }
           }
-          float mt = -INFINITY;
+          if (inf.valid != ~0ull) {           // partial tile: padded keys never attend
+            const uint32_t lo = static_cast<uint32_t>(inf.valid), hi = static_cast<uint32_t>(inf.valid >> 32);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            x[c] = ((inf.valid >> c) & 1ull) ? x[c] * a.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, x[c]);
+            for (int i = 0; i < 32; ++i) {
+              x[i] = ((lo >> i) & 1u) ? x[i] : -INFINITY;
+              x[32 + i] = ((hi >> i) & 1u) ? x[32 + i] : -INFINITY;
+            }
           }
-          const bool need = m_ref != -INFINITY && mt > m_ref + kRescaleLog2;
-          if (m_ref == -INFINITY) m_ref = mt;
+          const float mt = tree_max64(x) * c;
+          const bool need = ms != -INFINITY && mt > ms + kRescaleLog2;
+          if (ms == -INFINITY) ms = mt;       // first key tile of this row: O and l are still zero
           if (__any_sync(0xffffffffu, need)) {
             // rescale this warp's rows of O once the previous P V has landed
             if (!(ok = warp_wait(sm, sm.o_done, (step - 1) & 1, lane, a.err))) break;
             tc_fence_after();
-            const float f = need ? ex2_approx(m_ref - mt) : 1.0f;
+            const float f = need ? ex2_approx(ms - mt) : 1.0f;
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
               uint32_t u[32];
               tmem_ld32(lane_addr + kColO + ch * 32, u);
               tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * f);
+              for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * f);
               tmem_st32(lane_addr + kColO + ch * 32, u);
             }
             tmem_wait_st();
             if (need) {
               l *= f;
-              m_ref = mt;
+              ms = mt;
             }
           }
-          float ps = 0.f;
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float p0 = ex2_approx(x[8 * ch + 2 * e] - m_ref);
-              const float p1 = ex2_approx(x[8 * ch + 2 * e + 1] - m_ref);
-              ps += p0 + p1;
-              w[e] = pack_bf16x2(p0, p1);
-            }
-            *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2_approx(fmaf(x[2 * i], c, -ms));
+            const float p1 = ex2_approx(fmaf(x[2 * i + 1], c, -ms));
+            ps[i & 3] += p0 + p1;
+            pw[i] = pack_bf16x2(p0, p1);
           }
-          l += ps;
+          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         } else {
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(prow + (ch << 4)) = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 32; ++i) pw[i] = 0u;     // rows of the other query tile
         }
-        fence_proxy_async_smem();
+        tmem_st32(scol, pw);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&sm.p_full[step & 1]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[step & 1]));
         ++step;
       }
       if (!ok) break;
@@ -513,39 +558,40 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
         if (row_ok) {
           float y[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) y[c] = __uint_as_float(u[c]) * inv_l;
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(u[i]) * inv_l;
           if (oc) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              const float4 cv = *reinterpret_cast<const float4*>(oc + ch * 32 + c);
-              y[c] = fmaf(gate, cv.x, y[c]);
-              y[c + 1] = fmaf(gate, cv.y, y[c + 1]);
-              y[c + 2] = fmaf(gate, cv.z, y[c + 2]);
-              y[c + 3] = fmaf(gate, cv.w, y[c + 3]);
+            for (int i = 0; i < 32; i += 4) {
+              const float4 cv = *reinterpret_cast<const float4*>(oc + ch * 32 + i);
+              y[i] = fmaf(gate, cv.x, y[i]);
+              y[i + 1] = fmaf(gate, cv.y, y[i + 1]);
+              y[i + 2] = fmaf(gate, cv.z, y[i + 2]);
+              y[i + 3] = fmaf(gate, cv.w, y[i + 3]);
             }
           }
           const int64_t off = a.b * a.o_sb + tok * a.o_ss + it.h * a.o_sh + ch * 32;
           if (a.out_bf16) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + off);
 #pragma unroll
-            for (int c = 0; c < 32; c += 8)
-              dst[c / 8] = make_uint4(pack_bf16x2(y[c], y[c + 1]), pack_bf16x2(y[c + 2], y[c + 3]),
-                                      pack_bf16x2(y[c + 4], y[c + 5]), pack_bf16x2(y[c + 6], y[c + 7]));
+            for (int i = 0; i < 32; i += 8)
+              dst[i / 8] = make_uint4(pack_bf16x2(y[i], y[i + 1]), pack_bf16x2(y[i + 2], y[i + 3]),
+                                      pack_bf16x2(y[i + 4], y[i + 5]), pack_bf16x2(y[i + 6], y[i + 7]));
           } else {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + off);
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) dst[c / 4] = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
+            for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.o_empty));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -605,6 +651,7 @@ int sm_count() {
 }
 
 constexpr size_t kAttnWorkspace = 256;   // error word
+constexpr size_t kMaxAttnSmem = 227 * 1024;
 
 }  // namespace
 }  // namespace vsa
@@ -648,7 +695,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   int32_t want_kmax = 0;
   vsa_select_kmax(L, p, &want_kmax);
   if (kmax != want_kmax) return VSA_ERR_INVALID_ARG;
-  if (L->n_cond > kMaxCondTiles) return VSA_ERR_UNSUPPORTED;
+  const size_t smem = attn_smem_bytes(L->n_cond);
+  if (smem > kMaxAttnSmem) return VSA_ERR_UNSUPPORTED;   // more than ~16k conditioning tiles
   const int n_sm = sm_count();
   if (n_sm <= 0) return cuda_fail("vsa_sparse_attn_fwd: no current CUDA device");
 
@@ -690,13 +738,21 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.scale_log2 = effective_scale(p) * 1.4426950408889634f;
   a.err = static_cast<int*>(workspace);
 
-  const size_t smem = sizeof(AttnSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
+  // Two CTAs per SM when their shared memory fits (TMEM holds two 256-column
+  // CTAs); registers are bounded for two by __launch_bounds__.
+  int dev = 0, smem_sm = 0, smem_resv = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&smem_resv, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  const int per_sm = 2 * (smem + smem_resv) <= static_cast<size_t>(smem_sm) ? 2 : 1;
+  e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute(carveout)", e);
   e = cudaMemsetAsync(workspace, 0, kAttnWorkspace, stream);
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaMemsetAsync", e);
-  const int grid = std::max(1, std::min(a.n_items, n_sm));
+  const int grid = std::max(1, std::min(a.n_items, n_sm * per_sm));
   const uint16_t* qq = static_cast<const uint16_t*>(q);
   const uint16_t* kk = static_cast<const uint16_t*>(k);
   const uint16_t* vv = static_cast<const uint16_t*>(v);

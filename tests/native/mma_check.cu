@@ -5,6 +5,8 @@
 //   S2 = Q Kc^T  Kc = one 4x4x4 cube gathered by the 5-D video-grid map
 //   O  = P V     P [128 x 64] written to 128B-swizzled smem by threads,
 //                V [64 x 128] loaded by the 3-D map, used as an MN-major operand
+//   O2 = P V     the same product with P written to TMEM by tcgen05.st
+//                (row i in lane i, bf16 pairs per column) and read as A from TMEM
 // Same descriptors, swizzle and TMEM access pattern as vsa_attn.cu. All waits
 // are bounded; a wait that runs out writes 1 to *err.
 #include <cuda.h>
@@ -23,7 +25,7 @@ struct __align__(1024) CheckSmem {
   uint8_t kc[2][64 * 128];
   uint8_t v[2][64 * 128];
   uint8_t p[128 * 128];
-  uint64_t bar_load, bar_mma;
+  uint64_t bar_load, bar_mma, bar_ts;
   uint32_t tmem_base;
 };
 
@@ -33,17 +35,18 @@ __global__ void __launch_bounds__(128, 1)
 check_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tgrid,
              int cube_t0, int cube_h0, int cube_w0, int cube_head, const uint16_t* p_in,
-             float* s1_out, float* s2_out, float* o_out, int* err) {
+             float* s1_out, float* s2_out, float* o_out, float* o2_out, int* err) {
   extern __shared__ uint8_t raw[];
   CheckSmem& sm = *reinterpret_cast<CheckSmem*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     mbar_init(smem_u32(&sm.bar_load), 1);
     mbar_init(smem_u32(&sm.bar_mma), 1);
+    mbar_init(smem_u32(&sm.bar_ts), 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&sm.tmem_base), 256);
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
     tmem_relinquish();
   }
   // P: row r = thread, 64 bf16, written in the 128B-swizzled K-major layout
@@ -94,9 +97,31 @@ check_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
   }
   __syncthreads();
   ok = *reinterpret_cast<volatile int*>(err) == 0;
+  const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  if (ok) {
+    // P into TMEM columns 384..415 of this thread's lane, then O2 = P V from TMEM
+    tc_fence_after();
+    uint32_t w[32];
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(p_in + tid * 64);
+    for (int c = 0; c < 32; ++c) w[c] = src[c];
+    tmem_st32(la + 384, w);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (ok && tid == 0) {
+    tc_fence_after();
+    const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
+    for (int kk = 0; kk < 4; ++kk)
+      umma_ts(tmem + 256, tmem + 384 + kk * 8, smem_desc_sw128(smem_u32(sm.v[0]) + kk * 2048, 8192, 1024),
+              idPV, kk > 0);
+    umma_commit(smem_u32(&sm.bar_ts));
+    if (!mbar_wait(smem_u32(&sm.bar_ts), 0, nullptr, kTimeout)) *err = 1;
+  }
+  __syncthreads();
+  ok = *reinterpret_cast<volatile int*>(err) == 0;
   if (ok) {
     tc_fence_after();
-    const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     uint32_t u[32];
     for (int ch = 0; ch < 2; ++ch) {
       tmem_ld32(la + 128 + ch * 32, u);
@@ -110,13 +135,16 @@ check_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
       tmem_ld32(la + ch * 32, u);
       tmem_wait_ld();
       for (int c = 0; c < 32; ++c) o_out[tid * 128 + ch * 32 + c] = __uint_as_float(u[c]);
+      tmem_ld32(la + 256 + ch * 32, u);
+      tmem_wait_ld();
+      for (int c = 0; c < 32; ++c) o2_out[tid * 128 + ch * 32 + c] = __uint_as_float(u[c]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -141,11 +169,11 @@ bool encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims, 
 }  // namespace
 
 // q [128, 128], k [64, 128], v [64, 128], p [128, 64] bf16 row-major;
-// grid [T, Hg, W, 2 heads, 128] bf16; outputs fp32 s1 [128, 64], s2 [128, 64], o [128, 128].
+// grid [T, Hg, W, 2 heads, 128] bf16; outputs fp32 s1 [128, 64], s2 [128, 64], o and o2 [128, 128].
 // Returns 0 on success, 1 for a wait that ran out, 2 for a CUDA error.
 extern "C" int mma_check_run(const void* q, const void* k, const void* v, const void* p, const void* grid,
                              int T, int Hg, int W, int cube_t0, int cube_h0, int cube_w0, int cube_head,
-                             float* s1, float* s2, float* o, int* err_dev) {
+                             float* s1, float* s2, float* o, float* o2, int* err_dev) {
   CUtensorMap tq, tk, tv, tg;
   const cuuint32_t box3[3] = {64, 1, 64};
   const cuuint64_t dq[3] = {128, 1, 128}, dk[3] = {128, 1, 64};
@@ -162,7 +190,7 @@ extern "C" int mma_check_run(const void* q, const void* k, const void* v, const 
     return 2;
   cudaMemset(err_dev, 0, sizeof(int));
   check_kernel<<<1, 128, smem>>>(tq, tk, tv, tg, cube_t0, cube_h0, cube_w0, cube_head,
-                                 static_cast<const uint16_t*>(p), s1, s2, o, err_dev);
+                                 static_cast<const uint16_t*>(p), s1, s2, o, o2, err_dev);
   if (cudaDeviceSynchronize() != cudaSuccess) return 2;
   int err = 0;
   cudaMemcpy(&err, err_dev, sizeof(int), cudaMemcpyDeviceToHost);

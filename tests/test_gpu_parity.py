@@ -19,7 +19,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # --------------------------------------------- tcgen05 building blocks ----
 def test_tcgen05_building_blocks(cuda_ok):
-    """One S = Q K^T (3-D and 5-D TMA maps), one O = P V (swizzled P, MN-major V)."""
+    """One S = Q K^T (3-D and 5-D TMA maps), one O = P V (swizzled P, MN-major V),
+    and O = P V with P in TMEM."""
     import torch
     lib = ctypes.CDLL(os.path.join(ROOT, "tests", "native", "libmma_check.so"))
     lib.mma_check_run.restype = ctypes.c_int
@@ -28,12 +29,12 @@ def test_tcgen05_building_blocks(cuda_ok):
     q, k, v, p = r(128, 128), r(64, 128), r(64, 128), r(128, 64)
     T, Hg, Wd = 6, 5, 9
     grid = r(T, Hg, Wd, 2, 128)
-    s1, s2, o = (torch.zeros(128, n, device="cuda") for n in (64, 64, 128))
+    s1, s2, o, o2 = (torch.zeros(128, n, device="cuda") for n in (64, 64, 128, 128))
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     t0, h0, w0, head = 4, 4, 8, 1           # a cube cut by all three grid edges
     rc = lib.mma_check_run(*(ctypes.c_void_p(x.data_ptr()) for x in (q, k, v, p, grid)),
                            T, Hg, Wd, t0, h0, w0, head,
-                           *(ctypes.c_void_p(x.data_ptr()) for x in (s1, s2, o, err)))
+                           *(ctypes.c_void_p(x.data_ptr()) for x in (s1, s2, o, o2, err)))
     assert rc == 0
     f = lambda x: x.float().cpu()
     assert torch.allclose(f(s1), f(q) @ f(k).T, atol=1e-2, rtol=1e-3)
@@ -42,6 +43,7 @@ def test_tcgen05_building_blocks(cuda_ok):
     cube[: gc.shape[0], : gc.shape[1], : gc.shape[2]] = gc
     assert torch.allclose(f(s2), f(q) @ cube.reshape(64, 128).T, atol=1e-2, rtol=1e-3)
     assert torch.allclose(f(o), f(p) @ f(v), atol=1e-2, rtol=1e-3)
+    assert torch.allclose(f(o2), f(p) @ f(v), atol=1e-2, rtol=1e-3)     # A operand read from TMEM
 
 
 # --------------------------------------------------------- full checks ----
