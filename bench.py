@@ -321,7 +321,8 @@ def run_ours(args):
                           "bytes_per_call": sel_bytes, "ms_per_call": sel_ms},
             "e2e": {"value": world * flop / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-            "gpu_launches": 4 * wl.B * args.steps,
+            # per step: pool, coarse, select; permute, schedule, one attention launch per batch
+            "gpu_launches": (5 + wl.B) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

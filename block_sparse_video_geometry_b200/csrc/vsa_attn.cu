@@ -11,36 +11,36 @@
 //  * Work item = two query tiles of one (batch, head) stacked into a 128-row
 //    tcgen05 tile (M = 128). The key tiles of the item are the union of the two
 //    tiles' key lists; each 128x64 score block is masked per 64-row half for
-//    key tiles that only one of the two tiles selected. Conditioning key tiles
-//    are shared by every query tile, so they run at full M = 128 efficiency.
-//  * Q, K, V are read straight from the natural [B, S, H, 128] layout by TMA
-//    (no multicast): a 3-D map (d, head, token) for 64-token conditioning runs
-//    and a 5-D map (d, head, w, h, t) over the video latent grid whose 4x4x4
-//    box lands a video cube in shared memory in slot order; cubes cut by the
-//    grid edge are zero-filled by the TMA unit and masked in the softmax. Each
-//    64-key step gathers 256 rows of 128 B; a TMA issue occupies its warp for
-//    a few hundred cycles, so K and V have a producer warp each, and two CTAs
-//    per SM keep the TMA unit busy.
-//  * Warp roles per CTA: warp 0 walks the merged key list, loads Q and K and
-//    publishes per-step tile info; warp 1 loads V; warp 2 owns TMEM and issues
-//    tcgen05.mma (S = Q K^T into one of two TMEM score buffers; O += P V with P
-//    read from TMEM); warps 3-6 run the fp32 online softmax (exp2, lazy rescale
-//    of O in TMEM when the running max grows by more than 2^8), write P as bf16
-//    over the score buffer with tcgen05.st, and run the epilogue. About 100 KB
-//    of shared memory and 256 TMEM columns per CTA: two CTAs share an SM so
-//    that one's softmax overlaps the other's tensor work.
+//    key tiles that only one of the two tiles selected, and the rows of the
+//    other tile skip their exp2 work.
+//  * permute_kv_kernel first rewrites K and V tile-major into the workspace,
+//    each 64-token tile of each head one contiguous 16 KB block already in the
+//    128-byte-swizzled layout of the UMMA descriptors, padding slots zero, so
+//    a step's K or V tile arrives with one bulk copy. schedule_kernel writes
+//    every item's key-tile sequence as records, so that the copy warps only
+//    stream records (a copy warp shares its scheduler with a softmax warp, and
+//    every instruction it needs per step delays the copies).
+//  * Two CTAs per SM, each with 256 TMEM columns: O (128), S (64) and P (bf16,
+//    32). P has columns of its own, so S(j + 1) may be computed as soon as the
+//    softmax warps hold S(j) in registers. Q sits in shared memory.
+//  * Every tcgen05 instruction holds its issuing thread for about 46 cycles,
+//    so one warp issues the S MMAs and another the P V MMAs.
+//  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues S
+//    = Q K^T, 3 issues O += P V; 4-7 load each item's Q into shared memory,
+//    run the fp32 online softmax (one thread per row, exp2) and the epilogue.
+//    P is computed against the running max; the exact row max of a step is
+//    only formed when a row's sum of P exceeds 2^8 (then O and the sum are
+//    rescaled and P recomputed), which keeps every P at most 2^8.
 //  * Every wait is bounded: a wait that runs out sets an error word in the
 //    workspace, raises an abort flag that ends the other roles' loops, drains
-//    in-flight TMA and MMA work and frees TMEM before the block exits.
+//    in-flight copies and MMAs and frees TMEM before the block exits.
 
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <climits>
 #include <cmath>
-#include <mutex>
 
 #include "sm100.cuh"
 #include "vsa_internal.h"
@@ -52,15 +52,18 @@ using namespace sm100;
 
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-static_assert(kKStages == kVStages, "the producers share one stage counter");
-constexpr int kInfoSlots = 4;
-constexpr int kThreads = 224;
-constexpr int kWarpK = 0, kWarpV = 1, kWarpMma = 2;   // warps 3..6: softmax / epilogue
+constexpr int kInfoSlots = 8;        // info of step j is rewritten only after O += P(j) V was issued
+constexpr int kThreads = 256;
+constexpr int kWarpK = 0, kWarpV = 1, kWarpS = 2, kWarpPV = 3;   // warps 4..7: Q loads, softmax, epilogue
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;   // P (bf16) overwrites S columns 0..31
-constexpr float kRescaleLog2 = 8.0f;
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);    // S = Q K^T, both K-major
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // O = P V, V is MN-major
+// O: fp32 accumulator; S: fp32 scores of one key tile; P: their bf16 pairs.
+// P has columns of its own, so S(j + 1) may be computed as soon as the scores
+// of step j are in registers.
+constexpr uint32_t kColO = 0, kColS = 128, kColP = 192;
+constexpr uint32_t kTileBytes = 16384;    // one key tile of K or V: [d half 0][d half 1], 64 rows x 128 B
+constexpr float kPSumLimit = 256.0f;     // 2^8: see the softmax step
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // S = Q K^T, both K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // O = P V, V is MN-major
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
 
@@ -73,20 +76,22 @@ struct StageInfo {
 };
 
 struct AttnSmem {
-  uint8_t q[2][128 * 128];             // [d half][128 rows x 128 B], SW128
-  uint8_t k[kKStages][2][64 * 128];    // [stage][d half][64 keys x 128 B], SW128
-  uint8_t v[kVStages][2][64 * 128];
+  uint8_t q[2][128 * 128];             // [d half][128 rows x 128 B], SW128 K-major (rows 64..127: second tile)
+  uint8_t k[kKStages][kTileBytes];
+  uint8_t v[kVStages][kTileBytes];
   StageInfo info[kInfoSlots];
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t info_full[kInfoSlots];
-  uint64_t q_full, q_empty, s_full[2], p_full[2], o_done, o_full, o_empty, drain;
+  uint64_t q_full, s_full, s_free, p_full, pv_done, o_full, drain_s, drain_pv;
   uint32_t tmem_base;
   int abort;
   int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
 };
 
+// Dynamic shared memory starts 1024-byte aligned when a kernel has no static
+// shared memory (the kernel checks), so no alignment slack is requested.
 size_t attn_smem_bytes(int n_cond) {
-  return sizeof(AttnSmem) + sizeof(int2) * static_cast<size_t>(std::max(0, n_cond - 1)) + 1024;
+  return sizeof(AttnSmem) + sizeof(int2) * static_cast<size_t>(std::max(0, n_cond - 1));
 }
 
 struct Geom {
@@ -100,11 +105,18 @@ struct AttnArgs {
   Geom G;
   const int4* origin;        // device tile table (conditioning tiles are read once)
   const int32_t* count;
+  const uint8_t* kv;         // tile-major K/V: ((b * H + h) * n_tiles + tile) * 32 KB, K then V
+  const uint16_t* q;         // batch base of Q, element strides q_ss, q_sh
+  int64_t q_ss, q_sh;
   int32_t H, b, sink, kmax;
   int32_t c0;                // first query tile of the sparse item range
   int32_t np_dense, np_sparse, n_dense_items, n_items;
-  const int32_t* idx;
+  const int32_t* idx;         // selection lists (read by schedule_kernel)
   const int32_t* cnt;
+  const unsigned long long* valid;   // per-tile slot masks
+  int2* sched;               // step records: [b][item][max_steps]
+  int32_t* nsteps;           // steps per (b, item)
+  int32_t max_steps;
   const float* o_coarse;
   const uint16_t* g;
   int64_t g_sb, g_ss, g_sh;
@@ -174,50 +186,6 @@ __device__ __forceinline__ int64_t tile_token(const AttnSmem& sm, const Geom& G,
   return G.video_start + (static_cast<int64_t>(t) * G.Hg + h) * G.W + w;
 }
 
-// One 64x128 tile (two 64-column halves) of Q, K or V into shared memory.
-__device__ __forceinline__ void load_tile(const AttnSmem& sm, const Geom& G, const CUtensorMap* mc,
-                                          const CUtensorMap* mv, int tile, int h, uint32_t dst0,
-                                          uint32_t dst1, uint32_t bar) {
-  if (tile < G.n_cond) {
-    const int tok = sm.cond[tile].x;
-    tma_load_3d(dst0, mc, bar, 0, h, tok);
-    tma_load_3d(dst1, mc, bar, 64, h, tok);
-  } else {
-    int t0, h0, w0;
-    unsigned long long m;
-    video_cube(G, tile - G.n_cond, t0, h0, w0, m);
-    tma_load_5d(dst0, mv, bar, 0, h, w0, h0, t0);
-    tma_load_5d(dst1, mv, bar, 64, h, w0, h0, t0);
-  }
-}
-
-// Ascending list of video ordinals, read 32 at a time by the whole warp with
-// the next chunk prefetched; every lane sees the same sequence.
-struct ListReader {
-  const int32_t* base;
-  int n, pos;
-  int32_t chunk, pre;
-  __device__ __forceinline__ void init(const int32_t* b, int len, int lane) {
-    base = b;
-    n = len;
-    pos = 0;
-    chunk = lane < n ? b[lane] : INT_MAX;
-    pre = 32 + lane < n ? b[32 + lane] : INT_MAX;
-  }
-  __device__ __forceinline__ int32_t peek() const {
-    const int32_t x = __shfl_sync(0xffffffffu, chunk, pos & 31);
-    return pos < n ? x : INT_MAX;
-  }
-  __device__ __forceinline__ void pop(int lane) {
-    ++pos;
-    if ((pos & 31) == 0) {
-      chunk = pre;
-      const int nx = pos + 32 + lane;
-      pre = nx < n ? base[nx] : INT_MAX;
-    }
-  }
-};
-
 __device__ __forceinline__ void raise_abort(AttnSmem& sm, int* err) {
   atomicExch(err, VSA_ERR_TIMEOUT);
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
@@ -236,26 +204,164 @@ __device__ __forceinline__ bool warp_wait(AttnSmem& sm, uint64_t& bar, uint32_t 
   return ok != 0;
 }
 
-// Pairwise tree reductions over 64 values: short dependency chains.
-__device__ __forceinline__ float tree_max64(const float (&x)[64]) {
-  float t[32];
+// Sets the scores of the key slots whose bit in `valid` is clear to -inf.
+__device__ __forceinline__ void mask_invalid(float (&x)[64], unsigned long long valid) {
+  const uint32_t lo = static_cast<uint32_t>(valid), hi = static_cast<uint32_t>(valid >> 32);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) t[i] = fmaxf(x[i], x[i + 32]);
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-  return t[0];
+  for (int i = 0; i < 32; ++i) {
+    x[i] = ((lo >> i) & 1u) ? x[i] : -INFINITY;
+    x[32 + i] = ((hi >> i) & 1u) ? x[32 + i] : -INFINITY;
+  }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tq_c,
-                const __grid_constant__ CUtensorMap tq_v, const __grid_constant__ CUtensorMap tk_c,
-                const __grid_constant__ CUtensorMap tk_v, const __grid_constant__ CUtensorMap tv_c,
-                const __grid_constant__ CUtensorMap tv_v) {
-  extern __shared__ uint8_t smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+// Largest score of a key tile.
+__device__ __forceinline__ float row_max(const float (&x)[64]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = x[i];
+#pragma unroll
+  for (int i = 8; i < 64; ++i) m[i & 7] = fmaxf(m[i & 7], x[i]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// bf16 pairs of P = 2^(x c - ms) for one key tile; returns the fp32 sum of P.
+__device__ __forceinline__ float exp_pass(const float (&x)[64], float c, float ms, uint32_t (&pw)[32]) {
+  float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float p0 = ex2_approx(fmaf(x[2 * i], c, -ms));
+    const float p1 = ex2_approx(fmaf(x[2 * i + 1], c, -ms));
+    ps[i & 3] += p0 + p1;
+    pw[i] = pack_bf16x2(p0, p1);
+  }
+  return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+}
+
+// K and V into tile-major order for the attention kernel:
+//   kv[((b * H + h) * n_tiles + tile) * 32 KB + which * 16 KB + j * 8 KB + r * 128 B + 16 * (c ^ (r & 7))]
+// holds 16-byte chunk c of d-half j of slot r (which = 0 for K, 1 for V), i.e.
+// each 16 KB block is the 128-byte-swizzled K-major layout the UMMA
+// descriptors read; padding slots are zero. Consecutive threads write
+// consecutive 16-byte chunks and read the chunks of one 128-byte row.
+__global__ void __launch_bounds__(256)
+permute_kv_kernel(DevLayout L, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int64_t sb,
+                  int64_t ss, int64_t sh, int H, uint8_t* __restrict__ kv) {
+  const int tile = blockIdx.x, b = blockIdx.y;
+  __shared__ int tok[kTile];
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
+  __syncthreads();
+  const int n = H * 2048;   // (head, tensor, d-half, row, chunk)
+  for (int w = threadIdx.x; w < n; w += blockDim.x) {
+    const int pc = w & 7, r = (w >> 3) & 63, j = (w >> 9) & 1, which = (w >> 10) & 1, h = w >> 11;
+    const int t = tok[r];
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= 0) {
+      const uint16_t* src = (which ? v : k) + b * sb + static_cast<int64_t>(t) * ss + h * sh + j * 64 +
+                            ((pc ^ (r & 7)) << 3);
+      val = __ldg(reinterpret_cast<const uint4*>(src));
+    }
+    uint8_t* dst = kv + ((static_cast<size_t>(b) * H + h) * L.n_tiles + tile) * 32768u + which * 16384 +
+                   j * 8192 + r * 128 + pc * 16;
+    *reinterpret_cast<uint4*>(dst) = val;
+  }
+}
+
+// Step schedule of each work item, built once per call so that the copy warps
+// of the attention kernel only stream records. Record = (key tile, flags):
+// bits 0-1 which of the item's query tiles list the key tile, bit 4 last step
+// of the item, bit 5 the key tile has padding slots. Key tiles come in the
+// item's order: the dense part (conditioning tiles, or all tiles for dense
+// rows), then the union of the two selection lists, ascending.
+// One warp per item; the union is formed with bitmaps in shared memory.
+constexpr int kSchedWarps = 4;
+
+size_t sched_smem_per_warp(int n_tiles, int n_video) {
+  return align_up(static_cast<size_t>(2 * ((n_video + 31) / 32)) * 4 + static_cast<size_t>(n_tiles) * 5, 16);
+}
+
+__global__ void __launch_bounds__(kSchedWarps * 32) schedule_kernel(const __grid_constant__ AttnArgs a,
+                                                                     int per_warp_bytes) {
+  extern __shared__ __align__(16) uint8_t sh[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x * kSchedWarps + warp;
+  const int b = blockIdx.y;
+  if (item >= a.n_items) return;
+  const Geom& G = a.G;
+  const Item it = decode_item(a, item);
+  const int nw = (G.n_video + 31) / 32;
+  uint32_t* bma = reinterpret_cast<uint32_t*>(sh + warp * per_warp_bytes);
+  uint32_t* bmb = bma + nw;
+  int32_t* tl = reinterpret_cast<int32_t*>(bmb + nw);
+  uint8_t* mk = reinterpret_cast<uint8_t*>(tl + G.n_tiles);
+  const int both = it.qb >= 0 ? 3 : 1;
+  const int n_dense = it.dense ? G.n_tiles : G.n_cond;
+  for (int i = lane; i < n_dense; i += 32) {
+    tl[i] = i;
+    mk[i] = static_cast<uint8_t>(both);
+  }
+  int total = n_dense;
+  if (!it.dense) {
+    for (int w = lane; w < nw; w += 32) bma[w] = bmb[w] = 0u;
+    __syncwarp();
+    const size_t row = (static_cast<size_t>(b) * a.H + it.h) * G.n_tiles;
+    // entries outside [0, n_video) (never written by vsa_coarse_select) are skipped
+    const int na = min(a.cnt[row + it.qa], a.kmax);
+    for (int i = lane; i < na; i += 32) {
+      const int t = a.idx[(row + it.qa) * a.kmax + i];
+      if (static_cast<unsigned>(t) < static_cast<unsigned>(G.n_video)) atomicOr(&bma[t >> 5], 1u << (t & 31));
+    }
+    if (it.qb >= 0) {
+      const int nb = min(a.cnt[row + it.qb], a.kmax);
+      for (int i = lane; i < nb; i += 32) {
+        const int t = a.idx[(row + it.qb) * a.kmax + i];
+        if (static_cast<unsigned>(t) < static_cast<unsigned>(G.n_video)) atomicOr(&bmb[t >> 5], 1u << (t & 31));
+      }
+    }
+    __syncwarp();
+    // each lane owns a contiguous range of bitmap words; a warp scan gives its output offset
+    const int wpl = (nw + 31) / 32, w0 = min(nw, lane * wpl), w1 = min(nw, w0 + wpl);
+    int mine = 0;
+    for (int w = w0; w < w1; ++w) mine += __popc(bma[w] | bmb[w]);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = n_dense + incl - mine;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t u = bma[w] | bmb[w];
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1u;
+        tl[pos] = G.n_cond + w * 32 + bit;
+        mk[pos] = static_cast<uint8_t>(((bma[w] >> bit) & 1u) | (((bmb[w] >> bit) & 1u) << 1));
+        ++pos;
+      }
+    }
+    total = n_dense + __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  const int n_steps = total;
+  int2* rec = a.sched + (static_cast<size_t>(b) * a.n_items + item) * a.max_steps;
+  for (int r = lane; r < n_steps; r += 32) {
+    const int t = tl[r];
+    uint32_t fl = mk[r];
+    if (r == n_steps - 1) fl |= 16u;
+    if (a.valid[t] != ~0ull) fl |= 32u;
+    rec[r] = make_int2(t, static_cast<int>(fl));
+  }
+  if (lane == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = n_steps;
+}
+
+// 128 registers per thread: two CTAs of 256 threads fit one SM's register file.
+__global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {          // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
+    return;
+  }
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Geom& G = a.G;
 
@@ -271,27 +377,18 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
       mbar_init(smem_u32(&sm.v_empty[s]), 1);
     }
     for (int s = 0; s < kInfoSlots; ++s) mbar_init(smem_u32(&sm.info_full[s]), 1);
-    mbar_init(smem_u32(&sm.q_full), 1);
-    mbar_init(smem_u32(&sm.q_empty), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.p_full[i]), 4);     // one arrival per softmax warp
-    }
-    mbar_init(smem_u32(&sm.o_done), 1);
+    mbar_init(smem_u32(&sm.q_full), 4);          // one arrival per softmax warp
+    mbar_init(smem_u32(&sm.s_full), 1);
+    mbar_init(smem_u32(&sm.s_free), 4);
+    mbar_init(smem_u32(&sm.p_full), 4);
+    mbar_init(smem_u32(&sm.pv_done), 1);
     mbar_init(smem_u32(&sm.o_full), 1);
-    mbar_init(smem_u32(&sm.o_empty), 4);
-    mbar_init(smem_u32(&sm.drain), 1);
+    mbar_init(smem_u32(&sm.drain_s), 1);
+    mbar_init(smem_u32(&sm.drain_pv), 1);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    for (const CUtensorMap* m : {&tq_c, &tq_v, &tk_c, &tk_v}) tma_prefetch_desc(m);
-  }
-  if (warp == kWarpV && lane == 0) {
-    tma_prefetch_desc(&tv_c);
-    tma_prefetch_desc(&tv_v);
-  }
-  if (warp == kWarpMma) {
+  if (warp == kWarpS) {
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -302,258 +399,266 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
 
   if (warp == kWarpK || warp == kWarpV) {
     // ----------------------------------------------------------- producers
-    // Both producer warps walk the same key list; the K warp also loads Q and
-    // publishes the per-step tile info.
+    // Both stream the item's step records (one key tile each) and copy the
+    // tile's 16 KB block of K or V; the K warp also publishes per-step info.
     const bool is_k = warp == kWarpK;
-    const CUtensorMap* mc = is_k ? &tk_c : &tv_c;
-    const CUtensorMap* mv = is_k ? &tk_v : &tv_v;
     uint64_t* full = is_k ? sm.k_full : sm.v_full;
     uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
+    const int nst = is_k ? kKStages : kVStages;
     uint32_t step = 0, issued = 0;
-    int it_n = 0, q_loads = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
-      const Item it = decode_item(a, item);
-      if (is_k) {
-        if (!(ok = warp_wait(sm, sm.q_empty, (it_n & 1) ^ 1, lane, a.err))) break;
+    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+      const size_t bi = static_cast<size_t>(a.b) * a.n_items + item;
+      const int2* rec = a.sched + bi * a.max_steps;
+      const int n = a.nsteps[bi];
+      const int h = decode_item(a, item).h;
+      const uint8_t* head_kv = a.kv + (static_cast<size_t>(a.b) * a.H + h) * G.n_tiles * 32768u + (is_k ? 0u : 16384u);
+      // records 32 at a time, one per lane, the next 32 prefetched
+      int2 cur = lane < n ? rec[lane] : make_int2(0, 0);
+      int2 nxt = 32 + lane < n ? rec[32 + lane] : make_int2(0, 0);
+      for (int jj = 0; jj < n; ++jj) {
+        if (jj > 0 && (jj & 31) == 0) {
+          cur = nxt;
+          nxt = jj + 32 + lane < n ? rec[jj + 32 + lane] : make_int2(0, 0);
+        }
+        const int tile = __shfl_sync(0xffffffffu, cur.x, jj & 31);
+        const int fl = __shfl_sync(0xffffffffu, cur.y, jj & 31);
+        const int st = step % nst;
+        if (!(ok = warp_wait(sm, empty[st], ((step / nst) & 1) ^ 1, lane, a.err))) break;
         if (lane == 0) {
-          const uint32_t bar = smem_u32(&sm.q_full);
-          mbar_arrive_expect_tx(bar, (it.qb >= 0 ? 2u : 1u) * 16384u);
-          load_tile(sm, G, &tq_c, &tq_v, it.qa, it.h, smem_u32(sm.q[0]), smem_u32(sm.q[1]), bar);
-          if (it.qb >= 0)
-            load_tile(sm, G, &tq_c, &tq_v, it.qb, it.h, smem_u32(sm.q[0] + 8192),
-                      smem_u32(sm.q[1] + 8192), bar);
-        }
-        ++q_loads;
-      }
-      const int both = it.qb >= 0 ? 3 : 1;
-      const int n_dense = it.dense ? G.n_tiles : G.n_cond;
-      ListReader la, lb;
-      const size_t row = (static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles;
-      const int na = it.dense ? 0 : a.cnt[row + it.qa];
-      const int nb = (it.dense || it.qb < 0) ? 0 : a.cnt[row + it.qb];
-      la.init(a.idx + (row + it.qa) * a.kmax, na, lane);
-      lb.init(a.idx + (row + (it.qb >= 0 ? it.qb : it.qa)) * a.kmax, nb, lane);
-      int j = 0;
-      // next key tile of the item: the dense part first, then the merged lists
-      auto next = [&](int& tile, int& mask) -> bool {
-        if (j < n_dense) {
-          tile = j++;
-          mask = both;
-          return true;
-        }
-        const int32_t x0 = la.peek(), y0 = lb.peek();
-        if (x0 == INT_MAX && y0 == INT_MAX) return false;
-        const int32_t t = min(x0, y0);
-        mask = (x0 == t ? 1 : 0) | (y0 == t ? 2 : 0);
-        if (x0 == t) la.pop(lane);
-        if (y0 == t) lb.pop(lane);
-        tile = G.n_cond + t;
-        return true;
-      };
-      int tile, mask, ntile, nmask;
-      bool have = next(tile, mask);
-      while (have) {
-        const bool more = next(ntile, nmask);
-        const int st = step % kKStages;
-        if (!(ok = warp_wait(sm, empty[st], ((step / kKStages) & 1) ^ 1, lane, a.err))) break;
-        if (is_k && lane == 0) {
-          StageInfo& inf = sm.info[step % kInfoSlots];
-          inf.tile = tile;
-          inf.mask = mask;
-          inf.last = more ? 0 : 1;
-          inf.valid = tile_mask(sm, G, tile);
-          mbar_arrive(smem_u32(&sm.info_full[step % kInfoSlots]));
-        }
-        if (lane == 0) {
-          uint8_t (*buf)[64 * 128] = is_k ? sm.k[st] : sm.v[st];
-          mbar_arrive_expect_tx(smem_u32(&full[st]), 16384u);
-          load_tile(sm, G, mc, mv, tile, it.h, smem_u32(buf[0]), smem_u32(buf[1]), smem_u32(&full[st]));
+          if (is_k) {
+            StageInfo& inf = sm.info[step % kInfoSlots];
+            inf.tile = tile;
+            inf.mask = fl & 3;
+            inf.last = (fl >> 4) & 1;
+            inf.valid = (fl & 32) ? a.valid[tile] : ~0ull;
+            mbar_arrive(smem_u32(&sm.info_full[step % kInfoSlots]));
+          }
+          const uint32_t bar = smem_u32(&full[st]);
+          mbar_arrive_expect_tx(bar, kTileBytes);
+          bulk_load(smem_u32(is_k ? sm.k[st] : sm.v[st]), head_kv + static_cast<size_t>(tile) * 32768u, kTileBytes,
+                    bar);
         }
         __syncwarp();
         ++issued;
         ++step;
-        tile = ntile;
-        mask = nmask;
-        have = more;
       }
     }
     if (!ok && lane == 0) {
-      // let every issued TMA load land before the block can exit: the last
-      // fill of each stage, and the last Q load
-      for (uint32_t i = (issued > kKStages ? issued - kKStages : 0); i < issued; ++i)
-        mbar_wait(smem_u32(&full[i % kKStages]), (i / kKStages) & 1, nullptr, kDrainNs);
-      if (is_k && q_loads > 0) mbar_wait(smem_u32(&sm.q_full), (q_loads - 1) & 1, nullptr, kDrainNs);
+      // let every issued copy land before the block can exit
+      for (uint32_t i = (issued > static_cast<uint32_t>(nst) ? issued - nst : 0); i < issued; ++i)
+        mbar_wait(smem_u32(&full[i % nst]), (i / nst) & 1, nullptr, kDrainNs);
     }
-  } else if (warp == kWarpMma) {
-    // ----------------------------------------------------------------- MMA
+  } else if (warp == kWarpS) {
+    // ------------------------------------------------------ S = Q K^T issuer
+    // S(j) may overwrite the score columns once the softmax warps have read
+    // S(j - 1) into registers (s_free); Q of an item is in shared memory once
+    // q_full completes.
     bool ok = true;
     if (lane == 0) {
-      uint32_t step = 0;
+      uint32_t j = 0;
       int it_n = 0;
-      auto pv = [&](uint32_t st, bool first) -> bool {
-        if (!mbar_wait(smem_u32(&sm.p_full[st & 1]), (st >> 1) & 1, &sm.abort, kTimeoutNs)) return false;
-        if (first && !mbar_wait(smem_u32(&sm.o_empty), (it_n & 1) ^ 1, &sm.abort, kTimeoutNs)) return false;
-        const int vs = st % kVStages;
-        if (!mbar_wait(smem_u32(&sm.v_full[vs]), (st / kVStages) & 1, &sm.abort, kTimeoutNs)) return false;
-        tc_fence_after();
-        const uint32_t pcol = tmem + ((st & 1) ? kColS1 : kColS0);
-        const uint32_t vbase = smem_u32(sm.v[vs][0]);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
-          umma_ts(tmem + kColO, pcol + kk * 8, bd, kIdescPV, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(smem_u32(&sm.v_empty[vs]));
-        umma_commit(smem_u32(&sm.o_done));
-        return true;
-      };
+      const uint64_t qd = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
         if (!(ok = mbar_wait(smem_u32(&sm.q_full), it_n & 1, &sm.abort, kTimeoutNs))) break;
-        int j = 0;
         bool last = false;
         while (!last) {
-          const int ks = step % kKStages;
-          if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (step / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
+          const int ks = j % kKStages;
+          if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (j / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
+          if (j > 0 && !(ok = mbar_wait(smem_u32(&sm.s_free), (j - 1) & 1, &sm.abort, kTimeoutNs))) break;
           tc_fence_after();
-          last = sm.info[step % kInfoSlots].last != 0;
-          const uint32_t qbase = smem_u32(sm.q[0]);
-          const uint32_t kbase = smem_u32(sm.k[ks][0]);
-          const uint32_t dS = tmem + ((step & 1) ? kColS1 : kColS0);
+          last = sm.info[j % kInfoSlots].last != 0;
+          const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk & 3) * 32;   // 16 bf16 = 32 B K step inside a swizzle row
-            const uint64_t ad = smem_desc_sw128(qbase + (kk >> 2) * 16384 + off, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * 8192 + off, 16, 1024);
-            umma_ss(dS, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+            // 16 d per K step: 32 B inside a swizzle row of d half kk / 4
+            // (descriptor addresses count 16-byte units)
+            umma_ss(tmem + kColS, qd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2,
+                    kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS, kk > 0 ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm.k_empty[ks]));
-          umma_commit(smem_u32(&sm.s_full[step & 1]));
-          if (last) umma_commit(smem_u32(&sm.q_empty));
-          if (j > 0 && !(ok = pv(step - 1, j == 1))) break;
+          umma_commit(smem_u32(&sm.s_full));
           ++j;
-          ++step;
+        }
+      }
+      if (!ok) raise_abort(sm, a.err);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      umma_commit(smem_u32(&sm.drain_s));
+      mbar_wait(smem_u32(&sm.drain_s), 0, nullptr, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp == kWarpPV) {
+    // ----------------------------------------------------- O += P V issuer
+    // The first step of an item overwrites O; o_full fires after its last step.
+    bool ok = true;
+    if (lane == 0) {
+      uint32_t j = 0;
+      for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+        bool first = true, last = false;
+        while (!last) {
+          if (!(ok = mbar_wait(smem_u32(&sm.p_full), j & 1, &sm.abort, kTimeoutNs))) break;
+          last = sm.info[j % kInfoSlots].last != 0;   // read by the softmax warps before p_full
+          const int vs = j % kVStages;
+          if (!(ok = mbar_wait(smem_u32(&sm.v_full[vs]), (j / kVStages) & 1, &sm.abort, kTimeoutNs))) break;
+          tc_fence_after();
+          // V as MN-major B: 64-d blocks 8 KB apart, 16 keys = 2 KB per K step
+          const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[vs]), 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + kColO, tmem + kColP + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
+                    (first && kk == 0) ? 0u : 1u);
+          first = false;
+          umma_commit(smem_u32(&sm.v_empty[vs]));
+          umma_commit(smem_u32(&sm.pv_done));
+          ++j;
         }
         if (!ok) break;
-        if (!(ok = pv(step - 1, j == 1))) break;
         umma_commit(smem_u32(&sm.o_full));
       }
       if (!ok) raise_abort(sm, a.err);
-      // drain: every MMA issued so far has completed before TMEM is freed
-      umma_commit(smem_u32(&sm.drain));
-      mbar_wait(smem_u32(&sm.drain), 0, nullptr, kDrainNs);
+      umma_commit(smem_u32(&sm.drain_pv));
+      mbar_wait(smem_u32(&sm.drain_pv), 0, nullptr, kDrainNs);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------ softmax / epilogue
-    const int quad = warp & 3;              // TMEM lane quadrant of this warp
-    const int r = quad * 32 + lane;         // row of the 128-row tile
-    const int half = r >> 6;                // 0: first query tile, 1: second
+    // ------------------------------------------------ Q / softmax / epilogue
+    // One thread per row of the 128-row tile.
+    const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;                  // row of the 128-row tile
+    const int half = r >> 6;                         // 0: first query tile, 1: second
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float c = a.scale_log2;
-    uint32_t step = 0;
+    uint32_t j = 0;
     int it_n = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
       const Item it = decode_item(a, item);
+      const int qt = half ? it.qb : it.qa;
+      const int slot = r & 63;
+      const bool row_ok = qt >= 0 && ((tile_mask(sm, G, qt) >> slot) & 1ull);
+      const int64_t tok = row_ok ? tile_token(sm, G, qt, slot) : 0;
+      {
+        // this row's Q into shared memory, 128-byte swizzled (every MMA of the
+        // previous item has completed)
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + tok * a.q_ss + it.h * a.q_sh);
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          uint4 w[8];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) w[cc] = row_ok ? __ldg(src + hq * 8 + cc) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+            *reinterpret_cast<uint4*>(&sm.q[hq][r * 128 + ((cc ^ (r & 7)) << 4)]) = w[cc];
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.q_full));
+      }
       float ms = -INFINITY, l = 0.f;        // running max (scaled, log2 domain) and sum
       bool last = false;
+      // barrier phases of the next step are tested (without blocking) early in
+      // a step and read after its exp2 work, so that their latency is hidden
+      bool have_next = false, s_ready = false;
+      StageInfo next{};
       while (!last) {
-        if (!(ok = warp_wait(sm, sm.info_full[step % kInfoSlots], (step / kInfoSlots) & 1, lane, a.err))) break;
-        const StageInfo inf = sm.info[step % kInfoSlots];
+        StageInfo inf;
+        if (have_next) {
+          inf = next;
+        } else {
+          if (!(ok = warp_wait(sm, sm.info_full[j % kInfoSlots], (j / kInfoSlots) & 1, lane, a.err))) break;
+          inf = sm.info[j % kInfoSlots];
+        }
         last = inf.last != 0;
-        if (!(ok = warp_wait(sm, sm.s_full[step & 1], (step >> 1) & 1, lane, a.err))) break;
+        const bool act = (inf.mask >> half) & 1;     // the same for the whole warp
+        if (!s_ready && !(ok = warp_wait(sm, sm.s_full, j & 1, lane, a.err))) break;
         tc_fence_after();
-        const uint32_t scol = lane_addr + ((step & 1) ? kColS1 : kColS0);
+        uint32_t t_info = 0, t_s = 0, t_pv = 1;
+        if (!last) {
+          t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
+          t_s = mbar_test_wait(smem_u32(&sm.s_full), (j + 1) & 1);
+        }
+        if (j > 0) t_pv = mbar_test_wait(smem_u32(&sm.pv_done), (j - 1) & 1);
         uint32_t pw[32];
-        if ((inf.mask >> half) & 1) {
-          float x[64];
-          {
-            uint32_t u0[32], u1[32];
-            tmem_ld32(scol, u0);
-            tmem_ld32(scol + 32, u1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              x[i] = __uint_as_float(u0[i]);
-              x[32 + i] = __uint_as_float(u1[i]);
-            }
-          }
-          if (inf.valid != ~0ull) {           // partial tile: padded keys never attend
-            const uint32_t lo = static_cast<uint32_t>(inf.valid), hi = static_cast<uint32_t>(inf.valid >> 32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              x[i] = ((lo >> i) & 1u) ? x[i] : -INFINITY;
-              x[32 + i] = ((hi >> i) & 1u) ? x[32 + i] : -INFINITY;
-            }
-          }
-          const float mt = tree_max64(x) * c;
-          const bool need = ms != -INFINITY && mt > ms + kRescaleLog2;
-          if (ms == -INFINITY) ms = mt;       // first key tile of this row: O and l are still zero
-          if (__any_sync(0xffffffffu, need)) {
-            // rescale this warp's rows of O once the previous P V has landed
-            if (!(ok = warp_wait(sm, sm.o_done, (step - 1) & 1, lane, a.err))) break;
-            tc_fence_after();
-            const float f = need ? ex2_approx(ms - mt) : 1.0f;
+        float x[64];
+        if (act) tmem_ld64f(lane_addr + kColS, x);
+        tmem_wait_ld();
+        // the scores are in registers: S(j + 1) may overwrite them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.s_free));
+        if (act) {
+          if (inf.valid != ~0ull) mask_invalid(x, inf.valid);   // padding slots never attend
+          // exact row max of the step; O and l rescaled when it raises the running max
+          auto exact_max = [&]() -> bool {
+            const float mt = row_max(x) * c;
+            const bool need = ms != -INFINITY && mt > ms;
+            if (ms == -INFINITY) ms = mt;     // first key tile of this row: O and l are still zero
+            if (__any_sync(0xffffffffu, need)) {
+              // rescale this row of O once the previous P V has landed
+              if (j > 0 && !warp_wait(sm, sm.pv_done, (j - 1) & 1, lane, a.err)) return false;
+              tc_fence_after();
+              const float f = need ? ex2_approx(ms - mt) : 1.0f;
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-              uint32_t u[32];
-              tmem_ld32(lane_addr + kColO + ch * 32, u);
-              tmem_wait_ld();
+              for (int ch = 0; ch < 4; ++ch) {
+                uint32_t u[32];
+                tmem_ld32(lane_addr + kColO + 32 * ch, u);
+                tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * f);
-              tmem_st32(lane_addr + kColO + ch * 32, u);
+                for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * f);
+                tmem_st32(lane_addr + kColO + 32 * ch, u);
+              }
+              tmem_wait_st();
+              if (need) {
+                l *= f;
+                ms = mt;
+              }
             }
-            tmem_wait_st();
-            if (need) {
-              l *= f;
-              ms = mt;
-            }
+            return true;
+          };
+          // P against the running max ms. The softmax does not depend on that
+          // reference as long as no P is large, so the exact row max of the step
+          // is only formed when a row has no reference yet, or when its P sum
+          // exceeds 2^8 (then every P was at most 2^8: fine for bf16 and fp32).
+          if (__any_sync(0xffffffffu, ms == -INFINITY) && !(ok = exact_max())) break;
+          float psum = exp_pass(x, c, ms, pw);
+          if (__any_sync(0xffffffffu, psum > kPSumLimit)) {
+            if (!(ok = exact_max())) break;
+            psum = exp_pass(x, c, ms, pw);   // every P <= 1 now
           }
-          float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2_approx(fmaf(x[2 * i], c, -ms));
-            const float p1 = ex2_approx(fmaf(x[2 * i + 1], c, -ms));
-            ps[i & 3] += p0 + p1;
-            pw[i] = pack_bf16x2(p0, p1);
-          }
-          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+          l += psum;
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) pw[i] = 0u;     // rows of the other query tile
         }
-        tmem_st32(scol, pw);
+        // P of step j - 1 has been consumed once its P V completed
+        if (j > 0 && !__all_sync(0xffffffffu, t_pv) && !(ok = warp_wait(sm, sm.pv_done, (j - 1) & 1, lane, a.err)))
+          break;
+        tc_fence_after();
+        tmem_st32(lane_addr + kColP, pw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[step & 1]));
-        ++step;
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full));
+        have_next = !last && __all_sync(0xffffffffu, t_info);
+        if (have_next) next = sm.info[(j + 1) % kInfoSlots];
+        s_ready = !last && __all_sync(0xffffffffu, t_s);
+        ++j;
       }
       if (!ok) break;
       // epilogue: out = O / l + g * o_coarse
       if (!(ok = warp_wait(sm, sm.o_full, it_n & 1, lane, a.err))) break;
       tc_fence_after();
-      const int qt = half ? it.qb : it.qa;
-      const int slot = r & 63;
-      bool row_ok = qt >= 0;
-      int64_t tok = 0;
+      const float inv_l = 1.0f / l;
       float gate = 0.f;
       const float* oc = nullptr;
-      if (row_ok) row_ok = (tile_mask(sm, G, qt) >> slot) & 1ull;
-      if (row_ok) {
-        tok = tile_token(sm, G, qt, slot);
-        const bool coarse = !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && qt < G.n_cond);
-        if (coarse) {
-          gate = __uint_as_float(static_cast<uint32_t>(a.g[a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh]) << 16);
-          oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + qt) * kHeadDim;
-        }
+      if (row_ok && !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && qt < G.n_cond)) {
+        gate = __uint_as_float(static_cast<uint32_t>(a.g[a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh]) << 16);
+        oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + qt) * kHeadDim;
       }
-      const float inv_l = 1.0f / l;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t u[32];
-        tmem_ld32(lane_addr + kColO + ch * 32, u);
+        tmem_ld32(lane_addr + kColO + 32 * ch, u);
         tmem_wait_ld();
         if (row_ok) {
           float y[32];
@@ -584,65 +689,18 @@ vsa_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUte
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty));
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kWarpS) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 3-D map (d, head, token) over a [S, H, 128] bf16 slab; box 64 x 1 x 64.
-bool make_cond_map(CUtensorMap* m, const void* base, int64_t S, int H, int64_t ss, int64_t sh) {
-  auto enc = get_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H),
-                        static_cast<cuuint64_t>(S)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(sh * 2), static_cast<cuuint64_t>(ss * 2)};
-  cuuint32_t box[3] = {64, 1, 64};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 5-D map (d, head, w, h, t) over the video latent grid; box 64 x 1 x 4 x 4 x 4.
-bool make_video_map(CUtensorMap* m, const void* base, int T, int Hg, int W, int H, int64_t ss,
-                    int64_t sh) {
-  auto enc = get_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[5] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H),
-                        static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(Hg),
-                        static_cast<cuuint64_t>(T)};
-  cuuint64_t strides[4] = {static_cast<cuuint64_t>(sh * 2), static_cast<cuuint64_t>(ss * 2),
-                           static_cast<cuuint64_t>(ss * 2 * W),
-                           static_cast<cuuint64_t>(ss * 2 * W * Hg)};
-  cuuint32_t box[5] = {64, 1, 4, 4, 4};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -650,8 +708,43 @@ int sm_count() {
   return n;
 }
 
-constexpr size_t kAttnWorkspace = 256;   // error word
+constexpr size_t kAttnHeader = 256;   // error word
 constexpr size_t kMaxAttnSmem = 227 * 1024;
+
+// Work decomposition shared by the host and the kernels (see decode_item).
+struct ItemCounts {
+  int32_t c0, np_dense, np_sparse, n_dense_items, n_items, max_steps;
+};
+
+ItemCounts item_counts(const vsa_layout* L, int H, const vsa_params* p, int32_t kmax) {
+  ItemCounts c{};
+  const bool rows = p->sink == VSA_SINK_EXACT_KV_AND_ROWS;
+  c.c0 = rows ? L->n_cond : 0;
+  c.np_dense = rows ? (L->n_cond + 1) / 2 : 0;
+  c.np_sparse = (L->n_tiles - c.c0 + 1) / 2;
+  c.n_dense_items = c.np_dense * H;
+  c.n_items = c.n_dense_items + c.np_sparse * H;
+  const int sparse_tiles = L->n_cond + std::min(2 * kmax, L->n_video);
+  c.max_steps = std::max(rows ? L->n_tiles : 0, sparse_tiles);
+  return c;
+}
+
+// [error word][tile-major K/V][step records][steps per item]
+struct AttnWorkspace {
+  size_t kv, sched, nsteps, total;
+};
+
+AttnWorkspace attn_workspace(const vsa_layout* L, int B, int H, const vsa_params* p) {
+  int32_t kmax = 0;
+  vsa_select_kmax(L, p, &kmax);
+  const ItemCounts c = item_counts(L, H, p, kmax);
+  AttnWorkspace w{};
+  w.kv = kAttnHeader;
+  w.sched = w.kv + static_cast<size_t>(B) * H * L->n_tiles * 32768u;
+  w.nsteps = w.sched + align_up(static_cast<size_t>(B) * c.n_items * c.max_steps * sizeof(int2), 256);
+  w.total = w.nsteps + align_up(static_cast<size_t>(B) * c.n_items * sizeof(int32_t), 256);
+  return w;
+}
 
 }  // namespace
 }  // namespace vsa
@@ -665,7 +758,7 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* L, int32_t B, int32_
   if (!L || !bytes || B <= 0 || H <= 0) return VSA_ERR_INVALID_ARG;
   vsa_status st = check_params(p);
   if (st != VSA_OK) return st;
-  *bytes = kAttnWorkspace;
+  *bytes = attn_workspace(L, B, H, p).total;
   return VSA_OK;
 }
 
@@ -690,13 +783,14 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
     return VSA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(o_coarse) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
     return VSA_ERR_INVALID_ARG;
-  if (workspace_bytes < kAttnWorkspace) return VSA_ERR_WORKSPACE_TOO_SMALL;
+  const AttnWorkspace ws = attn_workspace(L, B, H, p);
+  if (workspace_bytes < ws.total) return VSA_ERR_WORKSPACE_TOO_SMALL;
   if (!L->dev_buf) return VSA_ERR_NOT_UPLOADED;
   int32_t want_kmax = 0;
   vsa_select_kmax(L, p, &want_kmax);
   if (kmax != want_kmax) return VSA_ERR_INVALID_ARG;
   const size_t smem = attn_smem_bytes(L->n_cond);
-  if (smem > kMaxAttnSmem) return VSA_ERR_UNSUPPORTED;   // more than ~16k conditioning tiles
+  if (smem > kMaxAttnSmem) return VSA_ERR_UNSUPPORTED;   // thousands of conditioning tiles
   const int n_sm = sm_count();
   if (n_sm <= 0) return cuda_fail("vsa_sparse_attn_fwd: no current CUDA device");
 
@@ -714,15 +808,19 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.G.video_start = L->video_start;
   a.origin = D.origin;
   a.count = D.count;
+  a.q_ss = ss;
+  a.q_sh = sh;
   a.H = H;
   a.sink = p->sink;
   a.kmax = kmax;
-  const bool rows = p->sink == VSA_SINK_EXACT_KV_AND_ROWS;
-  a.c0 = rows ? L->n_cond : 0;
-  a.np_dense = rows ? (L->n_cond + 1) / 2 : 0;
-  a.np_sparse = (L->n_tiles - a.c0 + 1) / 2;
-  a.n_dense_items = a.np_dense * H;
-  a.n_items = a.n_dense_items + a.np_sparse * H;
+  const ItemCounts ic = item_counts(L, H, p, kmax);
+  a.c0 = ic.c0;
+  a.np_dense = ic.np_dense;
+  a.np_sparse = ic.np_sparse;
+  a.n_dense_items = ic.n_dense_items;
+  a.n_items = ic.n_items;
+  a.max_steps = ic.max_steps;
+  a.valid = D.valid;
   a.idx = idx;
   a.cnt = cnt;
   a.o_coarse = o_coarse;
@@ -741,33 +839,31 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   cudaError_t e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
-  // Two CTAs per SM when their shared memory fits (TMEM holds two 256-column
-  // CTAs); registers are bounded for two by __launch_bounds__.
-  int dev = 0, smem_sm = 0, smem_resv = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-  cudaDeviceGetAttribute(&smem_resv, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-  const int per_sm = 2 * (smem + smem_resv) <= static_cast<size_t>(smem_sm) ? 2 : 1;
-  e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute(carveout)", e);
-  e = cudaMemsetAsync(workspace, 0, kAttnWorkspace, stream);
+  e = cudaMemsetAsync(workspace, 0, kAttnHeader, stream);
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaMemsetAsync", e);
-  const int grid = std::max(1, std::min(a.n_items, n_sm * per_sm));
-  const uint16_t* qq = static_cast<const uint16_t*>(q);
-  const uint16_t* kk = static_cast<const uint16_t*>(k);
-  const uint16_t* vv = static_cast<const uint16_t*>(v);
+  const int grid = std::max(1, std::min(a.n_items, 2 * n_sm));   // two CTAs per SM, 256 TMEM columns each
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  a.kv = wsb + ws.kv;
+  a.sched = reinterpret_cast<int2*>(wsb + ws.sched);
+  a.nsteps = reinterpret_cast<int32_t*>(wsb + ws.nsteps);
+  permute_kv_kernel<<<dim3(L->n_tiles, B), 256, 0, stream>>>(D, static_cast<const uint16_t*>(k),
+                                                            static_cast<const uint16_t*>(v), sb, ss, sh, H,
+                                                            wsb + ws.kv);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: permute launch", e);
+  const size_t per_warp = sched_smem_per_warp(L->n_tiles, L->n_video);
+  if (per_warp * kSchedWarps > kMaxAttnSmem) return VSA_ERR_UNSUPPORTED;
+  e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(per_warp * kSchedWarps));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
+  schedule_kernel<<<dim3((a.n_items + kSchedWarps - 1) / kSchedWarps, B), kSchedWarps * 32, per_warp * kSchedWarps,
+                    stream>>>(a, static_cast<int>(per_warp));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: schedule launch", e);
   for (int b = 0; b < B; ++b) {
-    CUtensorMap m[6];
-    const int64_t vo = L->video_start * ss;
-    const uint16_t* bases[3] = {qq + b * sb, kk + b * sb, vv + b * sb};
-    for (int t = 0; t < 3; ++t) {
-      if (!make_cond_map(&m[2 * t], bases[t], L->seq_len, H, ss, sh))
-        return cuda_fail("vsa_sparse_attn_fwd: cuTensorMapEncodeTiled (token map)");
-      if (!make_video_map(&m[2 * t + 1], bases[t] + vo, L->grid_t, L->grid_h, L->grid_w, H, ss, sh))
-        return cuda_fail("vsa_sparse_attn_fwd: cuTensorMapEncodeTiled (video grid map)");
-    }
     a.b = b;
-    vsa_attn_kernel<<<grid, kThreads, smem, stream>>>(a, m[0], m[1], m[2], m[3], m[4], m[5]);
+    a.q = static_cast<const uint16_t*>(q) + b * sb;
+    vsa_attn_kernel<<<grid, kThreads, smem, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: launch", e);
   }

@@ -143,7 +143,9 @@ def test_calls_validate_before_any_gpu_work():
                                  None) == vsa.ERR_INVALID_ARG
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_BF16, S * 256, 256, 129, fake,
                                  256, None) == vsa.ERR_INVALID_ARG
+    ws = lay.sparse_attn_workspace_size(1, 2, good)
+    assert ws >= 256 + 2 * lay.info.n_tiles * 32768          # error word + tile-major K/V
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
-                                 16, None) == vsa.ERR_WORKSPACE_TOO_SMALL
+                                 ws - 16, None) == vsa.ERR_WORKSPACE_TOO_SMALL
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
-                                 256, None) == vsa.ERR_NOT_UPLOADED
+                                 ws, None) == vsa.ERR_NOT_UPLOADED
