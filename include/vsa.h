@@ -259,8 +259,8 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* layout, int32_t B, i
  *                     all written by the call before use: an error word; a
  *                     tile-major copy of K and V (32 KB per (batch, head,
  *                     tile); 1.64 GB for the 24-head 133,696-token shape); the
- *                     key-tile schedule of every pair of query tiles (16 bytes
- *                     per two key tiles; about 0.1 GB for that shape).
+ *                     key-tile schedule of every pair of query tiles (8 bytes
+ *                     per key tile; about 0.1 GB for that shape).
  * Softmax statistics and accumulation are fp32; the probabilities enter the
  * second tensor-core product as bf16. A kernel wait that runs out is recorded
  * in the workspace and reported by vsa_sparse_attn_status. */
