@@ -268,7 +268,33 @@ def run_ours(args):
         torch.cuda.synchronize()
         sel_ms.append(e[0].elapsed_time(e[1]))
         att_ms.append(e[1].elapsed_time(e[2]))
+    call_ms = sorted(a_ + s_ for a_, s_ in zip(att_ms, sel_ms))
+    call_p50 = statistics.median(call_ms)
+    call_p90 = call_ms[min(len(call_ms) - 1, int(round(0.9 * (len(call_ms) - 1))))]
     sel_ms, att_ms = statistics.median(sel_ms), statistics.median(att_ms)
+
+    # ---- dense comparator: torch scaled_dot_product_attention on the same Q, K, V (a library
+    # kernel, timed for context; the method replaces it)
+    dense_ms = None
+    if not args.no_dense:
+        try:
+            qd, kd, vd = (x.transpose(1, 2) for x in (q, k, v))      # [B, H, S, 128] views
+            with torch.cuda.stream(stream):
+                for _ in range(2):
+                    torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+                d_ms = []
+                for _ in range(3):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    d_ms.append(e0.elapsed_time(e1))
+            dense_ms = statistics.median(d_ms)
+        except RuntimeError as ex:   # e.g. out of memory on a smaller GPU
+            dense_ms = None
+            print("dense comparator skipped: %s" % ex, file=sys.stderr)
+        torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers
     host_in = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in bits]
@@ -324,6 +350,10 @@ def run_ours(args):
             # per step: pool, coarse, select; permute, schedule, one attention launch per batch
             "gpu_launches": (5 + wl.B) * args.steps,
             "clocks": clocks.summary(),
+            "call_ms": {"p50": call_p50, "p90": call_p90, "samples": len(call_ms)},
+            "dense_sdpa": None if dense_ms is None else {
+                "ms": dense_ms, "call_speedup": dense_ms / call_p50,
+                "what": "torch scaled_dot_product_attention, bf16, same Q, K, V, no mask"},
         }
         if world == 1 and not args.no_cpu_baseline:
             from oracle import vsa_oracle as O
@@ -348,6 +378,7 @@ def main():
     ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32")
     ap.add_argument("--ref-tiles", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the torch SDPA comparator")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -56,10 +56,11 @@ constexpr int kInfoSlots = 8;        // info of step j is rewritten only after O
 constexpr int kThreads = 256;
 constexpr int kWarpK = 0, kWarpV = 1, kWarpS = 2, kWarpPV = 3;   // warps 4..7: Q loads, softmax, epilogue
 constexpr uint32_t kTmemCols = 256;
-// O: fp32 accumulator; S: fp32 scores of one key tile; P: their bf16 pairs.
-// P has columns of its own, so S(j + 1) may be computed as soon as the scores
-// of step j are in registers.
-constexpr uint32_t kColO = 0, kColS = 128, kColP = 192;
+// O: fp32 accumulator; S: fp32 scores of one key tile; P_0, P_1: bf16 pairs of
+// the probabilities of the even / odd steps. P has columns of its own, so S(j + 1)
+// may be computed as soon as the scores of step j are in registers, and two of
+// them, so P(j) only waits for O += P(j - 2) V.
+constexpr uint32_t kColO = 0, kColS = 128, kColP0 = 192, kColP1 = 224;
 constexpr uint32_t kTileBytes = 16384;    // one key tile of K or V: [d half 0][d half 1], 64 rows x 128 B
 constexpr float kPSumLimit = 256.0f;     // 2^8: see the softmax step
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // S = Q K^T, both K-major
@@ -82,7 +83,7 @@ struct AttnSmem {
   StageInfo info[kInfoSlots];
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t info_full[kInfoSlots];
-  uint64_t q_full, s_full, s_free, p_full, pv_done, o_full, drain_s, drain_pv;
+  uint64_t q_full, s_full, s_free, p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per P buffer
   uint32_t tmem_base;
   int abort;
   int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
@@ -380,8 +381,10 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     mbar_init(smem_u32(&sm.q_full), 4);          // one arrival per softmax warp
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.s_free), 4);
-    mbar_init(smem_u32(&sm.p_full), 4);
-    mbar_init(smem_u32(&sm.pv_done), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.p_full[i]), 4);
+      mbar_init(smem_u32(&sm.pv_done[i]), 1);
+    }
     mbar_init(smem_u32(&sm.o_full), 1);
     mbar_init(smem_u32(&sm.drain_s), 1);
     mbar_init(smem_u32(&sm.drain_pv), 1);
@@ -496,7 +499,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
         bool first = true, last = false;
         while (!last) {
-          if (!(ok = mbar_wait(smem_u32(&sm.p_full), j & 1, &sm.abort, kTimeoutNs))) break;
+          const uint32_t pb = j & 1;           // P buffer of step j; its use count is j >> 1
+          if (!(ok = mbar_wait(smem_u32(&sm.p_full[pb]), (j >> 1) & 1, &sm.abort, kTimeoutNs))) break;
           last = sm.info[j % kInfoSlots].last != 0;   // read by the softmax warps before p_full
           const int vs = j % kVStages;
           if (!(ok = mbar_wait(smem_u32(&sm.v_full[vs]), (j / kVStages) & 1, &sm.abort, kTimeoutNs))) break;
@@ -505,11 +509,11 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[vs]), 8192, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tmem + kColO, tmem + kColP + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
+            umma_ts(tmem + kColO, tmem + (pb ? kColP1 : kColP0) + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
                     (first && kk == 0) ? 0u : 1u);
           first = false;
           umma_commit(smem_u32(&sm.v_empty[vs]));
-          umma_commit(smem_u32(&sm.pv_done));
+          umma_commit(smem_u32(&sm.pv_done[pb]));
           ++j;
         }
         if (!ok) break;
@@ -577,7 +581,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
           t_s = mbar_test_wait(smem_u32(&sm.s_full), (j + 1) & 1);
         }
-        if (j > 0) t_pv = mbar_test_wait(smem_u32(&sm.pv_done), (j - 1) & 1);
+        // O += P(j - 2) V has read P buffer j & 1 (the use count of a buffer is j >> 1)
+        if (j > 1) t_pv = mbar_test_wait(smem_u32(&sm.pv_done[j & 1]), ((j >> 1) - 1) & 1);
         uint32_t pw[32];
         float x[64];
         if (act) tmem_ld64f(lane_addr + kColS, x);
@@ -594,8 +599,9 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
             const bool need = ms != -INFINITY && mt > ms;
             if (ms == -INFINITY) ms = mt;     // first key tile of this row: O and l are still zero
             if (__any_sync(0xffffffffu, need)) {
-              // rescale this row of O once the previous P V has landed
-              if (j > 0 && !warp_wait(sm, sm.pv_done, (j - 1) & 1, lane, a.err)) return false;
+              // rescale this row of O once every earlier P V has landed: the last one
+              // is O += P(j - 1) V, which follows O += P(j - 2) V in issue order
+              if (j > 0 && !warp_wait(sm, sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lane, a.err)) return false;
               tc_fence_after();
               const float f = need ? ex2_approx(ms - mt) : 1.0f;
 #pragma unroll 1
@@ -630,15 +636,18 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
 #pragma unroll
           for (int i = 0; i < 32; ++i) pw[i] = 0u;     // rows of the other query tile
         }
-        // P of step j - 1 has been consumed once its P V completed
-        if (j > 0 && !__all_sync(0xffffffffu, t_pv) && !(ok = warp_wait(sm, sm.pv_done, (j - 1) & 1, lane, a.err)))
+        // P(j - 2), in the buffer P(j) goes to, has been consumed once its P V
+        // completed; that completion also needs every warp's P(j - 2), so this
+        // warp's arrivals on p_full[j & 1] stay in step order
+        if (j > 1 && !__all_sync(0xffffffffu, t_pv) &&
+            !(ok = warp_wait(sm, sm.pv_done[j & 1], ((j >> 1) - 1) & 1, lane, a.err)))
           break;
         tc_fence_after();
-        tmem_st32(lane_addr + kColP, pw);
+        tmem_st32(lane_addr + ((j & 1) ? kColP1 : kColP0), pw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full));
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[j & 1]));
         have_next = !last && __all_sync(0xffffffffu, t_info);
         if (have_next) next = sm.info[(j + 1) % kInfoSlots];
         s_ready = !last && __all_sync(0xffffffffu, t_s);
