@@ -56,11 +56,10 @@ constexpr int kInfoSlots = 8;        // info of step j is rewritten only after O
 constexpr int kThreads = 256;
 constexpr int kWarpK = 0, kWarpV = 1, kWarpS = 2, kWarpPV = 3;   // warps 4..7: Q loads, softmax, epilogue
 constexpr uint32_t kTmemCols = 256;
-// O: fp32 accumulator; S: fp32 scores of one key tile; P_0, P_1: bf16 pairs of
-// the probabilities of the even / odd steps. P has columns of its own, so S(j + 1)
-// may be computed as soon as the scores of step j are in registers, and two of
-// them, so P(j) only waits for O += P(j - 2) V.
-constexpr uint32_t kColO = 0, kColS = 128, kColP0 = 192, kColP1 = 224;
+// O: fp32 accumulator; S_0, S_1: fp32 scores of the even / odd steps, then the
+// bf16 pairs of their P over the first 32 columns. S(j + 2) reuses the buffer of
+// step j once O += P(j) V has completed.
+constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;
 constexpr uint32_t kTileBytes = 16384;    // one key tile of K or V: [d half 0][d half 1], 64 rows x 128 B
 constexpr float kPSumLimit = 256.0f;     // 2^8: see the softmax step
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // S = Q K^T, both K-major
@@ -83,7 +82,7 @@ struct AttnSmem {
   StageInfo info[kInfoSlots];
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t info_full[kInfoSlots];
-  uint64_t q_full, s_full, s_free, p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per P buffer
+  uint64_t q_full, s_full[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per score buffer
   uint32_t tmem_base;
   int abort;
   int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
@@ -379,9 +378,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     }
     for (int s = 0; s < kInfoSlots; ++s) mbar_init(smem_u32(&sm.info_full[s]), 1);
     mbar_init(smem_u32(&sm.q_full), 4);          // one arrival per softmax warp
-    mbar_init(smem_u32(&sm.s_full), 1);
-    mbar_init(smem_u32(&sm.s_free), 4);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
       mbar_init(smem_u32(&sm.p_full[i]), 4);
       mbar_init(smem_u32(&sm.pv_done[i]), 1);
     }
@@ -454,9 +452,9 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     }
   } else if (warp == kWarpS) {
     // ------------------------------------------------------ S = Q K^T issuer
-    // S(j) may overwrite the score columns once the softmax warps have read
-    // S(j - 1) into registers (s_free); Q of an item is in shared memory once
-    // q_full completes.
+    // S(j) goes to buffer j & 1 once O += P(j - 2) V, which reads P(j - 2) from
+    // that buffer, has completed; Q of an item is in shared memory once q_full
+    // completes.
     bool ok = true;
     if (lane == 0) {
       uint32_t j = 0;
@@ -468,7 +466,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         while (!last) {
           const int ks = j % kKStages;
           if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (j / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
-          if (j > 0 && !(ok = mbar_wait(smem_u32(&sm.s_free), (j - 1) & 1, &sm.abort, kTimeoutNs))) break;
+          if (j > 1 && !(ok = mbar_wait(smem_u32(&sm.pv_done[j & 1]), ((j >> 1) - 1) & 1, &sm.abort, kTimeoutNs)))
+            break;
           tc_fence_after();
           last = sm.info[j % kInfoSlots].last != 0;
           const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]), 16, 1024);
@@ -476,11 +475,11 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           for (int kk = 0; kk < 8; ++kk) {
             // 16 d per K step: 32 B inside a swizzle row of d half kk / 4
             // (descriptor addresses count 16-byte units)
-            umma_ss(tmem + kColS, qd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2,
+            umma_ss(tmem + ((j & 1) ? kColS1 : kColS0), qd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2,
                     kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS, kk > 0 ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm.k_empty[ks]));
-          umma_commit(smem_u32(&sm.s_full));
+          umma_commit(smem_u32(&sm.s_full[j & 1]));
           ++j;
         }
       }
@@ -499,7 +498,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
         bool first = true, last = false;
         while (!last) {
-          const uint32_t pb = j & 1;           // P buffer of step j; its use count is j >> 1
+          const uint32_t pb = j & 1;           // score / P buffer of step j; its use count is j >> 1
           if (!(ok = mbar_wait(smem_u32(&sm.p_full[pb]), (j >> 1) & 1, &sm.abort, kTimeoutNs))) break;
           last = sm.info[j % kInfoSlots].last != 0;   // read by the softmax warps before p_full
           const int vs = j % kVStages;
@@ -509,7 +508,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[vs]), 8192, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tmem + kColO, tmem + (pb ? kColP1 : kColP0) + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
+            umma_ts(tmem + kColO, tmem + (pb ? kColS1 : kColS0) + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
                     (first && kk == 0) ? 0u : 1u);
           first = false;
           umma_commit(smem_u32(&sm.v_empty[vs]));
@@ -574,24 +573,19 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         }
         last = inf.last != 0;
         const bool act = (inf.mask >> half) & 1;     // the same for the whole warp
-        if (!s_ready && !(ok = warp_wait(sm, sm.s_full, j & 1, lane, a.err))) break;
+        if (!s_ready && !(ok = warp_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, lane, a.err))) break;
         tc_fence_after();
-        uint32_t t_info = 0, t_s = 0, t_pv = 1;
+        uint32_t t_info = 0, t_s = 0;
         if (!last) {
           t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
-          t_s = mbar_test_wait(smem_u32(&sm.s_full), (j + 1) & 1);
+          t_s = mbar_test_wait(smem_u32(&sm.s_full[(j + 1) & 1]), ((j + 1) >> 1) & 1);
         }
-        // O += P(j - 2) V has read P buffer j & 1 (the use count of a buffer is j >> 1)
-        if (j > 1) t_pv = mbar_test_wait(smem_u32(&sm.pv_done[j & 1]), ((j >> 1) - 1) & 1);
+        const uint32_t scol = lane_addr + ((j & 1) ? kColS1 : kColS0);
         uint32_t pw[32];
         float x[64];
-        if (act) tmem_ld64f(lane_addr + kColS, x);
-        tmem_wait_ld();
-        // the scores are in registers: S(j + 1) may overwrite them
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.s_free));
         if (act) {
+          tmem_ld64f(scol, x);
+          tmem_wait_ld();
           if (inf.valid != ~0ull) mask_invalid(x, inf.valid);   // padding slots never attend
           // exact row max of the step; O and l rescaled when it raises the running max
           auto exact_max = [&]() -> bool {
@@ -636,14 +630,11 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
 #pragma unroll
           for (int i = 0; i < 32; ++i) pw[i] = 0u;     // rows of the other query tile
         }
-        // P(j - 2), in the buffer P(j) goes to, has been consumed once its P V
-        // completed; that completion also needs every warp's P(j - 2), so this
-        // warp's arrivals on p_full[j & 1] stay in step order
-        if (j > 1 && !__all_sync(0xffffffffu, t_pv) &&
-            !(ok = warp_wait(sm, sm.pv_done[j & 1], ((j >> 1) - 1) & 1, lane, a.err)))
-          break;
-        tc_fence_after();
-        tmem_st32(lane_addr + ((j & 1) ? kColP1 : kColP0), pw);
+        // P(j) over the first 32 columns of its own score buffer (the scores were
+        // read above). A warp reaches step j + 2 only after S(j + 2), which waited
+        // for O += P(j) V and so for every warp's P(j): arrivals on p_full[j & 1]
+        // stay in step order.
+        tmem_st32(scol, pw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
