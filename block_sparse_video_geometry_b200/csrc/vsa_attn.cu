@@ -8,11 +8,12 @@
 // attend the whole sequence. The epilogue writes o_fine + g * o_coarse.
 //
 // Design (B200):
-//  * Work item = two query tiles of one (batch, head) stacked into a 128-row
-//    tcgen05 tile (M = 128). The key tiles of the item are the union of the two
-//    tiles' key lists; each 128x64 score block is masked per 64-row half for
-//    key tiles that only one of the two tiles selected, and the rows of the
-//    other tile skip their exp2 work.
+//  * Work item = one 64-token query tile of one (batch, head), computed with
+//    M = 64 tcgen05 MMAs; its key tiles are the dense part (all conditioning
+//    tiles, or all tiles for dense conditioning rows) followed by its own
+//    selection list. (Stacking two query tiles into one M = 128 tile needs the
+//    union of their lists; the selections of neighbouring tiles barely overlap,
+//    so most of that work would be masked.)
 //  * permute_kv_kernel first rewrites K and V tile-major into the workspace,
 //    each 64-token tile of each head one contiguous 16 KB block already in the
 //    128-byte-swizzled layout of the UMMA descriptors, padding slots zero, so
@@ -20,17 +21,21 @@
 //    every item's key-tile sequence as records, so that the copy warps only
 //    stream records (a copy warp shares its scheduler with a softmax warp, and
 //    every instruction it needs per step delays the copies).
-//  * Two CTAs per SM, each with 256 TMEM columns: O (128), S (64) and P (bf16,
-//    32). P has columns of its own, so S(j + 1) may be computed as soon as the
-//    softmax warps hold S(j) in registers. Q sits in shared memory.
+//  * Two CTAs per SM, each with 256 TMEM columns: O (128) and two 64-column
+//    score buffers, all M = 64 accumulators (rows in the first 16 lanes of each
+//    lane quadrant). Q and the bf16 P of the even / odd steps sit in shared
+//    memory; S(j + 2) reuses the score buffer of step j once the softmax warps
+//    are done with it, and P(j) waits only for O += P(j - 2) V.
 //  * Every tcgen05 instruction holds its issuing thread for about 46 cycles,
 //    so one warp issues the S MMAs and another the P V MMAs.
 //  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues S
 //    = Q K^T, 3 issues O += P V; 4-7 load each item's Q into shared memory,
-//    run the fp32 online softmax (one thread per row, exp2) and the epilogue.
-//    P is computed against the running max; the exact row max of a step is
-//    only formed when a row's sum of P exceeds 2^8 (then O and the sum are
-//    rescaled and P recomputed), which keeps every P at most 2^8.
+//    run the fp32 online softmax and the epilogue: two threads per row (the
+//    16x32bx2 TMEM shape gives the two half-warps the same 16 lanes at two
+//    column offsets), 32 keys each per step, exp2. P is computed against the
+//    running max; the exact row max of a step is only formed when a row's sum
+//    of P exceeds 2^8 (then O and the sum are rescaled and P recomputed),
+//    which keeps every P at most 2^8.
 //  * Every wait is bounded: a wait that runs out sets an error word in the
 //    workspace, raises an abort flag that ends the other roles' loops, drains
 //    in-flight copies and MMAs and frees TMEM before the block exits.
@@ -56,33 +61,31 @@ constexpr int kInfoSlots = 8;        // info of step j is rewritten only after O
 constexpr int kThreads = 256;
 constexpr int kWarpK = 0, kWarpV = 1, kWarpS = 2, kWarpPV = 3;   // warps 4..7: Q loads, softmax, epilogue
 constexpr uint32_t kTmemCols = 256;
-// O: fp32 accumulator; S_0, S_1: fp32 scores of the even / odd steps, then the
-// bf16 pairs of their P over the first 32 columns. S(j + 2) reuses the buffer of
-// step j once O += P(j) V has completed.
+// M = 64 accumulators (rows in the first 16 lanes of each quadrant): O (fp32,
+// 128 columns) and the fp32 scores of the even / odd steps.
 constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;
 constexpr uint32_t kTileBytes = 16384;    // one key tile of K or V: [d half 0][d half 1], 64 rows x 128 B
 constexpr float kPSumLimit = 256.0f;     // 2^8: see the softmax step
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // S = Q K^T, both K-major
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // O = P V, V is MN-major
+constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, 0, 0);      // S = Q K^T, both K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 128, 0, 1);    // O = P V, P K-major, V MN-major
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
 
 struct StageInfo {
   int32_t tile;
-  int32_t mask;   // bit 0: first query tile lists it, bit 1: second query tile lists it
   int32_t last;   // last key tile of the work item
-  int32_t pad;
   unsigned long long valid;
 };
 
 struct AttnSmem {
-  uint8_t q[2][128 * 128];             // [d half][128 rows x 128 B], SW128 K-major (rows 64..127: second tile)
+  uint8_t q[2][64 * 128];              // [d half][64 rows x 128 B], SW128 K-major
+  uint8_t p[2][64 * 128];              // P of the even / odd steps: 64 rows x 64 keys bf16, SW128 K-major
   uint8_t k[kKStages][kTileBytes];
   uint8_t v[kVStages][kTileBytes];
   StageInfo info[kInfoSlots];
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t info_full[kInfoSlots];
-  uint64_t q_full, s_full[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per score buffer
+  uint64_t q_full, s_full[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per step parity
   uint32_t tmem_base;
   int abort;
   int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
@@ -110,7 +113,7 @@ struct AttnArgs {
   int64_t q_ss, q_sh;
   int32_t H, b, sink, kmax;
   int32_t c0;                // first query tile of the sparse item range
-  int32_t np_dense, np_sparse, n_dense_items, n_items;
+  int32_t nq_dense, nq_sparse, n_dense_items, n_items;   // query tiles per head: dense rows, sparse rows
   const int32_t* idx;         // selection lists (read by schedule_kernel)
   const int32_t* cnt;
   const unsigned long long* valid;   // per-tile slot masks
@@ -127,22 +130,21 @@ struct AttnArgs {
   int* err;
 };
 
+// Work item = one query tile of one (batch, head).
 struct Item {
-  int h, qa, qb, dense;
+  int h, qt, dense;
 };
 
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item) {
   Item it;
   if (item < a.n_dense_items) {
-    it.h = item / a.np_dense;
-    it.qa = 2 * (item % a.np_dense);
-    it.qb = it.qa + 1 < a.G.n_cond ? it.qa + 1 : -1;
+    it.h = item / a.nq_dense;
+    it.qt = item % a.nq_dense;
     it.dense = 1;
   } else {
     const int r = item - a.n_dense_items;
-    it.h = r / a.np_sparse;
-    it.qa = a.c0 + 2 * (r % a.np_sparse);
-    it.qb = it.qa + 1 < a.G.n_tiles ? it.qa + 1 : -1;
+    it.h = r / a.nq_sparse;
+    it.qt = a.c0 + r % a.nq_sparse;
     it.dense = 0;
   }
   return it;
@@ -214,21 +216,11 @@ __device__ __forceinline__ void mask_invalid(float (&x)[64], unsigned long long 
   }
 }
 
-// Largest score of a key tile.
-__device__ __forceinline__ float row_max(const float (&x)[64]) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = x[i];
-#pragma unroll
-  for (int i = 8; i < 64; ++i) m[i & 7] = fmaxf(m[i & 7], x[i]);
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
-}
-
-// bf16 pairs of P = 2^(x c - ms) for one key tile; returns the fp32 sum of P.
-__device__ __forceinline__ float exp_pass(const float (&x)[64], float c, float ms, uint32_t (&pw)[32]) {
+// bf16 pairs of P = 2^(x c - ms) for 32 keys; returns the fp32 sum of P.
+__device__ __forceinline__ float exp_pass(const float (&x)[32], float c, float ms, uint32_t (&pw)[16]) {
   float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < 16; ++i) {
     const float p0 = ex2_approx(fmaf(x[2 * i], c, -ms));
     const float p1 = ex2_approx(fmaf(x[2 * i + 1], c, -ms));
     ps[i & 3] += p0 + p1;
@@ -267,91 +259,36 @@ permute_kv_kernel(DevLayout L, const uint16_t* __restrict__ k, const uint16_t* _
 }
 
 // Step schedule of each work item, built once per call so that the copy warps
-// of the attention kernel only stream records. Record = (key tile, flags):
-// bits 0-1 which of the item's query tiles list the key tile, bit 4 last step
-// of the item, bit 5 the key tile has padding slots. Key tiles come in the
-// item's order: the dense part (conditioning tiles, or all tiles for dense
-// rows), then the union of the two selection lists, ascending.
-// One warp per item; the union is formed with bitmaps in shared memory.
-constexpr int kSchedWarps = 4;
+// of the attention kernel only stream records. Record = (key tile, flags): bit 4
+// last step of the item, bit 5 the key tile has padding slots. Key tiles come in
+// the item's order: the dense part (conditioning tiles, or all tiles for dense
+// rows), then the query tile's selection list (ascending video ordinals).
+constexpr int kSchedThreads = 128;
 
-size_t sched_smem_per_warp(int n_tiles, int n_video) {
-  return align_up(static_cast<size_t>(2 * ((n_video + 31) / 32)) * 4 + static_cast<size_t>(n_tiles) * 5, 16);
-}
-
-__global__ void __launch_bounds__(kSchedWarps * 32) schedule_kernel(const __grid_constant__ AttnArgs a,
-                                                                     int per_warp_bytes) {
-  extern __shared__ __align__(16) uint8_t sh[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int item = blockIdx.x * kSchedWarps + warp;
-  const int b = blockIdx.y;
-  if (item >= a.n_items) return;
+__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_constant__ AttnArgs a) {
+  const int item = blockIdx.x, b = blockIdx.y;
   const Geom& G = a.G;
   const Item it = decode_item(a, item);
-  const int nw = (G.n_video + 31) / 32;
-  uint32_t* bma = reinterpret_cast<uint32_t*>(sh + warp * per_warp_bytes);
-  uint32_t* bmb = bma + nw;
-  int32_t* tl = reinterpret_cast<int32_t*>(bmb + nw);
-  uint8_t* mk = reinterpret_cast<uint8_t*>(tl + G.n_tiles);
-  const int both = it.qb >= 0 ? 3 : 1;
   const int n_dense = it.dense ? G.n_tiles : G.n_cond;
-  for (int i = lane; i < n_dense; i += 32) {
-    tl[i] = i;
-    mk[i] = static_cast<uint8_t>(both);
-  }
-  int total = n_dense;
-  if (!it.dense) {
-    for (int w = lane; w < nw; w += 32) bma[w] = bmb[w] = 0u;
-    __syncwarp();
-    const size_t row = (static_cast<size_t>(b) * a.H + it.h) * G.n_tiles;
-    // entries outside [0, n_video) (never written by vsa_coarse_select) are skipped
-    const int na = min(a.cnt[row + it.qa], a.kmax);
-    for (int i = lane; i < na; i += 32) {
-      const int t = a.idx[(row + it.qa) * a.kmax + i];
-      if (static_cast<unsigned>(t) < static_cast<unsigned>(G.n_video)) atomicOr(&bma[t >> 5], 1u << (t & 31));
-    }
-    if (it.qb >= 0) {
-      const int nb = min(a.cnt[row + it.qb], a.kmax);
-      for (int i = lane; i < nb; i += 32) {
-        const int t = a.idx[(row + it.qb) * a.kmax + i];
-        if (static_cast<unsigned>(t) < static_cast<unsigned>(G.n_video)) atomicOr(&bmb[t >> 5], 1u << (t & 31));
-      }
-    }
-    __syncwarp();
-    // each lane owns a contiguous range of bitmap words; a warp scan gives its output offset
-    const int wpl = (nw + 31) / 32, w0 = min(nw, lane * wpl), w1 = min(nw, w0 + wpl);
-    int mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(bma[w] | bmb[w]);
-    int incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = n_dense + incl - mine;
-    for (int w = w0; w < w1; ++w) {
-      uint32_t u = bma[w] | bmb[w];
-      while (u) {
-        const int bit = __ffs(u) - 1;
-        u &= u - 1u;
-        tl[pos] = G.n_cond + w * 32 + bit;
-        mk[pos] = static_cast<uint8_t>(((bma[w] >> bit) & 1u) | (((bmb[w] >> bit) & 1u) << 1));
-        ++pos;
-      }
-    }
-    total = n_dense + __shfl_sync(0xffffffffu, incl, 31);
-  }
-  __syncwarp();
-  const int n_steps = total;
+  const size_t row = (static_cast<size_t>(b) * a.H + it.h) * G.n_tiles + it.qt;
+  const int n_sel = it.dense ? 0 : min(max(a.cnt[row], 0), a.kmax);
+  const int n = n_dense + n_sel;
   int2* rec = a.sched + (static_cast<size_t>(b) * a.n_items + item) * a.max_steps;
-  for (int r = lane; r < n_steps; r += 32) {
-    const int t = tl[r];
-    uint32_t fl = mk[r];
-    if (r == n_steps - 1) fl |= 16u;
+  for (int r = threadIdx.x; r < n; r += kSchedThreads) {
+    int t;
+    if (r < n_dense) {
+      t = r;
+    } else {
+      // entries outside [0, n_video) (never written by vsa_coarse_select) are clamped: memory stays in bounds
+      const int v = a.idx[row * a.kmax + (r - n_dense)];
+      t = G.n_cond + min(max(v, 0), G.n_video - 1);
+    }
+    uint32_t fl = 0u;
+    if (r == n - 1) fl |= 16u;
     if (a.valid[t] != ~0ull) fl |= 32u;
     rec[r] = make_int2(t, static_cast<int>(fl));
   }
-  if (lane == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = n_steps;
+  if (threadIdx.x == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = n;
 }
 
 // 128 registers per thread: two CTAs of 256 threads fit one SM's register file.
@@ -430,7 +367,6 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           if (is_k) {
             StageInfo& inf = sm.info[step % kInfoSlots];
             inf.tile = tile;
-            inf.mask = fl & 3;
             inf.last = (fl >> 4) & 1;
             inf.valid = (fl & 32) ? a.valid[tile] : ~0ull;
             mbar_arrive(smem_u32(&sm.info_full[step % kInfoSlots]));
@@ -452,9 +388,9 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     }
   } else if (warp == kWarpS) {
     // ------------------------------------------------------ S = Q K^T issuer
-    // S(j) goes to buffer j & 1 once O += P(j - 2) V, which reads P(j - 2) from
-    // that buffer, has completed; Q of an item is in shared memory once q_full
-    // completes.
+    // S(j) goes to score buffer j & 1 once the softmax warps are done with
+    // S(j - 2) (p_full of step j - 2); Q of an item is in shared memory once
+    // q_full completes.
     bool ok = true;
     if (lane == 0) {
       uint32_t j = 0;
@@ -466,7 +402,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         while (!last) {
           const int ks = j % kKStages;
           if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (j / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
-          if (j > 1 && !(ok = mbar_wait(smem_u32(&sm.pv_done[j & 1]), ((j >> 1) - 1) & 1, &sm.abort, kTimeoutNs)))
+          if (j > 1 && !(ok = mbar_wait(smem_u32(&sm.p_full[j & 1]), ((j >> 1) - 1) & 1, &sm.abort, kTimeoutNs)))
             break;
           tc_fence_after();
           last = sm.info[j % kInfoSlots].last != 0;
@@ -475,7 +411,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           for (int kk = 0; kk < 8; ++kk) {
             // 16 d per K step: 32 B inside a swizzle row of d half kk / 4
             // (descriptor addresses count 16-byte units)
-            umma_ss(tmem + ((j & 1) ? kColS1 : kColS0), qd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2,
+            umma_ss(tmem + ((j & 1) ? kColS1 : kColS0), qd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2,
                     kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS, kk > 0 ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm.k_empty[ks]));
@@ -491,25 +427,27 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     __syncwarp();
   } else if (warp == kWarpPV) {
     // ----------------------------------------------------- O += P V issuer
-    // The first step of an item overwrites O; o_full fires after its last step.
+    // P(j) sits in shared-memory buffer j & 1. The first step of an item
+    // overwrites O; o_full fires after its last step.
     bool ok = true;
     if (lane == 0) {
       uint32_t j = 0;
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
         bool first = true, last = false;
         while (!last) {
-          const uint32_t pb = j & 1;           // score / P buffer of step j; its use count is j >> 1
+          const uint32_t pb = j & 1;           // P buffer of step j; its use count is j >> 1
           if (!(ok = mbar_wait(smem_u32(&sm.p_full[pb]), (j >> 1) & 1, &sm.abort, kTimeoutNs))) break;
           last = sm.info[j % kInfoSlots].last != 0;   // read by the softmax warps before p_full
           const int vs = j % kVStages;
           if (!(ok = mbar_wait(smem_u32(&sm.v_full[vs]), (j / kVStages) & 1, &sm.abort, kTimeoutNs))) break;
           tc_fence_after();
-          // V as MN-major B: 64-d blocks 8 KB apart, 16 keys = 2 KB per K step
+          // P: 64 rows x 64 keys, K-major; V as MN-major B: 64-d blocks 8 KB apart,
+          // 16 keys = 32 B of P and 2 KB of V per K step
+          const uint64_t pd = smem_desc_sw128(smem_u32(sm.p[pb]), 16, 1024);
           const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[vs]), 8192, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tmem + kColO, tmem + (pb ? kColS1 : kColS0) + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
-                    (first && kk == 0) ? 0u : 1u);
+            umma_ss(tmem + kColO, pd + kk * 2, vd + kk * (2048 >> 4), kIdescPV, (first && kk == 0) ? 0u : 1u);
           first = false;
           umma_commit(smem_u32(&sm.v_empty[vs]));
           umma_commit(smem_u32(&sm.pv_done[pb]));
@@ -525,10 +463,12 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     __syncwarp();
   } else {
     // ------------------------------------------------ Q / softmax / epilogue
-    // One thread per row of the 128-row tile.
-    const int quad = warp & 3;                       // TMEM lane quadrant of this warp
-    const int r = quad * 32 + lane;                  // row of the 128-row tile
-    const int half = r >> 6;                         // 0: first query tile, 1: second
+    // M = 64 layout: warp q (TMEM lanes 32q..32q+31) owns rows 16q..16q+15 in
+    // its first 16 lanes; thread t handles row 16q + (t & 15) and the key (or
+    // output column) half t >> 4, its partner is thread t ^ 16.
+    const int quad = warp & 3;
+    const int hf = lane >> 4;                        // 0: keys 0..31 / d 0..63, 1: keys 32..63 / d 64..127
+    const int r = quad * 16 + (lane & 15);           // row of the 64-row tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float c = a.scale_log2;
     uint32_t j = 0;
@@ -536,28 +476,22 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     bool ok = true;
     for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
       const Item it = decode_item(a, item);
-      const int qt = half ? it.qb : it.qa;
-      const int slot = r & 63;
-      const bool row_ok = qt >= 0 && ((tile_mask(sm, G, qt) >> slot) & 1ull);
-      const int64_t tok = row_ok ? tile_token(sm, G, qt, slot) : 0;
+      const bool row_ok = (tile_mask(sm, G, it.qt) >> r) & 1ull;
+      const int64_t tok = row_ok ? tile_token(sm, G, it.qt, r) : 0;
       {
-        // this row's Q into shared memory, 128-byte swizzled (every MMA of the
-        // previous item has completed)
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + tok * a.q_ss + it.h * a.q_sh);
+        // this row's half of Q (d in [64 hf, 64 hf + 64)) into shared memory,
+        // 128-byte swizzled (every MMA of the previous item has completed)
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + tok * a.q_ss + it.h * a.q_sh + 64 * hf);
+        uint4 w[8];
 #pragma unroll
-        for (int hq = 0; hq < 2; ++hq) {
-          uint4 w[8];
+        for (int cc = 0; cc < 8; ++cc) w[cc] = row_ok ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) w[cc] = row_ok ? __ldg(src + hq * 8 + cc) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
-            *reinterpret_cast<uint4*>(&sm.q[hq][r * 128 + ((cc ^ (r & 7)) << 4)]) = w[cc];
-        }
+        for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(&sm.q[hf][r * 128 + ((cc ^ (r & 7)) << 4)]) = w[cc];
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.q_full));
       }
-      float ms = -INFINITY, l = 0.f;        // running max (scaled, log2 domain) and sum
+      float ms = -INFINITY, l = 0.f;        // running max (scaled, log2 domain, same in both halves) and half sum
       bool last = false;
       // barrier phases of the next step are tested (without blocking) early in
       // a step and read after its exp2 work, so that their latency is hidden
@@ -572,70 +506,87 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           inf = sm.info[j % kInfoSlots];
         }
         last = inf.last != 0;
-        const bool act = (inf.mask >> half) & 1;     // the same for the whole warp
         if (!s_ready && !(ok = warp_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, lane, a.err))) break;
         tc_fence_after();
-        uint32_t t_info = 0, t_s = 0;
+        uint32_t t_info = 0, t_s = 0, t_pv = 1;
         if (!last) {
           t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
           t_s = mbar_test_wait(smem_u32(&sm.s_full[(j + 1) & 1]), ((j + 1) >> 1) & 1);
         }
+        // O += P(j - 2) V has read P buffer j & 1 (the use count of a buffer is j >> 1)
+        if (j > 1) t_pv = mbar_test_wait(smem_u32(&sm.pv_done[j & 1]), ((j >> 1) - 1) & 1);
         const uint32_t scol = lane_addr + ((j & 1) ? kColS1 : kColS0);
-        uint32_t pw[32];
-        float x[64];
-        if (act) {
-          tmem_ld64f(scol, x);
+        float x[32];
+        auto load_scores = [&]() {
+          tmem_ld16x2_32f<32>(scol, x);
           tmem_wait_ld();
-          if (inf.valid != ~0ull) mask_invalid(x, inf.valid);   // padding slots never attend
-          // exact row max of the step; O and l rescaled when it raises the running max
-          auto exact_max = [&]() -> bool {
-            const float mt = row_max(x) * c;
-            const bool need = ms != -INFINITY && mt > ms;
-            if (ms == -INFINITY) ms = mt;     // first key tile of this row: O and l are still zero
-            if (__any_sync(0xffffffffu, need)) {
-              // rescale this row of O once every earlier P V has landed: the last one
-              // is O += P(j - 1) V, which follows O += P(j - 2) V in issue order
-              if (j > 0 && !warp_wait(sm, sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lane, a.err)) return false;
-              tc_fence_after();
-              const float f = need ? ex2_approx(ms - mt) : 1.0f;
-#pragma unroll 1
-              for (int ch = 0; ch < 4; ++ch) {
-                uint32_t u[32];
-                tmem_ld32(lane_addr + kColO + 32 * ch, u);
-                tmem_wait_ld();
+          if (inf.valid != ~0ull) {           // padding slots never attend
+            const uint32_t vm = static_cast<uint32_t>(inf.valid >> (32 * hf));
 #pragma unroll
-                for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * f);
-                tmem_st32(lane_addr + kColO + 32 * ch, u);
-              }
-              tmem_wait_st();
-              if (need) {
-                l *= f;
-                ms = mt;
-              }
-            }
-            return true;
-          };
-          // P against the running max ms. The softmax does not depend on that
-          // reference as long as no P is large, so the exact row max of the step
-          // is only formed when a row has no reference yet, or when its P sum
-          // exceeds 2^8 (then every P was at most 2^8: fine for bf16 and fp32).
-          if (__any_sync(0xffffffffu, ms == -INFINITY) && !(ok = exact_max())) break;
-          float psum = exp_pass(x, c, ms, pw);
-          if (__any_sync(0xffffffffu, psum > kPSumLimit)) {
-            if (!(ok = exact_max())) break;
-            psum = exp_pass(x, c, ms, pw);   // every P <= 1 now
+            for (int i = 0; i < 32; ++i) x[i] = ((vm >> i) & 1u) ? x[i] : -INFINITY;
           }
-          l += psum;
-        } else {
+        };
+        // exact row max of the step; O and l rescaled when it raises the running max
+        auto exact_max = [&]() -> bool {
+          float m = x[0];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pw[i] = 0u;     // rows of the other query tile
+          for (int i = 1; i < 32; ++i) m = fmaxf(m, x[i]);
+          const float mt = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16)) * c;
+          const bool need = ms != -INFINITY && mt > ms;
+          if (ms == -INFINITY) ms = mt;       // first key tile of this row: O and l are still zero
+          if (__any_sync(0xffffffffu, need)) {
+            // rescale this half row of O once every earlier P V has landed: the
+            // last one is O += P(j - 1) V, which follows O += P(j - 2) V in issue order
+            if (j > 0 && !warp_wait(sm, sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lane, a.err)) return false;
+            tc_fence_after();
+            const float f = need ? ex2_approx(ms - mt) : 1.0f;
+#pragma unroll 1
+            for (int ch = 0; ch < 2; ++ch) {
+              float u[32];
+              tmem_ld16x2_32f<64>(lane_addr + kColO + 32 * ch, u);
+              tmem_wait_ld();
+              uint32_t w[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(u[i] * f);
+              tmem_st16x2_32<64>(lane_addr + kColO + 32 * ch, w);
+            }
+            tmem_wait_st();
+            if (need) {
+              l *= f;
+              ms = mt;
+            }
+          }
+          return true;
+        };
+        // P against the running max ms. The softmax does not depend on that
+        // reference as long as no P is large, so the exact row max of the step
+        // is only formed when a row has no reference yet, or when its P sum
+        // exceeds 2^8 (then every P was at most 2^8: fine for bf16 and fp32).
+        uint32_t pw[16];
+        load_scores();
+        if (__any_sync(0xffffffffu, ms == -INFINITY) && !(ok = exact_max())) break;
+        float psum = exp_pass(x, c, ms, pw);
+        if (__any_sync(0xffffffffu, psum + __shfl_xor_sync(0xffffffffu, psum, 16) > kPSumLimit)) {
+          load_scores();
+          if (!(ok = exact_max())) break;
+          psum = exp_pass(x, c, ms, pw);     // every P <= 1 now
         }
-        // P(j) over the first 32 columns of its own score buffer (the scores were
-        // read above). A warp reaches step j + 2 only after S(j + 2), which waited
-        // for O += P(j) V and so for every warp's P(j): arrivals on p_full[j & 1]
-        // stay in step order.
-        tmem_st32(scol, pw);
-        tmem_wait_st();
+        l += psum;
+        // P(j - 2), in the buffer P(j) goes to, has been consumed once its P V
+        // completed; that completion also needs every warp's P(j - 2), so this
+        // warp's arrivals on p_full[j & 1] stay in step order
+        if (j > 1 && !__all_sync(0xffffffffu, t_pv) &&
+            !(ok = warp_wait(sm, sm.pv_done[j & 1], ((j >> 1) - 1) & 1, lane, a.err)))
+          break;
+        {
+          // this half row of P: 32 keys = 64 B = 16-byte chunks 4 hf .. 4 hf + 3 of row r
+          uint8_t* prow = sm.p[j & 1] + r * 128;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            *reinterpret_cast<uint4*>(prow + (((4 * hf + cc) ^ (r & 7)) << 4)) =
+                make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
+        }
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[j & 1]));
@@ -645,25 +596,24 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         ++j;
       }
       if (!ok) break;
-      // epilogue: out = O / l + g * o_coarse
+      // epilogue: out = O / l + g * o_coarse over this thread's half row (64 columns)
       if (!(ok = warp_wait(sm, sm.o_full, it_n & 1, lane, a.err))) break;
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      const float inv_l = 1.0f / (l + __shfl_xor_sync(0xffffffffu, l, 16));
       float gate = 0.f;
       const float* oc = nullptr;
-      if (row_ok && !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && qt < G.n_cond)) {
+      if (row_ok && !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && it.qt < G.n_cond)) {
         gate = __uint_as_float(static_cast<uint32_t>(a.g[a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh]) << 16);
-        oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + qt) * kHeadDim;
+        oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + it.qt) * kHeadDim + 64 * hf;
       }
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t u[32];
-        tmem_ld32(lane_addr + kColO + 32 * ch, u);
+      for (int ch = 0; ch < 2; ++ch) {
+        float y[32];
+        tmem_ld16x2_32f<64>(lane_addr + kColO + 32 * ch, y);
         tmem_wait_ld();
         if (row_ok) {
-          float y[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(u[i]) * inv_l;
+          for (int i = 0; i < 32; ++i) y[i] *= inv_l;
           if (oc) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
@@ -674,7 +624,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
               y[i + 3] = fmaf(gate, cv.w, y[i + 3]);
             }
           }
-          const int64_t off = a.b * a.o_sb + tok * a.o_ss + it.h * a.o_sh + ch * 32;
+          const int64_t off = a.b * a.o_sb + tok * a.o_ss + it.h * a.o_sh + 64 * hf + ch * 32;
           if (a.out_bf16) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + off);
 #pragma unroll
@@ -713,19 +663,18 @@ constexpr size_t kMaxAttnSmem = 227 * 1024;
 
 // Work decomposition shared by the host and the kernels (see decode_item).
 struct ItemCounts {
-  int32_t c0, np_dense, np_sparse, n_dense_items, n_items, max_steps;
+  int32_t c0, nq_dense, nq_sparse, n_dense_items, n_items, max_steps;
 };
 
 ItemCounts item_counts(const vsa_layout* L, int H, const vsa_params* p, int32_t kmax) {
   ItemCounts c{};
   const bool rows = p->sink == VSA_SINK_EXACT_KV_AND_ROWS;
   c.c0 = rows ? L->n_cond : 0;
-  c.np_dense = rows ? (L->n_cond + 1) / 2 : 0;
-  c.np_sparse = (L->n_tiles - c.c0 + 1) / 2;
-  c.n_dense_items = c.np_dense * H;
-  c.n_items = c.n_dense_items + c.np_sparse * H;
-  const int sparse_tiles = L->n_cond + std::min(2 * kmax, L->n_video);
-  c.max_steps = std::max(rows ? L->n_tiles : 0, sparse_tiles);
+  c.nq_dense = rows ? L->n_cond : 0;
+  c.nq_sparse = L->n_tiles - c.c0;
+  c.n_dense_items = c.nq_dense * H;
+  c.n_items = c.n_dense_items + c.nq_sparse * H;
+  c.max_steps = std::max(rows ? L->n_tiles : 0, L->n_cond + std::min(kmax, L->n_video));
   return c;
 }
 
@@ -815,8 +764,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.kmax = kmax;
   const ItemCounts ic = item_counts(L, H, p, kmax);
   a.c0 = ic.c0;
-  a.np_dense = ic.np_dense;
-  a.np_sparse = ic.np_sparse;
+  a.nq_dense = ic.nq_dense;
+  a.nq_sparse = ic.nq_sparse;
   a.n_dense_items = ic.n_dense_items;
   a.n_items = ic.n_items;
   a.max_steps = ic.max_steps;
@@ -851,13 +800,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
                                                             wsb + ws.kv);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: permute launch", e);
-  const size_t per_warp = sched_smem_per_warp(L->n_tiles, L->n_video);
-  if (per_warp * kSchedWarps > kMaxAttnSmem) return VSA_ERR_UNSUPPORTED;
-  e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(per_warp * kSchedWarps));
-  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
-  schedule_kernel<<<dim3((a.n_items + kSchedWarps - 1) / kSchedWarps, B), kSchedWarps * 32, per_warp * kSchedWarps,
-                    stream>>>(a, static_cast<int>(per_warp));
+  schedule_kernel<<<dim3(a.n_items, B), kSchedThreads, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: schedule launch", e);
   for (int b = 0; b < B; ++b) {
