@@ -24,8 +24,8 @@
 //  * Two CTAs per SM, each with 256 TMEM columns: O (128) and two 64-column
 //    score buffers, all M = 64 accumulators (rows in the first 16 lanes of each
 //    lane quadrant). Q and the bf16 P of the even / odd steps sit in shared
-//    memory; S(j + 2) reuses the score buffer of step j once the softmax warps
-//    are done with it, and P(j) waits only for O += P(j - 2) V.
+//    memory; S(j + 2) reuses the score buffer of step j as soon as the softmax
+//    warps hold S(j) in registers, and P(j) waits only for O += P(j - 2) V.
 //  * Every tcgen05 instruction holds its issuing thread for about 46 cycles,
 //    so one warp issues the S MMAs and another the P V MMAs.
 //  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues S
@@ -85,7 +85,7 @@ struct AttnSmem {
   StageInfo info[kInfoSlots];
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t info_full[kInfoSlots];
-  uint64_t q_full, s_full[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per step parity
+  uint64_t q_full, s_full[2], s_free[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per step parity
   uint32_t tmem_base;
   int abort;
   int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
@@ -317,6 +317,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     mbar_init(smem_u32(&sm.q_full), 4);          // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.s_free[i]), 4);
       mbar_init(smem_u32(&sm.p_full[i]), 4);
       mbar_init(smem_u32(&sm.pv_done[i]), 1);
     }
@@ -388,8 +389,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     }
   } else if (warp == kWarpS) {
     // ------------------------------------------------------ S = Q K^T issuer
-    // S(j) goes to score buffer j & 1 once the softmax warps are done with
-    // S(j - 2) (p_full of step j - 2); Q of an item is in shared memory once
+    // S(j) goes to score buffer j & 1 once the softmax warps hold S(j - 2) in
+    // registers (s_free of step j - 2); Q of an item is in shared memory once
     // q_full completes.
     bool ok = true;
     if (lane == 0) {
@@ -402,7 +403,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         while (!last) {
           const int ks = j % kKStages;
           if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (j / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
-          if (j > 1 && !(ok = mbar_wait(smem_u32(&sm.p_full[j & 1]), ((j >> 1) - 1) & 1, &sm.abort, kTimeoutNs)))
+          if (j > 1 && !(ok = mbar_wait(smem_u32(&sm.s_free[j & 1]), ((j >> 1) - 1) & 1, &sm.abort, kTimeoutNs)))
             break;
           tc_fence_after();
           last = sm.info[j % kInfoSlots].last != 0;
@@ -564,10 +565,15 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         // exceeds 2^8 (then every P was at most 2^8: fine for bf16 and fp32).
         uint32_t pw[16];
         load_scores();
+        // the scores stay in registers for the rest of the step: S(j + 2) may
+        // overwrite the buffer. A warp reaches step j + 2 only after S(j + 2),
+        // which needed every warp's s_free of step j: arrivals stay in step order.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[j & 1]));
         if (__any_sync(0xffffffffu, ms == -INFINITY) && !(ok = exact_max())) break;
         float psum = exp_pass(x, c, ms, pw);
         if (__any_sync(0xffffffffu, psum + __shfl_xor_sync(0xffffffffu, psum, 16) > kPSumLimit)) {
-          load_scores();
           if (!(ok = exact_max())) break;
           psum = exp_pass(x, c, ms, pw);     // every P <= 1 now
         }
