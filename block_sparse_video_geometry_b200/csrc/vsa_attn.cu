@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 
@@ -86,6 +87,7 @@ struct AttnSmem {
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t info_full[kInfoSlots];
   uint64_t q_full, s_full[2], s_free[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per step parity
+  uint64_t never;                      // nothing arrives on it: the injected wait of vsa_debug_inject_wait_timeout
   uint32_t tmem_base;
   int abort;
   int2 cond[1];                        // conditioning tiles (first token, count); n_cond entries
@@ -128,6 +130,7 @@ struct AttnArgs {
   int64_t o_sb, o_ss, o_sh;
   float scale_log2;
   int* err;
+  uint64_t stall_ns;         // > 0: the S-issue warp first waits this long on a barrier nothing arrives on
 };
 
 // Work item = one query tile of one (batch, head).
@@ -324,6 +327,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     mbar_init(smem_u32(&sm.o_full), 1);
     mbar_init(smem_u32(&sm.drain_s), 1);
     mbar_init(smem_u32(&sm.drain_pv), 1);
+    mbar_init(smem_u32(&sm.never), 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -397,6 +401,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
       uint32_t j = 0;
       int it_n = 0;
       const uint64_t qd = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      // injected failure (vsa_debug_inject_wait_timeout): a bounded wait that runs out
+      if (a.stall_ns) ok = mbar_wait(smem_u32(&sm.never), 0, &sm.abort, a.stall_ns);
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
         if (!(ok = mbar_wait(smem_u32(&sm.q_full), it_n & 1, &sm.abort, kTimeoutNs))) break;
         bool last = false;
@@ -665,6 +671,8 @@ int sm_count() {
 }
 
 constexpr size_t kAttnHeader = 256;   // error word
+
+std::atomic<uint64_t> g_stall_ns{0};   // vsa_debug_inject_wait_timeout
 constexpr size_t kMaxAttnSmem = 227 * 1024;
 
 // Work decomposition shared by the host and the kernels (see decode_item).
@@ -790,6 +798,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.o_sh = o_sh;
   a.scale_log2 = effective_scale(p) * 1.4426950408889634f;
   a.err = static_cast<int*>(workspace);
+  a.stall_ns = g_stall_ns.load(std::memory_order_relaxed);
 
   cudaError_t e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -816,6 +825,11 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: launch", e);
   }
+  return VSA_OK;
+}
+
+vsa_status vsa_debug_inject_wait_timeout(uint64_t timeout_ns) {
+  g_stall_ns.store(timeout_ns, std::memory_order_relaxed);
   return VSA_OK;
 }
 

@@ -71,6 +71,7 @@ _SIGNATURES = {
                                    _P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64, _I64,
                                    _P, _SZ, _P]),
     "vsa_sparse_attn_status": (_I32, [_P, _P]),
+    "vsa_debug_inject_wait_timeout": (_I32, [ctypes.c_uint64]),
     "vsa_status_string": (ctypes.c_char_p, [_I32]),
     "vsa_version": (_I32, []),
     "vsa_last_error_detail": (ctypes.c_char_p, []),
@@ -235,6 +236,12 @@ def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: 
 def sparse_attn_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns the kernel's status word (OK or ERR_TIMEOUT)."""
     return lib().vsa_sparse_attn_status(workspace.data_ptr(), _stream_handle(stream))
+
+
+def debug_inject_wait_timeout(timeout_ns):
+    """Test hook: while timeout_ns > 0, each sparse_attn_fwd runs into a bounded
+    wait that nothing completes and reports ERR_TIMEOUT (see vsa.h); 0 disarms."""
+    lib().vsa_debug_inject_wait_timeout(int(timeout_ns))
 
 
 class Forward:

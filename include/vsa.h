@@ -281,6 +281,16 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* layout, const vsa_params* param
  * wait in the kernel ran out; the output is incomplete) or VSA_ERR_CUDA. */
 vsa_status vsa_sparse_attn_status(const void* workspace, cudaStream_t stream);
 
+/* vsa_debug_inject_wait_timeout: failure-injection hook for tests (no
+ * counterpart on the pages). While timeout_ns > 0, every vsa_sparse_attn_fwd
+ * of this process makes its MMA-issue warp wait, before any work, on a barrier
+ * that nothing arrives on, bounded by timeout_ns: the wait runs out, the kernel
+ * takes its abort path (drains its copies and MMAs, frees tensor memory, exits)
+ * and vsa_sparse_attn_status reports VSA_ERR_TIMEOUT; the output is not
+ * written. Nothing faults, traps or hangs, and the CUDA context stays usable.
+ * timeout_ns = 0 disarms it. Always returns VSA_OK. */
+vsa_status vsa_debug_inject_wait_timeout(uint64_t timeout_ns);
+
 const char* vsa_status_string(vsa_status status);
 
 /* Text of the most recent VSA_ERR_CUDA returned on the calling thread (the
