@@ -23,19 +23,22 @@
 //    every instruction it needs per step delays the copies).
 //  * Two CTAs per SM, each with 256 TMEM columns: O (128) and two 64-column
 //    score buffers, all M = 64 accumulators (rows in the first 16 lanes of each
-//    lane quadrant). Q and the bf16 P of the even / odd steps sit in shared
-//    memory; S(j + 2) reuses the score buffer of step j as soon as the softmax
-//    warps hold S(j) in registers, and P(j) waits only for O += P(j - 2) V.
-//  * Every tcgen05 instruction holds its issuing thread for about 46 cycles,
-//    so one warp issues the S MMAs and another the P V MMAs.
-//  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues S
-//    = Q K^T, 3 issues O += P V; 4-7 load each item's Q into shared memory,
-//    run the fp32 online softmax and the epilogue: two threads per row (the
-//    16x32bx2 TMEM shape gives the two half-warps the same 16 lanes at two
-//    column offsets), 32 keys each per step, exp2. P is computed against the
-//    running max; the exact row max of a step is only formed when a row's sum
-//    of P exceeds 2^8 (then O and the sum are rescaled and P recomputed),
-//    which keeps every P at most 2^8.
+//    lane quadrant); P of a step is written as bf16 pairs over the first 32
+//    columns of its own score buffer and is the TMEM operand of O += P V. Q and
+//    two K and two V stages sit in shared memory.
+//  * One warp issues every MMA, in the order ..., O += P(j - 1) V, S(j + 1),
+//    O += P(j) V, S(j + 2), ...; MMAs from one thread run in issue order, so
+//    S(j + 2) cannot overwrite P(j) early, and no issue waits for a completion.
+//    A K (V) stage is free again once S (O += P V) of its previous step has
+//    completed.
+//  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues the
+//    MMAs; 3-6 load each item's Q into shared memory, run the fp32 online
+//    softmax and the epilogue: two threads per row (the 16x32bx2 TMEM shape
+//    gives the two half-warps the same 16 lanes at two column offsets), 32 keys
+//    each per step, exp2. P is computed against the running max; the exact row
+//    max of a step is only formed when a row's sum of P exceeds 2^8 (then O
+//    and the sum are rescaled and P recomputed), which keeps every P at most
+//    2^8.
 //  * Every wait is bounded: a wait that runs out sets an error word in the
 //    workspace, raises an abort flag that ends the other roles' loops, drains
 //    in-flight copies and MMAs and frees TMEM before the block exits.
@@ -56,19 +59,18 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kKStages = 2;
-constexpr int kVStages = 2;
 constexpr int kInfoSlots = 8;        // info of step j is rewritten only after O += P(j) V was issued
-constexpr int kThreads = 256;
-constexpr int kWarpK = 0, kWarpV = 1, kWarpS = 2, kWarpPV = 3;   // warps 4..7: Q loads, softmax, epilogue
+constexpr int kThreads = 224;
+constexpr int kWarpK = 0, kWarpV = 1, kWarpMma = 2;   // warps 3..6: Q loads, softmax, epilogue
 constexpr uint32_t kTmemCols = 256;
 // M = 64 accumulators (rows in the first 16 lanes of each quadrant): O (fp32,
-// 128 columns) and the fp32 scores of the even / odd steps.
+// 128 columns) and the fp32 scores of the even / odd steps; P of a step is
+// written as bf16 pairs over the first 32 columns of its own score buffer.
 constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;
 constexpr uint32_t kTileBytes = 16384;    // one key tile of K or V: [d half 0][d half 1], 64 rows x 128 B
 constexpr float kPSumLimit = 256.0f;     // 2^8: see the softmax step
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, 0, 0);      // S = Q K^T, both K-major
-constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 128, 0, 1);    // O = P V, P K-major, V MN-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 128, 0, 1);    // O = P V, P K-major in TMEM, V MN-major
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
 
@@ -78,15 +80,15 @@ struct StageInfo {
   unsigned long long valid;
 };
 
+// K, V and the score buffers all go by step parity: stage / buffer j & 1.
 struct AttnSmem {
   uint8_t q[2][64 * 128];              // [d half][64 rows x 128 B], SW128 K-major
-  uint8_t p[2][64 * 128];              // P of the even / odd steps: 64 rows x 64 keys bf16, SW128 K-major
-  uint8_t k[kKStages][kTileBytes];
-  uint8_t v[kVStages][kTileBytes];
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
   StageInfo info[kInfoSlots];
-  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t k_full[2], v_full[2], s_full[2], p_full[2], pv_done[2];
   uint64_t info_full[kInfoSlots];
-  uint64_t q_full, s_full[2], s_free[2], p_full[2], pv_done[2], o_full, drain_s, drain_pv;   // [2]: per step parity
+  uint64_t q_full, o_full, drain;
   uint64_t never;                      // nothing arrives on it: the injected wait of vsa_debug_inject_wait_timeout
   uint32_t tmem_base;
   int abort;
@@ -294,8 +296,8 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_co
   if (threadIdx.x == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = n;
 }
 
-// 128 registers per thread: two CTAs of 256 threads fit one SM's register file.
-__global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArgs a) {
+// 144 registers per thread: two CTAs of 224 threads fit one SM's register file.
+__global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {          // swizzled tiles need 1024-byte alignment
     if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
@@ -308,30 +310,22 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
   for (int i = threadIdx.x; i < G.n_cond; i += kThreads)
     sm.cond[i] = make_int2(a.origin[i].x, a.count[i]);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(smem_u32(&sm.k_full[s]), 1);
-      mbar_init(smem_u32(&sm.k_empty[s]), 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
-      mbar_init(smem_u32(&sm.v_full[s]), 1);
-      mbar_init(smem_u32(&sm.v_empty[s]), 1);
-    }
-    for (int s = 0; s < kInfoSlots; ++s) mbar_init(smem_u32(&sm.info_full[s]), 1);
-    mbar_init(smem_u32(&sm.q_full), 4);          // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.k_full[i]), 1);
+      mbar_init(smem_u32(&sm.v_full[i]), 1);
       mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.s_free[i]), 4);
-      mbar_init(smem_u32(&sm.p_full[i]), 4);
+      mbar_init(smem_u32(&sm.p_full[i]), 4);     // one arrival per softmax warp
       mbar_init(smem_u32(&sm.pv_done[i]), 1);
     }
+    for (int s = 0; s < kInfoSlots; ++s) mbar_init(smem_u32(&sm.info_full[s]), 1);
+    mbar_init(smem_u32(&sm.q_full), 4);
     mbar_init(smem_u32(&sm.o_full), 1);
-    mbar_init(smem_u32(&sm.drain_s), 1);
-    mbar_init(smem_u32(&sm.drain_pv), 1);
+    mbar_init(smem_u32(&sm.drain), 1);
     mbar_init(smem_u32(&sm.never), 1);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpS) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -343,11 +337,13 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
   if (warp == kWarpK || warp == kWarpV) {
     // ----------------------------------------------------------- producers
     // Both stream the item's step records (one key tile each) and copy the
-    // tile's 16 KB block of K or V; the K warp also publishes per-step info.
+    // tile's 16 KB block of K or V into stage j & 1. A K stage is free again
+    // once S of its previous step has completed (s_full), a V stage once O +=
+    // P V of its previous step has (pv_done). The K warp also publishes
+    // per-step tile info.
     const bool is_k = warp == kWarpK;
     uint64_t* full = is_k ? sm.k_full : sm.v_full;
-    uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
-    const int nst = is_k ? kKStages : kVStages;
+    uint64_t* freed = is_k ? sm.s_full : sm.pv_done;
     uint32_t step = 0, issued = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
@@ -366,8 +362,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         }
         const int tile = __shfl_sync(0xffffffffu, cur.x, jj & 31);
         const int fl = __shfl_sync(0xffffffffu, cur.y, jj & 31);
-        const int st = step % nst;
-        if (!(ok = warp_wait(sm, empty[st], ((step / nst) & 1) ^ 1, lane, a.err))) break;
+        const int st = step & 1;
+        if (step >= 2 && !(ok = warp_wait(sm, freed[st], ((step >> 1) - 1) & 1, lane, a.err))) break;
         if (lane == 0) {
           if (is_k) {
             StageInfo& inf = sm.info[step % kInfoSlots];
@@ -388,84 +384,67 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
     }
     if (!ok && lane == 0) {
       // let every issued copy land before the block can exit
-      for (uint32_t i = (issued > static_cast<uint32_t>(nst) ? issued - nst : 0); i < issued; ++i)
-        mbar_wait(smem_u32(&full[i % nst]), (i / nst) & 1, nullptr, kDrainNs);
+      for (uint32_t i = (issued > 2u ? issued - 2u : 0u); i < issued; ++i)
+        mbar_wait(smem_u32(&full[i & 1]), (i >> 1) & 1, nullptr, kDrainNs);
     }
-  } else if (warp == kWarpS) {
-    // ------------------------------------------------------ S = Q K^T issuer
-    // S(j) goes to score buffer j & 1 once the softmax warps hold S(j - 2) in
-    // registers (s_free of step j - 2); Q of an item is in shared memory once
-    // q_full completes.
+  } else if (warp == kWarpMma) {
+    // ----------------------------------------------------------------- MMA
+    // One thread issues, in the order ..., O += P(j - 1) V, S(j + 1), O += P(j) V,
+    // S(j + 2), ... . P(j) sits over the first 32 columns of score buffer j & 1,
+    // and MMAs from one thread run in issue order, so S(j + 2) cannot overwrite
+    // P(j) before O += P(j) V has read it.
     bool ok = true;
     if (lane == 0) {
       uint32_t j = 0;
       int it_n = 0;
       const uint64_t qd = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      auto pv = [&](uint32_t t, bool first) -> bool {
+        const uint32_t b = t & 1;
+        if (!mbar_wait(smem_u32(&sm.p_full[b]), (t >> 1) & 1, &sm.abort, kTimeoutNs)) return false;
+        if (!mbar_wait(smem_u32(&sm.v_full[b]), (t >> 1) & 1, &sm.abort, kTimeoutNs)) return false;
+        tc_fence_after();
+        // V as MN-major B: 64-d blocks 8 KB apart, 16 keys = 2 KB per K step;
+        // P (A, in TMEM): 16 keys = 8 columns of bf16 pairs per K step
+        const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[b]), 8192, 1024);
+        const uint32_t pcol = tmem + (b ? kColS1 : kColS0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tmem + kColO, pcol + kk * 8, vd + kk * (2048 >> 4), kIdescPV, (first && kk == 0) ? 0u : 1u);
+        umma_commit(smem_u32(&sm.pv_done[b]));
+        return true;
+      };
       // injected failure (vsa_debug_inject_wait_timeout): a bounded wait that runs out
       if (a.stall_ns) ok = mbar_wait(smem_u32(&sm.never), 0, &sm.abort, a.stall_ns);
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
         if (!(ok = mbar_wait(smem_u32(&sm.q_full), it_n & 1, &sm.abort, kTimeoutNs))) break;
+        int jj = 0;
         bool last = false;
         while (!last) {
-          const int ks = j % kKStages;
-          if (!(ok = mbar_wait(smem_u32(&sm.k_full[ks]), (j / kKStages) & 1, &sm.abort, kTimeoutNs))) break;
-          if (j > 1 && !(ok = mbar_wait(smem_u32(&sm.s_free[j & 1]), ((j >> 1) - 1) & 1, &sm.abort, kTimeoutNs)))
-            break;
+          const uint32_t b = j & 1;
+          if (!(ok = mbar_wait(smem_u32(&sm.k_full[b]), (j >> 1) & 1, &sm.abort, kTimeoutNs))) break;
           tc_fence_after();
           last = sm.info[j % kInfoSlots].last != 0;
-          const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]), 16, 1024);
+          const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[b]), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             // 16 d per K step: 32 B inside a swizzle row of d half kk / 4
             // (descriptor addresses count 16-byte units)
-            umma_ss(tmem + ((j & 1) ? kColS1 : kColS0), qd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2,
+            umma_ss(tmem + (b ? kColS1 : kColS0), qd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2,
                     kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS, kk > 0 ? 1u : 0u);
           }
-          umma_commit(smem_u32(&sm.k_empty[ks]));
-          umma_commit(smem_u32(&sm.s_full[j & 1]));
-          ++j;
-        }
-      }
-      if (!ok) raise_abort(sm, a.err);
-      // drain: every MMA this thread issued has completed before TMEM is freed
-      umma_commit(smem_u32(&sm.drain_s));
-      mbar_wait(smem_u32(&sm.drain_s), 0, nullptr, kDrainNs);
-    }
-    __syncwarp();
-  } else if (warp == kWarpPV) {
-    // ----------------------------------------------------- O += P V issuer
-    // P(j) sits in shared-memory buffer j & 1. The first step of an item
-    // overwrites O; o_full fires after its last step.
-    bool ok = true;
-    if (lane == 0) {
-      uint32_t j = 0;
-      for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
-        bool first = true, last = false;
-        while (!last) {
-          const uint32_t pb = j & 1;           // P buffer of step j; its use count is j >> 1
-          if (!(ok = mbar_wait(smem_u32(&sm.p_full[pb]), (j >> 1) & 1, &sm.abort, kTimeoutNs))) break;
-          last = sm.info[j % kInfoSlots].last != 0;   // read by the softmax warps before p_full
-          const int vs = j % kVStages;
-          if (!(ok = mbar_wait(smem_u32(&sm.v_full[vs]), (j / kVStages) & 1, &sm.abort, kTimeoutNs))) break;
-          tc_fence_after();
-          // P: 64 rows x 64 keys, K-major; V as MN-major B: 64-d blocks 8 KB apart,
-          // 16 keys = 32 B of P and 2 KB of V per K step
-          const uint64_t pd = smem_desc_sw128(smem_u32(sm.p[pb]), 16, 1024);
-          const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[vs]), 8192, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_ss(tmem + kColO, pd + kk * 2, vd + kk * (2048 >> 4), kIdescPV, (first && kk == 0) ? 0u : 1u);
-          first = false;
-          umma_commit(smem_u32(&sm.v_empty[vs]));
-          umma_commit(smem_u32(&sm.pv_done[pb]));
+          umma_commit(smem_u32(&sm.s_full[b]));
+          if (jj > 0 && !(ok = pv(j - 1, jj == 1))) break;
+          ++jj;
           ++j;
         }
         if (!ok) break;
+        if (!(ok = pv(j - 1, jj == 1))) break;
         umma_commit(smem_u32(&sm.o_full));
       }
       if (!ok) raise_abort(sm, a.err);
-      umma_commit(smem_u32(&sm.drain_pv));
-      mbar_wait(smem_u32(&sm.drain_pv), 0, nullptr, kDrainNs);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      umma_commit(smem_u32(&sm.drain));
+      mbar_wait(smem_u32(&sm.drain), 0, nullptr, kDrainNs);
     }
     __syncwarp();
   } else {
@@ -515,24 +494,20 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         last = inf.last != 0;
         if (!s_ready && !(ok = warp_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, lane, a.err))) break;
         tc_fence_after();
-        uint32_t t_info = 0, t_s = 0, t_pv = 1;
+        uint32_t t_info = 0, t_s = 0;
         if (!last) {
           t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
           t_s = mbar_test_wait(smem_u32(&sm.s_full[(j + 1) & 1]), ((j + 1) >> 1) & 1);
         }
-        // O += P(j - 2) V has read P buffer j & 1 (the use count of a buffer is j >> 1)
-        if (j > 1) t_pv = mbar_test_wait(smem_u32(&sm.pv_done[j & 1]), ((j >> 1) - 1) & 1);
         const uint32_t scol = lane_addr + ((j & 1) ? kColS1 : kColS0);
         float x[32];
-        auto load_scores = [&]() {
-          tmem_ld16x2_32f<32>(scol, x);
-          tmem_wait_ld();
-          if (inf.valid != ~0ull) {           // padding slots never attend
-            const uint32_t vm = static_cast<uint32_t>(inf.valid >> (32 * hf));
+        tmem_ld16x2_32f<32>(scol, x);
+        tmem_wait_ld();
+        if (inf.valid != ~0ull) {             // padding slots never attend
+          const uint32_t vm = static_cast<uint32_t>(inf.valid >> (32 * hf));
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = ((vm >> i) & 1u) ? x[i] : -INFINITY;
-          }
-        };
+          for (int i = 0; i < 32; ++i) x[i] = ((vm >> i) & 1u) ? x[i] : -INFINITY;
+        }
         // exact row max of the step; O and l rescaled when it raises the running max
         auto exact_max = [&]() -> bool {
           float m = x[0];
@@ -542,8 +517,8 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           const bool need = ms != -INFINITY && mt > ms;
           if (ms == -INFINITY) ms = mt;       // first key tile of this row: O and l are still zero
           if (__any_sync(0xffffffffu, need)) {
-            // rescale this half row of O once every earlier P V has landed: the
-            // last one is O += P(j - 1) V, which follows O += P(j - 2) V in issue order
+            // rescale this half row of O once every earlier P V has landed (the
+            // last one, O += P(j - 1) V, was issued after all the others)
             if (j > 0 && !warp_wait(sm, sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lane, a.err)) return false;
             tc_fence_after();
             const float f = need ? ex2_approx(ms - mt) : 1.0f;
@@ -570,13 +545,6 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         // is only formed when a row has no reference yet, or when its P sum
         // exceeds 2^8 (then every P was at most 2^8: fine for bf16 and fp32).
         uint32_t pw[16];
-        load_scores();
-        // the scores stay in registers for the rest of the step: S(j + 2) may
-        // overwrite the buffer. A warp reaches step j + 2 only after S(j + 2),
-        // which needed every warp's s_free of step j: arrivals stay in step order.
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[j & 1]));
         if (__any_sync(0xffffffffu, ms == -INFINITY) && !(ok = exact_max())) break;
         float psum = exp_pass(x, c, ms, pw);
         if (__any_sync(0xffffffffu, psum + __shfl_xor_sync(0xffffffffu, psum, 16) > kPSumLimit)) {
@@ -584,21 +552,13 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
           psum = exp_pass(x, c, ms, pw);     // every P <= 1 now
         }
         l += psum;
-        // P(j - 2), in the buffer P(j) goes to, has been consumed once its P V
-        // completed; that completion also needs every warp's P(j - 2), so this
-        // warp's arrivals on p_full[j & 1] stay in step order
-        if (j > 1 && !__all_sync(0xffffffffu, t_pv) &&
-            !(ok = warp_wait(sm, sm.pv_done[j & 1], ((j >> 1) - 1) & 1, lane, a.err)))
-          break;
-        {
-          // this half row of P: 32 keys = 64 B = 16-byte chunks 4 hf .. 4 hf + 3 of row r
-          uint8_t* prow = sm.p[j & 1] + r * 128;
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            *reinterpret_cast<uint4*>(prow + (((4 * hf + cc) ^ (r & 7)) << 4)) =
-                make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
-        }
-        fence_proxy_async_smem();
+        // P(j) over the first 32 columns of its own score buffer (this half row:
+        // keys 32 hf..32 hf + 31 = columns 16 hf..16 hf + 15); the scores were
+        // read above. A warp reaches step j + 2 only after S(j + 2), issued after
+        // O += P(j) V, which needed every warp's P(j): arrivals on p_full[j & 1]
+        // stay in step order.
+        tmem_st16x2_16<16>(scol, pw);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[j & 1]));
@@ -656,7 +616,7 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpS) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
