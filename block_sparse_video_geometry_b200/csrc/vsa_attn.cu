@@ -63,13 +63,19 @@ constexpr int kInfoSlots = 8;        // info of step j is rewritten only after O
 constexpr int kThreads = 224;
 constexpr int kWarpK = 0, kWarpV = 1, kWarpMma = 2;   // warps 3..6: Q loads, softmax, epilogue
 constexpr uint32_t kTmemCols = 256;
-// M = 64 accumulators (rows in the first 16 lanes of each quadrant): O (fp32,
-// 128 columns) and the fp32 scores of the even / odd steps; P of a step is
-// written as bf16 pairs over the first 32 columns of its own score buffer.
-constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 192;
+// An M = 64 operand or accumulator takes 16 lanes of each 32-lane quadrant
+// (row r at lane 32 (r / 16) + r % 16 + lane offset). Both 16-lane halves are
+// used: even steps run in half 0 (lane offset 0), odd steps in half 1 (lane
+// offset 16). Each half holds a copy of Q (bf16 pairs, 64 columns), the O of
+// its own steps (fp32, 128 columns) and the scores S of its current step
+// (fp32, 64 columns), overwritten in place by P (bf16 pairs, 32 columns). An
+// MMA with A in TMEM needs A and D in the same lanes, which each half keeps;
+// the output is O(half 0) + O(half 1).
+constexpr uint32_t kColQ = 0, kColO = 64, kColS = 192;
+constexpr uint32_t kHalfLanes = 16u << 16;
 constexpr uint32_t kTileBytes = 16384;    // one key tile of K or V: [d half 0][d half 1], 64 rows x 128 B
 constexpr float kPSumLimit = 256.0f;     // 2^8: see the softmax step
-constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, 0, 0);      // S = Q K^T, both K-major
+constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, 0, 0);      // S = Q K^T: Q K-major in TMEM, K K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 128, 0, 1);    // O = P V, P K-major in TMEM, V MN-major
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
@@ -80,9 +86,8 @@ struct StageInfo {
   unsigned long long valid;
 };
 
-// K, V and the score buffers all go by step parity: stage / buffer j & 1.
+// K and V stages and the TMEM halves all go by step parity: stage / half j & 1.
 struct AttnSmem {
-  uint8_t q[2][64 * 128];              // [d half][64 rows x 128 B], SW128 K-major
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
   StageInfo info[kInfoSlots];
@@ -209,16 +214,6 @@ __device__ __forceinline__ bool warp_wait(AttnSmem& sm, uint64_t& bar, uint32_t 
   ok = __shfl_sync(0xffffffffu, ok, 0);
   __syncwarp();
   return ok != 0;
-}
-
-// Sets the scores of the key slots whose bit in `valid` is clear to -inf.
-__device__ __forceinline__ void mask_invalid(float (&x)[64], unsigned long long valid) {
-  const uint32_t lo = static_cast<uint32_t>(valid), hi = static_cast<uint32_t>(valid >> 32);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    x[i] = ((lo >> i) & 1u) ? x[i] : -INFINITY;
-    x[32 + i] = ((hi >> i) & 1u) ? x[32 + i] : -INFINITY;
-  }
 }
 
 // bf16 pairs of P = 2^(x c - ms) for 32 keys; returns the fp32 sum of P.
@@ -390,14 +385,13 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
   } else if (warp == kWarpMma) {
     // ----------------------------------------------------------------- MMA
     // One thread issues, in the order ..., O += P(j - 1) V, S(j + 1), O += P(j) V,
-    // S(j + 2), ... . P(j) sits over the first 32 columns of score buffer j & 1,
-    // and MMAs from one thread run in issue order, so S(j + 2) cannot overwrite
-    // P(j) before O += P(j) V has read it.
+    // S(j + 2), ... . P(j) sits over the scores of TMEM half j & 1, and MMAs
+    // from one thread run in issue order, so S(j + 2) cannot overwrite P(j)
+    // before O += P(j) V has read it.
     bool ok = true;
     if (lane == 0) {
       uint32_t j = 0;
       int it_n = 0;
-      const uint64_t qd = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
       auto pv = [&](uint32_t t, bool first) -> bool {
         const uint32_t b = t & 1;
         if (!mbar_wait(smem_u32(&sm.p_full[b]), (t >> 1) & 1, &sm.abort, kTimeoutNs)) return false;
@@ -406,10 +400,10 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
         // V as MN-major B: 64-d blocks 8 KB apart, 16 keys = 2 KB per K step;
         // P (A, in TMEM): 16 keys = 8 columns of bf16 pairs per K step
         const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[b]), 8192, 1024);
-        const uint32_t pcol = tmem + (b ? kColS1 : kColS0);
+        const uint32_t half = tmem + (b ? kHalfLanes : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tmem + kColO, pcol + kk * 8, vd + kk * (2048 >> 4), kIdescPV, (first && kk == 0) ? 0u : 1u);
+          umma_ts(half + kColO, half + kColS + kk * 8, vd + kk * (2048 >> 4), kIdescPV, (first && kk == 0) ? 0u : 1u);
         umma_commit(smem_u32(&sm.pv_done[b]));
         return true;
       };
@@ -425,20 +419,22 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
           tc_fence_after();
           last = sm.info[j % kInfoSlots].last != 0;
           const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[b]), 16, 1024);
+          const uint32_t half = tmem + (b ? kHalfLanes : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            // 16 d per K step: 32 B inside a swizzle row of d half kk / 4
-            // (descriptor addresses count 16-byte units)
-            umma_ss(tmem + (b ? kColS1 : kColS0), qd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2,
-                    kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS, kk > 0 ? 1u : 0u);
+            // 16 d per K step: 8 columns of Q pairs; 32 B inside a swizzle
+            // row of K's d half kk / 4 (descriptor addresses count 16-byte units)
+            umma_ts(half + kColS, half + kColQ + kk * 8, kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS,
+                    kk > 0 ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm.s_full[b]));
-          if (jj > 0 && !(ok = pv(j - 1, jj == 1))) break;
+          // the first two steps of an item start the O of their halves
+          if (jj > 0 && !(ok = pv(j - 1, jj <= 2))) break;
           ++jj;
           ++j;
         }
         if (!ok) break;
-        if (!(ok = pv(j - 1, jj == 1))) break;
+        if (!(ok = pv(j - 1, jj <= 2))) break;
         umma_commit(smem_u32(&sm.o_full));
       }
       if (!ok) raise_abort(sm, a.err);
@@ -449,9 +445,10 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
     __syncwarp();
   } else {
     // ------------------------------------------------ Q / softmax / epilogue
-    // M = 64 layout: warp q (TMEM lanes 32q..32q+31) owns rows 16q..16q+15 in
-    // its first 16 lanes; thread t handles row 16q + (t & 15) and the key (or
-    // output column) half t >> 4, its partner is thread t ^ 16.
+    // M = 64 layout: warp q (TMEM lanes 32q..32q+31) owns rows 16q..16q+15, in
+    // lanes 32q..32q+15 for even steps and 32q+16..32q+31 for odd steps;
+    // thread t handles row 16q + (t & 15) and the key (or output column) half
+    // t >> 4, its partner is thread t ^ 16.
     const int quad = warp & 3;
     const int hf = lane >> 4;                        // 0: keys 0..31 / d 0..63, 1: keys 32..63 / d 64..127
     const int r = quad * 16 + (lane & 15);           // row of the 64-row tile
@@ -465,18 +462,27 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
       const bool row_ok = (tile_mask(sm, G, it.qt) >> r) & 1ull;
       const int64_t tok = row_ok ? tile_token(sm, G, it.qt, r) : 0;
       {
-        // this row's half of Q (d in [64 hf, 64 hf + 64)) into shared memory,
-        // 128-byte swizzled (every MMA of the previous item has completed)
+        // this row's half of Q (d in [64 hf, 64 hf + 64): columns 32 hf ..
+        // 32 hf + 31 of bf16 pairs) into both TMEM halves (every MMA of the
+        // previous item has completed)
         const uint4* src = reinterpret_cast<const uint4*>(a.q + tok * a.q_ss + it.h * a.q_sh + 64 * hf);
-        uint4 w[8];
+        uint32_t w[32];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) w[cc] = row_ok ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(&sm.q[hf][r * 128 + ((cc ^ (r & 7)) << 4)]) = w[cc];
-        fence_proxy_async_smem();
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 u = row_ok ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * cc] = u.x;
+          w[4 * cc + 1] = u.y;
+          w[4 * cc + 2] = u.z;
+          w[4 * cc + 3] = u.w;
+        }
+        tmem_st16x2_32<32>(lane_addr + kColQ, w);
+        tmem_st16x2_32<32>(lane_addr + kHalfLanes + kColQ, w);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.q_full));
       }
+      const uint32_t j0 = j;               // first step of the item
       float ms = -INFINITY, l = 0.f;        // running max (scaled, log2 domain, same in both halves) and half sum
       bool last = false;
       // barrier phases of the next step are tested (without blocking) early in
@@ -499,7 +505,7 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
           t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
           t_s = mbar_test_wait(smem_u32(&sm.s_full[(j + 1) & 1]), ((j + 1) >> 1) & 1);
         }
-        const uint32_t scol = lane_addr + ((j & 1) ? kColS1 : kColS0);
+        const uint32_t scol = lane_addr + ((j & 1) ? kHalfLanes : 0u) + kColS;
         float x[32];
         tmem_ld16x2_32f<32>(scol, x);
         tmem_wait_ld();
@@ -522,15 +528,18 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
             if (j > 0 && !warp_wait(sm, sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lane, a.err)) return false;
             tc_fence_after();
             const float f = need ? ex2_approx(ms - mt) : 1.0f;
+            // both halves (a half not yet started by this item holds stale
+            // values that its first O += P V overwrites)
 #pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint32_t oa = lane_addr + ((ch & 2) ? kHalfLanes : 0u) + kColO + 32 * (ch & 1);
               float u[32];
-              tmem_ld16x2_32f<64>(lane_addr + kColO + 32 * ch, u);
+              tmem_ld16x2_32f<64>(oa, u);
               tmem_wait_ld();
               uint32_t w[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(u[i] * f);
-              tmem_st16x2_32<64>(lane_addr + kColO + 32 * ch, w);
+              tmem_st16x2_32<64>(oa, w);
             }
             tmem_wait_st();
             if (need) {
@@ -552,7 +561,7 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
           psum = exp_pass(x, c, ms, pw);     // every P <= 1 now
         }
         l += psum;
-        // P(j) over the first 32 columns of its own score buffer (this half row:
+        // P(j) over the first 32 score columns of its TMEM half (this half row:
         // keys 32 hf..32 hf + 31 = columns 16 hf..16 hf + 15); the scores were
         // read above. A warp reaches step j + 2 only after S(j + 2), issued after
         // O += P(j) V, which needed every warp's P(j): arrivals on p_full[j & 1]
@@ -578,11 +587,23 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
         gate = __uint_as_float(static_cast<uint32_t>(a.g[a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh]) << 16);
         oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + it.qt) * kHeadDim + 64 * hf;
       }
+      // O = O(half of step j0) + O(other half) when the item had two steps or more
+      const uint32_t o_first = lane_addr + ((j0 & 1) ? kHalfLanes : 0u) + kColO;
+      const uint32_t o_second = lane_addr + ((j0 & 1) ? 0u : kHalfLanes) + kColO;
+      const bool two_halves = j - j0 >= 2;
 #pragma unroll 1
       for (int ch = 0; ch < 2; ++ch) {
         float y[32];
-        tmem_ld16x2_32f<64>(lane_addr + kColO + 32 * ch, y);
-        tmem_wait_ld();
+        tmem_ld16x2_32f<64>(o_first + 32 * ch, y);
+        if (two_halves) {
+          float z[32];
+          tmem_ld16x2_32f<64>(o_second + 32 * ch, z);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] += z[i];
+        } else {
+          tmem_wait_ld();
+        }
         if (row_ok) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] *= inv_l;
