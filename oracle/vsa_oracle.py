@@ -28,10 +28,13 @@ What it computes, step by step, in the order the pages describe it:
 4. Fine branch: exact softmax attention of each query token over every
    conditioning key token plus the tokens of the selected video tiles
    (sink_conditioning = exact_kv). With exact_kv_and_rows the conditioning query
-   rows attend to the whole sequence. ("BSAI FastH3 Native VSA (recipe)",
-   "The inputs that matter", sink_conditioning.)
+   rows attend to the whole sequence. With sink_conditioning = off no key tile
+   is protected: conditioning tiles are scored, selected and summarised like
+   video tiles. ("BSAI FastH3 Native VSA (recipe)", "The inputs that matter",
+   sink_conditioning.)
 5. Output: o = o_fine + g * o_coarse, g a per-token, per-head gate given as an
-   input (the to_gate_compress output).
+   input (the to_gate_compress output), either one value per (token, head) or
+   one per (token, head, channel).
 
 Where the pages leave a step open this module takes the plainest reading and
 says so in the docstring of the function concerned. Every floating-point step
@@ -52,7 +55,7 @@ HEAD_DIM = 128     # head_dim of the native kernel ("BSAI FastH3 Native VSA", ba
 SEG_TEXT, SEG_REF_IMAGE, SEG_REF_AUDIO, SEG_OTHER_COND, SEG_VIDEO = 0, 1, 2, 3, 4
 
 MODE_TOPK, MODE_ADAPTIVE = 0, 1
-SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS = 0, 1
+SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS, SINK_OFF = 0, 1, 2
 
 
 # --------------------------------------------------------------------------- #
@@ -208,14 +211,32 @@ def default_scale(head_dim: int = HEAD_DIM) -> float:
     return 1.0 / math.sqrt(head_dim)
 
 
-def tile_scores(qbar: np.ndarray, kbar: np.ndarray, layout: Layout, scale: float) -> np.ndarray:
-    """s[qt, v] = scale * <qbar[qt], kbar[n_cond + v]> for every query tile qt and
-    every VIDEO key tile v (column v is video tile ordinal v, tile id n_cond+v).
+def candidate_tiles(layout: Layout, sink: int) -> tuple[int, int]:
+    """(first tile id, count) of the key tiles that are scored, selected and
+    summarised by the coarse branch.
+
+    exact_kv and exact_kv_and_rows protect the conditioning keys, so only the
+    video tiles are candidates ("Video-Only Sparse Attention"). Reading of
+    sink_conditioning = off ("cheapest", "The inputs that matter"): nothing is
+    protected, so every tile, conditioning or video, is a candidate on equal
+    terms and no key is attended exactly unless its tile is selected.
+    """
+    if sink == SINK_OFF:
+        return 0, layout.n_tiles
+    return layout.n_cond_tiles, layout.n_video_tiles
+
+
+def tile_scores(qbar: np.ndarray, kbar: np.ndarray, layout: Layout, scale: float,
+                sink: int = SINK_EXACT_KV) -> np.ndarray:
+    """s[qt, c] = scale * <qbar[qt], kbar[first + c]> for every query tile qt and
+    every candidate key tile c (see candidate_tiles; with the conditioning
+    protected, column c is video tile ordinal c, tile id n_cond + c).
 
     Reading: the score is the scaled logit of the pooled query against the
-    pooled key; only video key tiles are scored because only they are pruned.
+    pooled key; only candidate key tiles are scored because only they are pruned.
     """
-    kv = kbar[layout.n_cond_tiles:]
+    first, count = candidate_tiles(layout, sink)
+    kv = kbar[first:first + count]
     return scale * (qbar @ kv.T)
 
 
@@ -271,14 +292,17 @@ def select_adaptive(scores: np.ndarray, tau: float) -> tuple[list[np.ndarray], f
     return out, thr
 
 
-def coarse_branch(scores: np.ndarray, vbar: np.ndarray, layout: Layout) -> np.ndarray:
-    """o_coarse[qt] = sum_v softmax_v(s[qt, :]) * vbar[n_cond + v].
+def coarse_branch(scores: np.ndarray, vbar: np.ndarray, layout: Layout,
+                  sink: int = SINK_EXACT_KV) -> np.ndarray:
+    """o_coarse[qt] = sum_c softmax_c(s[qt, :]) * vbar[first + c].
 
-    Reading: the compressed branch attends, at tile resolution, to every video
-    key tile with the same scores used for selection; its query is the pooled
-    query of the tile, broadcast to the tile's tokens.
+    Reading: the compressed branch attends, at tile resolution, to every
+    candidate key tile (the video tiles, or every tile with sink off) with the
+    same scores used for selection; its query is the pooled query of the tile,
+    broadcast to the tile's tokens.
     """
-    vv = vbar[layout.n_cond_tiles:]
+    first, count = candidate_tiles(layout, sink)
+    vv = vbar[first:first + count]
     m = scores.max(axis=1, keepdims=True)
     p = np.exp(scores - m)
     p /= p.sum(axis=1, keepdims=True)
@@ -293,15 +317,17 @@ def key_tokens_for_tile(layout: Layout, qt: int, selected: np.ndarray, sink: int
 
     exact_kv: every conditioning token plus the tokens of the selected video
     tiles. exact_kv_and_rows: a conditioning query tile attends every token.
-    Reading: under exact_kv the conditioning query tiles are treated like video
-    query tiles (the pages only say that video queries see the conditioning
-    rows exactly).
+    off: the tokens of the selected tiles only (candidate ordinals, see
+    candidate_tiles). Reading: under exact_kv and off the conditioning query
+    tiles are treated like video query tiles (the pages only say that video
+    queries see the conditioning rows exactly).
     """
     if sink == SINK_EXACT_KV_AND_ROWS and qt < layout.n_cond_tiles:
         return np.arange(layout.seq_len, dtype=np.int64)
-    parts = [layout.cond_tokens()]
-    for v in selected:
-        parts.append(layout.tile_tokens(layout.n_cond_tiles + int(v)))
+    first, _ = candidate_tiles(layout, sink)
+    parts = [] if sink == SINK_OFF else [layout.cond_tokens()]
+    for c in selected:
+        parts.append(layout.tile_tokens(first + int(c)))
     return np.concatenate(parts)
 
 
@@ -351,13 +377,13 @@ def selection_for_head(q, k, v, layout: Layout, params: Params):
     """Steps 2-3 for one (batch, head): pooled Q/K/V, scores, selection, coarse."""
     scale = params.scale if params.scale > 0 else default_scale(q.shape[1])
     qbar, kbar, vbar = pool_tiles(q, layout), pool_tiles(k, layout), pool_tiles(v, layout)
-    scores = tile_scores(qbar, kbar, layout, scale)
+    scores = tile_scores(qbar, kbar, layout, scale, params.sink)
     if params.mode == MODE_TOPK:
-        sel = select_topk(scores, topk_count(params.keep, layout.n_video_tiles))
+        sel = select_topk(scores, topk_count(params.keep, candidate_tiles(layout, params.sink)[1]))
         thr = None
     else:
         sel, thr = select_adaptive(scores, params.tau)
-    o_coarse = coarse_branch(scores, vbar, layout)
+    o_coarse = coarse_branch(scores, vbar, layout, params.sink)
     return qbar, kbar, vbar, scores, sel, thr, o_coarse, scale
 
 
@@ -365,9 +391,10 @@ def output_rows_for_tile(q, k, v, g, layout: Layout, params: Params, qt: int,
                          selected: np.ndarray, o_coarse: np.ndarray, scale: float):
     """o_fine and out for the valid query tokens of tile qt.
 
-    out = o_fine + g * o_coarse[qt]; under exact_kv_and_rows the conditioning
-    query rows get the dense result only (no coarse term; reading: they are
-    run dense, and dense attention has no compressed branch).
+    out = o_fine + g * o_coarse[qt], g [S] (one gate per token, broadcast over
+    the head dimension) or [S, D] (one per channel); under exact_kv_and_rows
+    the conditioning query rows get the dense result only (no coarse term;
+    reading: they are run dense, and dense attention has no compressed branch).
     Returns (tokens, o_fine, out).
     """
     keys = key_tokens_for_tile(layout, qt, selected, params.sink)
@@ -376,14 +403,15 @@ def output_rows_for_tile(q, k, v, g, layout: Layout, params: Params, qt: int,
     if params.sink == SINK_EXACT_KV_AND_ROWS and qt < layout.n_cond_tiles:
         out = of.copy()
     else:
-        out = of + np.asarray(g, dtype=np.float64)[toks][:, None] * o_coarse[qt][None, :]
+        gt = np.asarray(g, dtype=np.float64)[toks]
+        out = of + (gt if gt.ndim == 2 else gt[:, None]) * o_coarse[qt][None, :]
     return toks, of, out
 
 
 def vsa_forward_head(q, k, v, g, layout: Layout, params: Params, tiles=None) -> HeadResult:
     """The whole forward pass for one (batch, head) slice.
 
-    q, k, v: [S, D] float64; g: [S] float64. If `tiles` is given, the fine
+    q, k, v: [S, D] float64; g: [S] or [S, D] float64. If `tiles` is given, the fine
     branch and output are computed for those query tiles only (rows of other
     tiles are left as NaN).
     """

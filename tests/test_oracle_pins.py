@@ -322,6 +322,76 @@ def test_gate_zero_and_one():
     assert np.allclose(r1.out, r1.o_fine + r1.o_coarse[tile], atol=1e-13)
 
 
+# ------------------------------------------------- sink off, channel gate --
+def test_sink_off_fine_equals_masked_dense_brute_force():
+    """sink off: a query attends exactly the tokens of its selected tiles and
+    nothing else; the mask is built from the token -> tile map alone."""
+    wl, lay, q, k, v, g = _tiny_case()
+    p = O.Params(keep=0.25, sink=O.SINK_OFF)
+    res = O.vsa_forward_head(q, k, v, g, lay, p)
+    S = lay.seq_len
+    tile = lay.inv // O.TILE
+    mask = np.zeros((S, S), bool)
+    for i in range(S):
+        for c in res.selected[tile[i]]:
+            mask[i, tile == c] = True                  # candidate ordinal = tile id
+    ref = O.dense_attention_masked(q, k, v, mask, O.default_scale())
+    assert np.allclose(res.o_fine, ref, atol=1e-12)
+
+
+def test_sink_off_selects_over_every_tile():
+    wl, lay, q, k, v, g = _tiny_case()
+    nt = lay.n_tiles
+    assert nt == 11
+    res = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.25, sink=O.SINK_OFF))
+    assert res.scores.shape == (nt, nt)
+    for qt in range(nt):
+        assert len(res.selected[qt]) == math.ceil(0.25 * nt) == 3
+        assert all(0 <= c < nt for c in res.selected[qt])
+    # brute force: the three highest scores of each row, ties to the lower tile
+    for qt in range(nt):
+        row = [(-res.scores[qt, c], c) for c in range(nt)]
+        assert sorted(c for _, c in sorted(row)[:3]) == list(res.selected[qt])
+    # a conditioning tile is selected somewhere (the tiny inputs give it the chance)
+    assert any(c < lay.n_cond_tiles for sel in res.selected for c in sel)
+
+
+def test_sink_off_keep_all_is_dense_attention():
+    wl, lay, q, k, v, g = _tiny_case()
+    res = O.vsa_forward_head(q, k, v, np.zeros_like(g), lay, O.Params(keep=1.0, sink=O.SINK_OFF))
+    assert np.allclose(res.out, O.softmax_attention(q, k, v, O.default_scale()), atol=1e-12)
+
+
+def test_sink_off_coarse_is_tile_resolution_attention_over_all_tiles():
+    wl = W.WORKLOADS["tiny"]
+    lay = layout_of(wl)
+    rng = np.random.default_rng(11)
+    qc, kc, vc = (rng.standard_normal((lay.n_tiles, 128)) for _ in range(3))
+    tile = lay.inv // O.TILE
+    q, k, v = qc[tile], kc[tile], vc[tile]
+    scale = O.default_scale()
+    s = O.tile_scores(O.pool_tiles(q, lay), O.pool_tiles(k, lay), lay, scale, O.SINK_OFF)
+    oc = O.coarse_branch(s, O.pool_tiles(v, lay), lay, O.SINK_OFF)
+    assert np.allclose(oc, O.softmax_attention(qc, kc, vc, scale), atol=1e-12)
+
+
+def test_channel_gate():
+    """g [S, D]: constant over channels equals the per-token gate; a one-hot
+    channel gate adds the coarse term to that channel only."""
+    wl, lay, q, k, v, g = _tiny_case()
+    p = O.Params(keep=0.5)
+    r_tok = O.vsa_forward_head(q, k, v, g, lay, p)
+    r_ch = O.vsa_forward_head(q, k, v, np.repeat(g[:, None], 128, axis=1), lay, p)
+    assert np.array_equal(r_tok.out, r_ch.out)
+    onehot = np.zeros((lay.seq_len, 128))
+    onehot[:, 37] = 2.0
+    r1 = O.vsa_forward_head(q, k, v, onehot, lay, p)
+    tile = lay.inv // O.TILE
+    d = r1.out - r1.o_fine
+    assert np.array_equal(np.delete(d, 37, axis=1), np.zeros((lay.seq_len, 127)))
+    assert np.allclose(d[:, 37], 2.0 * r1.o_coarse[tile][:, 37], atol=1e-14)
+
+
 # ------------------------------------------------------------- generator --
 def test_generator_is_seeded_and_bf16_rounded():
     import torch
