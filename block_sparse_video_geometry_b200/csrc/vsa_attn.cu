@@ -122,6 +122,8 @@ struct AttnArgs {
   int64_t q_ss, q_sh;
   int32_t H, b, sink, kmax;
   int32_t c0;                // first query tile of the sparse item range
+  int32_t n_fixed;           // key tiles every sparse item attends first (conditioning tiles, or none)
+  int32_t cand0, n_cand;     // candidate key tiles: tile ids cand0 .. cand0 + n_cand - 1
   int32_t nq_dense, nq_sparse, n_dense_items, n_items;   // query tiles per head: dense rows, sparse rows
   const int32_t* idx;         // selection lists (read by schedule_kernel)
   const int32_t* cnt;
@@ -131,7 +133,7 @@ struct AttnArgs {
   int32_t max_steps;
   const float* o_coarse;
   const uint16_t* g;
-  int64_t g_sb, g_ss, g_sh;
+  int64_t g_sb, g_ss, g_sh, g_sd;   // g_sd = 0: one gate per (token, head)
   void* out;
   int32_t out_bf16;
   int64_t o_sb, o_ss, o_sh;
@@ -261,15 +263,16 @@ permute_kv_kernel(DevLayout L, const uint16_t* __restrict__ k, const uint16_t* _
 // Step schedule of each work item, built once per call so that the copy warps
 // of the attention kernel only stream records. Record = (key tile, flags): bit 4
 // last step of the item, bit 5 the key tile has padding slots. Key tiles come in
-// the item's order: the dense part (conditioning tiles, or all tiles for dense
-// rows), then the query tile's selection list (ascending video ordinals).
+// the item's order: the dense part (the conditioning tiles unless the sink mode
+// is off, or all tiles for dense rows), then the query tile's selection list
+// (ascending candidate ordinals).
 constexpr int kSchedThreads = 128;
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_constant__ AttnArgs a) {
   const int item = blockIdx.x, b = blockIdx.y;
   const Geom& G = a.G;
   const Item it = decode_item(a, item);
-  const int n_dense = it.dense ? G.n_tiles : G.n_cond;
+  const int n_dense = it.dense ? G.n_tiles : a.n_fixed;
   const size_t row = (static_cast<size_t>(b) * a.H + it.h) * G.n_tiles + it.qt;
   const int n_sel = it.dense ? 0 : min(max(a.cnt[row], 0), a.kmax);
   const int n = n_dense + n_sel;
@@ -279,9 +282,9 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_co
     if (r < n_dense) {
       t = r;
     } else {
-      // entries outside [0, n_video) (never written by vsa_coarse_select) are clamped: memory stays in bounds
-      const int v = a.idx[row * a.kmax + (r - n_dense)];
-      t = G.n_cond + min(max(v, 0), G.n_video - 1);
+      // entries outside [0, n_cand) (never written by vsa_coarse_select) are clamped: memory stays in bounds
+      const int c = a.idx[row * a.kmax + (r - n_dense)];
+      t = a.cand0 + min(max(c, 0), a.n_cand - 1);
     }
     uint32_t fl = 0u;
     if (r == n - 1) fl |= 16u;
@@ -583,8 +586,11 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
       const float inv_l = 1.0f / (l + __shfl_xor_sync(0xffffffffu, l, 16));
       float gate = 0.f;
       const float* oc = nullptr;
+      const uint16_t* gp = nullptr;          // per-channel gate of this row (g_sd > 0)
       if (row_ok && !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && it.qt < G.n_cond)) {
-        gate = __uint_as_float(static_cast<uint32_t>(a.g[a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh]) << 16);
+        gp = a.g + a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh;
+        gate = __uint_as_float(static_cast<uint32_t>(gp[0]) << 16);
+        gp = a.g_sd ? gp + 64 * hf * a.g_sd : nullptr;
         oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + it.qt) * kHeadDim + 64 * hf;
       }
       // O = O(half of step j0) + O(other half) when the item had two steps or more
@@ -607,7 +613,17 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
         if (row_ok) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] *= inv_l;
-          if (oc) {
+          if (oc && gp) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 cv = *reinterpret_cast<const float4*>(oc + ch * 32 + i);
+              const int64_t d = ch * 32 + i;
+              y[i] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + d * a.g_sd)) << 16), cv.x, y[i]);
+              y[i + 1] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + (d + 1) * a.g_sd)) << 16), cv.y, y[i + 1]);
+              y[i + 2] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + (d + 2) * a.g_sd)) << 16), cv.z, y[i + 2]);
+              y[i + 3] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + (d + 3) * a.g_sd)) << 16), cv.w, y[i + 3]);
+            }
+          } else if (oc) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               const float4 cv = *reinterpret_cast<const float4*>(oc + ch * 32 + i);
@@ -658,7 +674,7 @@ constexpr size_t kMaxAttnSmem = 227 * 1024;
 
 // Work decomposition shared by the host and the kernels (see decode_item).
 struct ItemCounts {
-  int32_t c0, nq_dense, nq_sparse, n_dense_items, n_items, max_steps;
+  int32_t c0, nq_dense, nq_sparse, n_dense_items, n_items, n_fixed, max_steps;
 };
 
 ItemCounts item_counts(const vsa_layout* L, int H, const vsa_params* p, int32_t kmax) {
@@ -669,7 +685,8 @@ ItemCounts item_counts(const vsa_layout* L, int H, const vsa_params* p, int32_t 
   c.nq_sparse = L->n_tiles - c.c0;
   c.n_dense_items = c.nq_dense * H;
   c.n_items = c.n_dense_items + c.nq_sparse * H;
-  c.max_steps = std::max(rows ? L->n_tiles : 0, L->n_cond + std::min(kmax, L->n_video));
+  c.n_fixed = p->sink == VSA_SINK_OFF ? 0 : L->n_cond;
+  c.max_steps = std::max(rows ? L->n_tiles : 0, c.n_fixed + std::min(kmax, candidates(L, p->sink).count));
   return c;
 }
 
@@ -709,7 +726,7 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* L, int32_t B, int32_
 vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H,
                                const void* q, const void* k, const void* v, int64_t sb, int64_t ss,
                                int64_t sh, const void* g, int64_t g_sb, int64_t g_ss, int64_t g_sh,
-                               const int32_t* idx, const int32_t* cnt, int32_t kmax,
+                               int64_t g_sd, const int32_t* idx, const int32_t* cnt, int32_t kmax,
                                const float* o_coarse, void* out, int32_t out_dtype, int64_t o_sb,
                                int64_t o_ss, int64_t o_sh, void* workspace, size_t workspace_bytes,
                                cudaStream_t stream) {
@@ -720,7 +737,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   if (st != VSA_OK) return st;
   if (!g || !idx || !cnt || !o_coarse || !out || !workspace) return VSA_ERR_INVALID_ARG;
   if (out_dtype != VSA_OUT_F32 && out_dtype != VSA_OUT_BF16) return VSA_ERR_INVALID_ARG;
-  if (g_sb < 0 || g_ss <= 0 || g_sh <= 0 || o_sb < 0 || o_ss <= 0 || o_sh <= 0) return VSA_ERR_INVALID_ARG;
+  if (g_sb < 0 || g_ss <= 0 || g_sh <= 0 || g_sd < 0 || o_sb < 0 || o_ss <= 0 || o_sh <= 0)
+    return VSA_ERR_INVALID_ARG;
   const int elem = out_dtype == VSA_OUT_F32 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(out) % 16 || (o_sb * elem) % 16 || (o_ss * elem) % 16 ||
       (o_sh * elem) % 16)
@@ -759,6 +777,10 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.kmax = kmax;
   const ItemCounts ic = item_counts(L, H, p, kmax);
   a.c0 = ic.c0;
+  a.n_fixed = ic.n_fixed;
+  const Candidates cand = candidates(L, p->sink);
+  a.cand0 = cand.first;
+  a.n_cand = cand.count;
   a.nq_dense = ic.nq_dense;
   a.nq_sparse = ic.nq_sparse;
   a.n_dense_items = ic.n_dense_items;
@@ -772,6 +794,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.g_sb = g_sb;
   a.g_ss = g_ss;
   a.g_sh = g_sh;
+  a.g_sd = g_sd;
   a.out = out;
   a.out_bf16 = out_dtype == VSA_OUT_BF16;
   a.o_sb = o_sb;

@@ -75,8 +75,17 @@ struct vsa_layout {
 
 namespace vsa {
 
-// k for top-k selection: max(1, ceil(keep * Nv * (1 - 2^-20))), clamped to Nv.
-int32_t topk_count(float keep, int32_t n_video);
+// k for top-k selection: max(1, ceil(keep * Nc * (1 - 2^-20))), clamped to Nc.
+int32_t topk_count(float keep, int32_t n_cand);
+
+// Candidate key tiles of a sink mode: the video tiles, or every tile with
+// VSA_SINK_OFF. Candidate ordinal c is tile id first + c.
+struct Candidates {
+  int32_t first, count;
+};
+inline Candidates candidates(const vsa_layout* L, int32_t sink) {
+  return sink == VSA_SINK_OFF ? Candidates{0, L->n_tiles} : Candidates{L->n_cond, L->n_video};
+}
 
 // Records "where: cuda error string" for vsa_last_error_detail and returns
 // VSA_ERR_CUDA; a message-only variant for failures without a cudaError_t.
@@ -95,8 +104,8 @@ vsa_status check_qkv(const void* q, const void* k, const void* v, int64_t sb, in
 struct SelectWorkspace {
   size_t pooled, scores, stats, total;
   int32_t n_row_blocks;   // 64-query-tile blocks of the coarse kernel
-  int32_t ld_scores;      // score row stride: Nv rounded up to 64
+  int32_t ld_scores;      // score row stride: Nc rounded up to 64
 };
-SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H);
+SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H, const vsa_params* p);
 
 }  // namespace vsa

@@ -36,19 +36,20 @@ vsa_status cuda_fail(const char* where) {
 
 void set_detail(const char* msg) { std::snprintf(g_detail, sizeof(g_detail), "%s", msg); }
 
-int32_t topk_count(float keep, int32_t n_video) {
-  const double prod = static_cast<double>(keep) * static_cast<double>(n_video) *
+int32_t topk_count(float keep, int32_t n_cand) {
+  const double prod = static_cast<double>(keep) * static_cast<double>(n_cand) *
                       (1.0 - 1.0 / 1048576.0);
   double k = std::ceil(prod);
   if (k < 1.0) k = 1.0;
-  if (k > n_video) k = n_video;
+  if (k > n_cand) k = n_cand;
   return static_cast<int32_t>(k);
 }
 
 vsa_status check_params(const vsa_params* p) {
   if (!p) return VSA_ERR_INVALID_ARG;
   if (p->mode != VSA_SELECT_TOPK && p->mode != VSA_SELECT_ADAPTIVE) return VSA_ERR_INVALID_ARG;
-  if (p->sink != VSA_SINK_EXACT_KV && p->sink != VSA_SINK_EXACT_KV_AND_ROWS) return VSA_ERR_INVALID_ARG;
+  if (p->sink != VSA_SINK_EXACT_KV && p->sink != VSA_SINK_EXACT_KV_AND_ROWS && p->sink != VSA_SINK_OFF)
+    return VSA_ERR_INVALID_ARG;
   if (p->mode == VSA_SELECT_TOPK && !(p->keep > 0.0f && p->keep <= 1.0f)) return VSA_ERR_INVALID_ARG;
   if (p->mode == VSA_SELECT_ADAPTIVE && !(p->tau >= 0.0f && std::isfinite(p->tau)))
     return VSA_ERR_INVALID_ARG;
@@ -73,11 +74,11 @@ vsa_status check_qkv(const void* q, const void* k, const void* v, int64_t sb, in
   return VSA_OK;
 }
 
-SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H) {
+SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H, const vsa_params* p) {
   SelectWorkspace w{};
   const size_t bh = static_cast<size_t>(B) * H;
   w.n_row_blocks = (L->n_tiles + 63) / 64;
-  w.ld_scores = (L->n_video + 63) / 64 * 64;
+  w.ld_scores = (candidates(L, p->sink).count + 63) / 64 * 64;
   size_t off = 0;
   w.pooled = off;
   off = align_up(off + 3 * bh * L->n_tiles * kHeadDim * sizeof(float), 256);
@@ -263,7 +264,8 @@ vsa_status vsa_select_kmax(const vsa_layout* L, const vsa_params* p, int32_t* km
   if (!L || !kmax) return VSA_ERR_INVALID_ARG;
   vsa_status st = check_params(p);
   if (st != VSA_OK) return st;
-  *kmax = p->mode == VSA_SELECT_TOPK ? topk_count(p->keep, L->n_video) : L->n_video;
+  const int32_t nc = candidates(L, p->sink).count;
+  *kmax = p->mode == VSA_SELECT_TOPK ? topk_count(p->keep, nc) : nc;
   return VSA_OK;
 }
 
@@ -280,7 +282,7 @@ const char* vsa_status_string(vsa_status s) {
   return "unknown status";
 }
 
-int32_t vsa_version(void) { return (1 << 16) | 0; }
+int32_t vsa_version(void) { return (1 << 16) | 1; }
 
 const char* vsa_last_error_detail(void) { return g_detail; }
 

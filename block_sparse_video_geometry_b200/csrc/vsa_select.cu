@@ -4,15 +4,16 @@
 //                       (fp32), read straight from the natural [B, S, H, 128]
 //                       layout through the tile's token list.
 // 2. coarse_kernel    : for a block of 64 query tiles of one (batch, head):
-//                       s = scale * Qbar Kbar^T against every video tile, in
-//                       fp32 FMA; the scores go to the workspace for selection
+//                       s = scale * Qbar Kbar^T against every candidate
+//                       key tile (the video tiles, or every tile with
+//                       VSA_SINK_OFF), in fp32 FMA; the scores go to the workspace for selection
 //                       and feed an online softmax against Vbar that yields
 //                       o_coarse. With the adaptive threshold it also sums s
 //                       and s^2 in fp64 per block.
 // 3. select_kernel    : one warp per query tile: radix select of the k-th
 //                       largest score (ties -> lower tile) or the adaptive
 //                       threshold mean + tau * std, emitted as an ascending
-//                       list of video tile ordinals.
+//                       list of candidate ordinals.
 // Pages: "BSAI FastH3 Native VSA (recipe)", "The mechanism, briefly" (tiles
 // are scored and only the top slice is attended exactly); "ComfyUI Agrega Nodo
 // Central de Atencion Dispersa y Compilador Comfy", "Atencion dispersa por
@@ -21,7 +22,7 @@
 // compressed branch summarises K/V by mean pooling).
 //
 // These kernels are bound by HBM (pooling reads Q, K, V once) and by fp32
-// FMA throughput (scores and the coarse softmax, ~2 * Nt * Nv * 128 FMA per
+// FMA throughput (scores and the coarse softmax, ~2 * Nt * Nc * 128 FMA per
 // head). Scores stay fp32 end to end so that the selected sets match an fp64
 // evaluation except on near-ties.
 
@@ -39,7 +40,7 @@ namespace {
 
 constexpr int kPoolMaxThreads = 1024;
 constexpr int kCoarseRows = 64;       // query tiles per coarse block
-constexpr int kCoarseCols = 64;       // video tiles per streamed chunk
+constexpr int kCoarseCols = 64;       // candidate key tiles per streamed chunk
 constexpr int kCoarseThreads = 256;
 constexpr int kSelectWarps = 4;
 
@@ -85,7 +86,7 @@ pool_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restr
 
 // ------------------------------------------------------- scores + coarse
 // grid (ceil(n_tiles / 64), H, B), 256 threads. Thread (ty, tx) = (tid / 16,
-// tid % 16) owns query rows 4*ty .. 4*ty+3; in the score block it owns video
+// tid % 16) owns query rows 4*ty .. 4*ty+3; in the score block it owns candidate
 // columns 4*tx .. 4*tx+3 of the chunk, in the coarse product dims 8*tx .. +7.
 struct CoarseSmem {
   float qT[kHeadDim][kCoarseRows];        // pooled Q, transposed
@@ -95,7 +96,7 @@ struct CoarseSmem {
 
 template <bool kStats>
 __global__ void __launch_bounds__(kCoarseThreads, 2)
-coarse_kernel(int n_tiles, int n_cond, int n_video, int H, int B, const float* __restrict__ pooled,
+coarse_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __restrict__ pooled,
               float scale, float* __restrict__ scores, int ld_scores, float* __restrict__ o_coarse,
               double* __restrict__ stats) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -105,8 +106,8 @@ coarse_kernel(int n_tiles, int n_cond, int n_video, int H, int B, const float* _
   const size_t bh = static_cast<size_t>(b) * H + h;
   const size_t plane = static_cast<size_t>(B) * H * n_tiles * kHeadDim;
   const float* qbar = pooled + bh * n_tiles * kHeadDim;
-  const float* kbar = pooled + plane + (bh * n_tiles + n_cond) * kHeadDim;
-  const float* vbar = pooled + 2 * plane + (bh * n_tiles + n_cond) * kHeadDim;
+  const float* kbar = pooled + plane + (bh * n_tiles + cand0) * kHeadDim;
+  const float* vbar = pooled + 2 * plane + (bh * n_tiles + cand0) * kHeadDim;
 
   // pooled Q rows of this block, transposed; rows past n_tiles are zero
   for (int f = tid; f < kCoarseRows * kHeadDim / 4; f += kCoarseThreads) {
@@ -129,12 +130,12 @@ coarse_kernel(int n_tiles, int n_cond, int n_video, int H, int B, const float* _
   }
   double s1 = 0.0, s2 = 0.0;
 
-  for (int c0 = 0; c0 < n_video; c0 += kCoarseCols) {
+  for (int c0 = 0; c0 < n_cand; c0 += kCoarseCols) {
     __syncthreads();  // previous chunk's Vbar / p are consumed
     for (int f = tid; f < kCoarseCols * kHeadDim / 4; f += kCoarseThreads) {
       const int c = f % kCoarseCols, d4 = f / kCoarseCols;
       float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + c < n_video) val = reinterpret_cast<const float4*>(kbar + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
+      if (c0 + c < n_cand) val = reinterpret_cast<const float4*>(kbar + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
       sm.kv[(4 * d4 + 0) * kCoarseCols + c] = val.x;
       sm.kv[(4 * d4 + 1) * kCoarseCols + c] = val.y;
       sm.kv[(4 * d4 + 2) * kCoarseCols + c] = val.z;
@@ -166,8 +167,8 @@ coarse_kernel(int n_tiles, int n_cond, int n_video, int H, int B, const float* _
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int col = c0 + 4 * tx + j;
-        s[i][j] = col < n_video ? acc[i][j] * scale : -INFINITY;
-        if (kStats && col < n_video && row < n_tiles) {
+        s[i][j] = col < n_cand ? acc[i][j] * scale : -INFINITY;
+        if (kStats && col < n_cand && row < n_tiles) {
           s1 += static_cast<double>(s[i][j]);
           s2 += static_cast<double>(s[i][j]) * static_cast<double>(s[i][j]);
         }
@@ -202,7 +203,7 @@ coarse_kernel(int n_tiles, int n_cond, int n_video, int H, int B, const float* _
     for (int f = tid; f < kCoarseCols * kHeadDim / 4; f += kCoarseThreads) {
       const int c = f / (kHeadDim / 4), d4 = f % (kHeadDim / 4);
       float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + c < n_video) val = reinterpret_cast<const float4*>(vbar + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
+      if (c0 + c < n_cand) val = reinterpret_cast<const float4*>(vbar + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
       reinterpret_cast<float4*>(sm.kv)[f] = val;
     }
     __syncthreads();
@@ -270,7 +271,7 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 
 // grid (ceil(n_tiles / rows_per_block), H, B), rows_per_block warps.
 template <bool kAdaptive>
-__global__ void select_kernel(int n_tiles, int n_video, int H, const float* __restrict__ scores,
+__global__ void select_kernel(int n_tiles, int n_cand, int H, const float* __restrict__ scores,
                               int ld_scores, int k, float tau, const double* __restrict__ stats,
                               int n_row_blocks, int32_t* __restrict__ idx, int kmax,
                               int32_t* __restrict__ cnt) {
@@ -285,7 +286,7 @@ __global__ void select_kernel(int n_tiles, int n_video, int H, const float* __re
   const int h = blockIdx.y, b = blockIdx.z;
   const size_t bh = static_cast<size_t>(b) * H + h;
   const float* src = scores + (bh * n_tiles + qt) * ld_scores;
-  for (int i = lane; i < n_video; i += 32) row[i] = src[i];
+  for (int i = lane; i < n_cand; i += 32) row[i] = src[i];
   __syncwarp();
   int32_t* out = idx + (bh * n_tiles + qt) * kmax;
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -297,7 +298,7 @@ __global__ void select_kernel(int n_tiles, int n_video, int H, const float* __re
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = lane; i < 256; i += 32) hist[i] = 0;
       __syncwarp();
-      for (int i = lane; i < n_video; i += 32) {
+      for (int i = lane; i < n_cand; i += 32) {
         const uint32_t key = ordered_key(row[i]);
         if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
@@ -339,13 +340,13 @@ __global__ void select_kernel(int n_tiles, int n_video, int H, const float* __re
     }
     // prefix is the k-th largest key; krem of its equals are taken, lowest ordinals first
     int pos = 0, eq_seen = 0;
-    for (int base = 0; base < n_video; base += 32) {
+    for (int base = 0; base < n_cand; base += 32) {
       const int i = base + lane;
-      const uint32_t key = i < n_video ? ordered_key(row[i]) : 0u;
-      const bool eq = i < n_video && key == prefix;
+      const uint32_t key = i < n_cand ? ordered_key(row[i]) : 0u;
+      const bool eq = i < n_cand && key == prefix;
       const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
       const int eq_rank = eq_seen + __popc(eqb & lt_mask);
-      const bool sel = i < n_video && (key > prefix || (eq && eq_rank < krem));
+      const bool sel = i < n_cand && (key > prefix || (eq && eq_rank < krem));
       const uint32_t selb = __ballot_sync(0xffffffffu, sel);
       if (sel) out[pos + __popc(selb & lt_mask)] = i;
       pos += __popc(selb);
@@ -364,14 +365,14 @@ __global__ void select_kernel(int n_tiles, int n_video, int H, const float* __re
       a += __shfl_xor_sync(0xffffffffu, a, off);
       c += __shfl_xor_sync(0xffffffffu, c, off);
     }
-    const double nn = static_cast<double>(n_tiles) * static_cast<double>(n_video);
+    const double nn = static_cast<double>(n_tiles) * static_cast<double>(n_cand);
     const double mean = a / nn;
     const double var = fmax(c / nn - mean * mean, 0.0);
     const double thr = mean + static_cast<double>(tau) * sqrt(var);
     int pos = 0;
-    for (int base = 0; base < n_video; base += 32) {
+    for (int base = 0; base < n_cand; base += 32) {
       const int i = base + lane;
-      const bool sel = i < n_video && static_cast<double>(row[i]) >= thr;
+      const bool sel = i < n_cand && static_cast<double>(row[i]) >= thr;
       const uint32_t selb = __ballot_sync(0xffffffffu, sel);
       if (sel) out[pos + __popc(selb & lt_mask)] = i;
       pos += __popc(selb);
@@ -379,7 +380,7 @@ __global__ void select_kernel(int n_tiles, int n_video, int H, const float* __re
     if (pos == 0) {  // keep the argmax (lowest ordinal among equal maxima)
       float best = -INFINITY;
       int bi = 0x7fffffff;
-      for (int i = lane; i < n_video; i += 32) {
+      for (int i = lane; i < n_cand; i += 32) {
         if (row[i] > best) {
           best = row[i];
           bi = i;
@@ -414,7 +415,7 @@ vsa_status vsa_coarse_select_workspace_size(const vsa_layout* L, int32_t B, int3
   if (!L || !bytes || B <= 0 || H <= 0) return VSA_ERR_INVALID_ARG;
   vsa_status st = check_params(p);
   if (st != VSA_OK) return st;
-  *bytes = select_workspace(L, B, H).total;
+  *bytes = select_workspace(L, B, H, p).total;
   return VSA_OK;
 }
 
@@ -431,13 +432,14 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
   if (reinterpret_cast<uintptr_t>(o_coarse) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
     return VSA_ERR_INVALID_ARG;
   if (!L->dev_buf) return VSA_ERR_NOT_UPLOADED;
-  const SelectWorkspace ws = select_workspace(L, B, H);
+  const SelectWorkspace ws = select_workspace(L, B, H, p);
+  const Candidates cand = candidates(L, p->sink);
   if (workspace_bytes < ws.total) return VSA_ERR_WORKSPACE_TOO_SMALL;
 
   const int ld = ws.ld_scores;
   const size_t row_bytes = static_cast<size_t>(ld) * sizeof(float);
   const int rows_per_block = static_cast<int>(std::min<size_t>(kSelectWarps, (200u << 10) / row_bytes));
-  if (rows_per_block < 1) return VSA_ERR_UNSUPPORTED;   // more than 51200 video tiles
+  if (rows_per_block < 1) return VSA_ERR_UNSUPPORTED;   // more than 51200 candidate tiles
 
   char* w = static_cast<char*>(workspace);
   float* pooled = reinterpret_cast<float*>(w + ws.pooled);
@@ -460,14 +462,14 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
                                        static_cast<int>(coarse_smem));
   if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: cudaFuncSetAttribute(coarse)", e);
   ck<<<dim3(ws.n_row_blocks, H, B), kCoarseThreads, coarse_smem, stream>>>(
-      L->n_tiles, L->n_cond, L->n_video, H, B, pooled, scale, scores, ld, o_coarse, stats);
+      L->n_tiles, cand.first, cand.count, H, B, pooled, scale, scores, ld, o_coarse, stats);
 
   const size_t sel_smem = rows_per_block * row_bytes + rows_per_block * 256 * sizeof(uint32_t);
   auto sk = adaptive ? select_kernel<true> : select_kernel<false>;
   e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sel_smem));
   if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: cudaFuncSetAttribute(select)", e);
   sk<<<dim3((L->n_tiles + rows_per_block - 1) / rows_per_block, H, B), 32 * rows_per_block, sel_smem,
-       stream>>>(L->n_tiles, L->n_video, H, scores, ld, kmax, p->tau, stats, ws.n_row_blocks, idx,
+       stream>>>(L->n_tiles, cand.count, H, scores, ld, kmax, p->tau, stats, ws.n_row_blocks, idx,
                  kmax, cnt);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: launch", e);
@@ -512,7 +514,7 @@ extern "C" vsa_status vsa_coarse_select_noalloc(const vsa_layout* L, const vsa_p
   if (!L || B <= 0 || H <= 0) return VSA_ERR_INVALID_ARG;
   vsa_status st = check_params(p);
   if (st != VSA_OK) return st;
-  const size_t need = select_workspace(L, B, H).total;
+  const size_t need = select_workspace(L, B, H, p).total;
   if (need > kNoAllocScratchBytes) {
     char msg[160];
     std::snprintf(msg, sizeof(msg),

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libvsa.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, ERR_TIMEOUT, ERR_NOT_UPLOADED = range(7)
 SEG_TEXT, SEG_REF_IMAGE, SEG_REF_AUDIO, SEG_OTHER_COND, SEG_VIDEO = range(5)
 SELECT_TOPK, SELECT_ADAPTIVE = 0, 1
-SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS = 0, 1
+SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS, SINK_OFF = 0, 1, 2
 OUT_F32, OUT_BF16 = 0, 1
 TILE, HEAD_DIM = 64, 128
 
@@ -68,8 +68,8 @@ _SIGNATURES = {
                                          _P, _P, _P, _P]),
     "vsa_sparse_attn_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
     "vsa_sparse_attn_fwd": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
-                                   _P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64, _I64,
-                                   _P, _SZ, _P]),
+                                   _P, _I64, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64,
+                                   _I64, _P, _SZ, _P]),
     "vsa_sparse_attn_status": (_I32, [_P, _P]),
     "vsa_debug_inject_wait_timeout": (_I32, [ctypes.c_uint64]),
     "vsa_status_string": (ctypes.c_char_p, [_I32]),
@@ -215,9 +215,16 @@ def coarse_select_noalloc(layout: Layout, params: Params, q, k, v, idx, cnt, o_c
 
 def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: int, o_coarse, out,
                     workspace, stream=None) -> None:
-    """vsa_sparse_attn_fwd on torch tensors; out is float32 or bfloat16 [B, S, H, 128]."""
+    """vsa_sparse_attn_fwd on torch tensors; out is float32 or bfloat16 [B, S, H, 128];
+    g is bf16 [B, S, H] (one gate per token and head) or [B, S, H, 128] (one per channel)."""
     import torch
     B, S, H, _ = q.shape
+    if g.dim() == 3:
+        g_sd = 0
+    elif g.dim() == 4 and g.shape[3] == HEAD_DIM:
+        g_sd = g.stride(3)
+    else:
+        raise ValueError("g must be [B, S, H] or [B, S, H, 128]")
     sb, ss, sh = _qkv_strides(q, k, v)
     if out.dtype == torch.float32:
         od = OUT_F32
@@ -227,7 +234,7 @@ def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: 
         raise ValueError("out must be float32 or bfloat16")
     _check(lib().vsa_sparse_attn_fwd(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
                                      v.data_ptr(), sb, ss, sh, g.data_ptr(), g.stride(0), g.stride(1),
-                                     g.stride(2), idx.data_ptr(), cnt.data_ptr(), kmax, o_coarse.data_ptr(),
+                                     g.stride(2), g_sd, idx.data_ptr(), cnt.data_ptr(), kmax, o_coarse.data_ptr(),
                                      out.data_ptr(), od, out.stride(0), out.stride(1), out.stride(2),
                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                      _stream_handle(stream)), "vsa_sparse_attn_fwd")

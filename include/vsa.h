@@ -83,16 +83,23 @@ typedef enum { VSA_SELECT_TOPK = 0, VSA_SELECT_ADAPTIVE = 1 } vsa_select_mode;
 /* sink_conditioning ("BSAI FastH3 Native VSA (recipe)", "The inputs that
  * matter"): EXACT_KV = every query attends every conditioning key exactly;
  * EXACT_KV_AND_ROWS = in addition, conditioning query rows attend the whole
- * sequence densely (and get no coarse term). */
-typedef enum { VSA_SINK_EXACT_KV = 0, VSA_SINK_EXACT_KV_AND_ROWS = 1 } vsa_sink_mode;
+ * sequence densely (and get no coarse term); OFF = nothing is protected (the
+ * pages' cheapest mode; reading): every tile, conditioning or video, is a
+ * candidate key tile, scored, selected and summarised like a video tile, and
+ * a query attends exactly only the tokens of its selected tiles.
+ * Candidate key tiles: the video tiles (ordinal c = tile id - n_cond_tiles)
+ * under EXACT_KV and EXACT_KV_AND_ROWS, every tile (ordinal c = tile id) under
+ * OFF; Nc below is their number. */
+typedef enum { VSA_SINK_EXACT_KV = 0, VSA_SINK_EXACT_KV_AND_ROWS = 1, VSA_SINK_OFF = 2 } vsa_sink_mode;
 
 typedef enum { VSA_OUT_F32 = 0, VSA_OUT_BF16 = 1 } vsa_out_dtype;
 
 /* Selection parameters.
- *  mode  : VSA_SELECT_TOPK keeps k = max(1, ceil(keep * Nv)) video key tiles
- *          per query tile (Nv = number of video tiles; the product is taken in
- *          double with a relative guard of 2^-20); ties go to the lower tile.
- *          VSA_SELECT_ADAPTIVE keeps the video key tiles whose score is
+ *  mode  : VSA_SELECT_TOPK keeps k = max(1, ceil(keep * Nc)) candidate key
+ *          tiles per query tile (Nc = number of candidate tiles, see
+ *          vsa_sink_mode; the product is taken in double with a relative guard
+ *          of 2^-20); ties go to the lower tile.
+ *          VSA_SELECT_ADAPTIVE keeps the candidate key tiles whose score is
  *          >= mean + tau * std of that (batch, head)'s whole score matrix
  *          (population std), and at least the row's argmax.
  *  keep  : (0, 1], used by TOPK.
@@ -243,13 +250,19 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* layout, int32_t B, i
 
 /* vsa_sparse_attn_fwd: exact attention of every query tile over all
  * conditioning key tokens plus the video tiles of its list (EXACT_KV), or over
- * the whole sequence for conditioning query tiles (EXACT_KV_AND_ROWS), then
- * out = o_fine + g * o_coarse[tile] (no coarse term on dense conditioning rows).
+ * the whole sequence for conditioning query tiles (EXACT_KV_AND_ROWS), or over
+ * the tiles of its list only (OFF), then out = o_fine + g * o_coarse[tile] (no
+ * coarse term on dense conditioning rows).
  * ("BSAI FastH3 Native VSA (recipe)", "The inputs that matter",
  * sink_conditioning; "ComfyUI-Ref2VA-VSA", "Video-Only Sparse Attention".)
  *
  *  q, k, v, strides : as for vsa_coarse_select.
- *  g                : bf16 [B, S, H] gate at element strides (g_stride_*).
+ *  g                : bf16 gate at element strides g_stride_b, _s, _h, _d:
+ *                     [B, S, H] with g_stride_d = 0 (one gate per token and
+ *                     head, broadcast over head_dim), or [B, S, H, 128] with
+ *                     g_stride_d > 0 (one gate per channel, the output of a
+ *                     to_gate_compress projection: "ComfyUI-Ref2VA-VSA",
+ *                     "Technical Architecture").
  *  idx, cnt, kmax   : lists from vsa_coarse_select (same params).
  *  o_coarse         : float [B, H, n_tiles, 128] from vsa_coarse_select.
  *  out              : [B, S, H, 128] of out_dtype (vsa_out_dtype) at element
@@ -269,7 +282,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* layout, const vsa_params* param
                                const void* q, const void* k, const void* v,
                                int64_t stride_b, int64_t stride_s, int64_t stride_h,
                                const void* g, int64_t g_stride_b, int64_t g_stride_s,
-                               int64_t g_stride_h,
+                               int64_t g_stride_h, int64_t g_stride_d,
                                const int32_t* idx, const int32_t* cnt, int32_t kmax,
                                const float* o_coarse,
                                void* out, int32_t out_dtype, int64_t out_stride_b,

@@ -76,6 +76,22 @@ def test_layout_matches_oracle_bit_exact(cond, grid, after):
     assert lay.info.device_bytes >= perm.nbytes + inv.nbytes
 
 
+def test_sink_off_candidates_are_all_tiles():
+    segs, S = _segments(((0, 32), (1, 16), (2, 16)), (8, 8, 8))
+    lay = vsa.Layout(segs, S)
+    ref = O.build_layout([O.Segment(k, s, n, g) for (k, s, n, g) in segs], S)
+    nt = lay.info.n_tiles
+    for keep in (0.25, 0.5, 0.1, 1.0):
+        assert lay.kmax(vsa.make_params(keep=keep, sink=vsa.SINK_OFF)) == O.topk_count(keep, nt)
+        assert lay.kmax(vsa.make_params(keep=keep, sink=vsa.SINK_OFF)) == \
+            O.topk_count(keep, O.candidate_tiles(ref, O.SINK_OFF)[1])
+    assert lay.kmax(vsa.make_params(mode=vsa.SELECT_ADAPTIVE, sink=vsa.SINK_OFF)) == nt
+    # the score matrix spans every tile: the selection workspace grows accordingly
+    on = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5))
+    off = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5, sink=vsa.SINK_OFF))
+    assert off >= on
+
+
 def test_topk_count_matches_oracle():
     segs, S = _segments(((0, 64),), (8, 8, 8))
     rng = np.random.default_rng(0)
@@ -114,7 +130,7 @@ def test_calls_validate_before_any_gpu_work():
     good = vsa.make_params(keep=0.5)
     n = ctypes.c_size_t()
     for bad in [vsa.make_params(keep=0.0), vsa.make_params(keep=1.5), vsa.make_params(mode=3),
-                vsa.make_params(sink=5), vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=-1.0),
+                vsa.make_params(sink=5), vsa.make_params(sink=3), vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=-1.0),
                 vsa.make_params(scale=float("nan"))]:
         assert L.vsa_coarse_select_workspace_size(lay.handle, 1, 2, ctypes.byref(bad), ctypes.byref(n)) == \
             vsa.ERR_INVALID_ARG
@@ -137,12 +153,15 @@ def test_calls_validate_before_any_gpu_work():
                                args["sh"], fake, fake, fake, fake, n.value, None) == vsa.ERR_INVALID_ARG
     kmax = lay.kmax(good)
     common = (lay.handle, ctypes.byref(good), 1, 2, fake, fake, fake, args["sb"], args["ss"], args["sh"],
-              fake, 2, 2 * S, 2)
+              fake, 2, 2 * S, 2, 0)
     # wrong kmax, bad out dtype, unaligned out stride, not uploaded
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, 7, S * 256, 256, 128, fake, 256,
                                  None) == vsa.ERR_INVALID_ARG
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_BF16, S * 256, 256, 129, fake,
                                  256, None) == vsa.ERR_INVALID_ARG
+    # negative channel stride of the gate
+    assert L.vsa_sparse_attn_fwd(*common[:-1], -1, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128,
+                                 fake, 1 << 30, None) == vsa.ERR_INVALID_ARG
     ws = lay.sparse_attn_workspace_size(1, 2, good)
     assert ws >= 256 + 2 * lay.info.n_tiles * 32768          # error word + tile-major K/V
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,

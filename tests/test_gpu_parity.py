@@ -47,13 +47,13 @@ def test_tcgen05_building_blocks(cuda_ok):
 
 
 # --------------------------------------------------------- full checks ----
-def full_check(wl, out_dtype="f32", heads=None, out_tiles=None, **prm_over):
+def full_check(wl, out_dtype="f32", heads=None, out_tiles=None, channel_gate=False, **prm_over):
     lay = C.oracle_layout(wl)
-    bits = C.inputs(wl, lay)
+    bits = C.inputs(wl, lay, channel_gate)
     prm = C.params_of(wl, **prm_over)
     res = C.gpu_forward(wl, bits, prm, out_dtype)
     assert res["status"] == vsa.OK
-    C.check_lists_valid(res, lay)
+    C.check_lists_valid(res, lay, prm["sink"])
     worst = 0.0
     for b in range(wl.B):
         for h in (range(wl.H) if heads is None else heads):
@@ -78,7 +78,7 @@ def test_tiny_bf16_output(cuda_ok):
     full_check(W.WORKLOADS["tiny"], out_dtype="bf16")
 
 
-@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS])
+@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS, O.SINK_OFF])
 @pytest.mark.parametrize("keep", [0.125, 0.5, 1.0])
 def test_tiny_keep_and_sink(cuda_ok, keep, sink):
     full_check(W.WORKLOADS["tiny"], keep=keep, sink=sink)
@@ -106,9 +106,27 @@ EDGE_WORKLOADS = [
 
 
 @pytest.mark.parametrize("wl", EDGE_WORKLOADS, ids=lambda w: w.name)
-@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS])
+@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS, O.SINK_OFF])
 def test_edge_layouts(cuda_ok, wl, sink):
     full_check(wl, sink=sink)
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.5])
+def test_tiny_adaptive_sink_off(cuda_ok, tau):
+    full_check(W.WORKLOADS["tiny"].with_(mode=O.MODE_ADAPTIVE, tau=tau), sink=O.SINK_OFF)
+
+
+@pytest.mark.parametrize("wl", [W.WORKLOADS["tiny"], EDGE_WORKLOADS[0]], ids=lambda w: w.name)
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_channel_gate(cuda_ok, wl, out_dtype):
+    """g [B, S, H, 128]: one gate per channel."""
+    full_check(wl, out_dtype=out_dtype, channel_gate=True)
+
+
+def test_mid_sink_off_two_heads(cuda_ok):
+    wl = W.WORKLOADS["mid"].with_(H=4)
+    full_check(wl, heads=(0, 3), out_tiles=lambda lay: range(0, lay.n_tiles, 9), sink=O.SINK_OFF,
+               channel_gate=True)
 
 
 def test_k_equals_one(cuda_ok):

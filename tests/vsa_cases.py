@@ -28,8 +28,14 @@ def oracle_layout(wl):
     return O.build_layout([O.Segment(k, s, n, g) for (k, s, n, g) in wl.segments()], wl.seq_len)
 
 
-def inputs(wl, lay):
-    return W.make_inputs(wl, lay.inv // O.TILE)
+def inputs(wl, lay, channel_gate=False):
+    """Seeded (q, k, v, g) bf16 bits; with channel_gate, g is [B, S, H, 128]
+    (seeded U(0, 1) per channel) instead of [B, S, H]."""
+    q, k, v, g = W.make_inputs(wl, lay.inv // O.TILE)
+    if channel_gate:
+        rng = np.random.default_rng(1000 + wl.seed)
+        g = W.f32_to_bf16_bits(rng.uniform(0.0, 1.0, (wl.B, wl.seq_len, wl.H, wl.D)).astype(np.float32))
+    return q, k, v, g
 
 
 def params_of(wl, **kw):
@@ -79,10 +85,10 @@ class HeadOracle:
                                       self.sel[qt], self.o_coarse, self.scale)
 
 
-def check_lists_valid(res, lay):
-    """Every list is ascending, in range and as long as cnt says."""
+def check_lists_valid(res, lay, sink=O.SINK_EXACT_KV):
+    """Every list is ascending, in range (candidate ordinals) and as long as cnt says."""
     idx, cnt = res["idx"], res["cnt"]
-    nv = lay.n_video_tiles
+    nv = O.candidate_tiles(lay, sink)[1]
     assert cnt.min() >= 1 and cnt.max() <= res["kmax"]
     B, H, Nt, _ = idx.shape
     for b in range(B):
