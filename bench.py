@@ -36,17 +36,20 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ms per VSA attention call and effective TFLOP/s (% bf16 peak) at 129k tokens"
 WORKLOAD = "5s"
+SINKS = {"exact_kv": 0, "exact_kv_and_rows": 1, "off": 2}
 
 
-def valid_flop_fast(counts, n_cond, idx, cnt, sink_rows):
+def valid_flop_fast(counts, n_cond, idx, cnt, sink_rows, sink_off=False):
     """Valid fine-branch FLOP of one call: 4 * 128 per attended (valid query,
     valid key) pair; keys of a query tile = conditioning tokens + tokens of its
-    selected video tiles (all tokens for dense conditioning rows)."""
+    selected video tiles (all tokens for dense conditioning rows; with the sink
+    off, the tokens of its selected tiles only, any tile being a candidate)."""
     counts = counts.astype(np.float64)
-    vid = counts[n_cond:]
+    cand = counts if sink_off else counts[n_cond:]
+    fixed = 0.0 if sink_off else counts[:n_cond].sum()
     B, H, Nt, kmax = idx.shape
     mask = np.arange(kmax)[None, None, None, :] < cnt[..., None]
-    keys = np.where(mask, vid[np.clip(idx, 0, len(vid) - 1)], 0.0).sum(-1) + counts[:n_cond].sum()
+    keys = np.where(mask, cand[np.clip(idx, 0, len(cand) - 1)], 0.0).sum(-1) + fixed
     if sink_rows:
         keys[:, :, :n_cond] = counts.sum()
     return 4.0 * 128.0 * float((keys * counts[None, None, :]).sum())
@@ -110,7 +113,7 @@ def describe(wl) -> str:
     names = {0: "text", 1: "ref image", 2: "ref audio", 3: "other"}
     cond = " + ".join("%d %s" % (n, names.get(k, "cond")) for k, n in wl.cond)
     sel = ("keep %g%%" % (100 * wl.keep)) if wl.mode == 0 else ("adaptive tau %g" % wl.tau)
-    sink = "exact_kv" if wl.sink == 0 else "exact_kv_and_rows"
+    sink = {0: "exact_kv", 1: "exact_kv_and_rows", 2: "sink off"}[wl.sink]
     return "%s: %s conditioning + %dx%dx%d video tokens (S=%d), B=%d, H=%d, d=%d, %s, %s" % (
         wl.name, cond or "no", *wl.grid, wl.seq_len, wl.B, wl.H, wl.D, sel, sink)
 
@@ -167,6 +170,8 @@ def run_reference(args):
     from block_sparse_video_geometry_b200 import workloads as W
     from oracle import vsa_oracle as O
     wl = W.WORKLOADS[args.workload]
+    if args.sink is not None:
+        wl = wl.with_(sink=SINKS[args.sink])
     lay = O.build_layout([O.Segment(k, s, n, gr) for (k, s, n, gr) in wl.segments()], wl.seq_len)
     bits = W.make_inputs(wl, lay.inv // O.TILE)
     n_tiles = args.ref_tiles
@@ -213,6 +218,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     wl = W.WORKLOADS[args.workload].with_(seed=W.WORKLOADS[args.workload].seed + rank)
+    if args.sink is not None:
+        wl = wl.with_(sink=SINKS[args.sink])
     lay = vsa.Layout(wl.segments(), wl.seq_len)
     perm, inv, counts, kinds = lay.tables()
     bits = W.make_inputs(wl, inv // vsa.TILE)
@@ -237,7 +244,7 @@ def run_ours(args):
     if st != vsa.OK:
         raise RuntimeError("kernel status %s" % vsa.status_string(st))
     flop = valid_flop_fast(counts, lay.info.n_cond_tiles, fwd.idx.cpu().numpy(), fwd.cnt.cpu().numpy(),
-                           wl.sink == vsa.SINK_EXACT_KV_AND_ROWS)
+                           wl.sink == vsa.SINK_EXACT_KV_AND_ROWS, wl.sink == vsa.SINK_OFF)
 
     def barrier():
         torch.cuda.synchronize()
@@ -405,6 +412,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32")
+    ap.add_argument("--sink", choices=sorted(SINKS), default=None,
+                    help="override the workload's sink_conditioning mode")
     ap.add_argument("--ref-tiles", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the torch SDPA comparator")
