@@ -56,6 +56,7 @@ SEG_TEXT, SEG_REF_IMAGE, SEG_REF_AUDIO, SEG_OTHER_COND, SEG_VIDEO = 0, 1, 2, 3, 
 
 MODE_TOPK, MODE_ADAPTIVE = 0, 1
 SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS, SINK_OFF = 0, 1, 2
+COARSE_MEAN, COARSE_REWEIGHT = 0, 1
 
 
 # --------------------------------------------------------------------------- #
@@ -309,6 +310,60 @@ def coarse_branch(scores: np.ndarray, vbar: np.ndarray, layout: Layout,
     return p @ vv
 
 
+def video_query_anchor(q: np.ndarray, layout: Layout) -> np.ndarray:
+    """Mean query of every valid video token of one (batch, head): the per-head
+    anchor of Spark-Reweight ("Spark-H3: atencion dispersa por bloques ...",
+    "Que cambia Spark-Attn": the scoring uses the mean of the video queries as
+    a per-head anchor, which keeps the extra cost linear)."""
+    toks = np.concatenate([layout.tile_tokens(t) for t in range(layout.n_cond_tiles, layout.n_tiles)])
+    return np.asarray(q, dtype=np.float64)[toks].mean(axis=0)
+
+
+def reweighted_summaries(k: np.ndarray, v: np.ndarray, anchor: np.ndarray, layout: Layout,
+                         scale: float, sink: int = SINK_EXACT_KV):
+    """Spark-Reweight summaries of the candidate key tiles (same section).
+
+    Mean pooling scores a tile with exp(E[x]) where attention weighs it with
+    E[exp(x)]; Spark-Reweight uses weighted summaries plus a log-mass bias.
+    Reading, per candidate tile t with valid tokens i and anchor logits
+    x_i = scale * <anchor, k_i>:
+      weights  w_i = exp(x_i) / sum_j exp(x_j)          (the anchor's softmax inside t)
+      K~_t = sum_i w_i k_i,  V~_t = sum_i w_i v_i
+      b_t  = log(mean_i exp(x_i)) - scale * <anchor, K~_t>
+    so that the anchor's effective pooled logit scale * <anchor, K~_t> + b_t has
+    an exponential equal to the tile's expected exponential mean_i exp(x_i).
+    Returns (K~ [n_cand, D], V~ [n_cand, D], b [n_cand]).
+    """
+    first, count = candidate_tiles(layout, sink)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    D = k.shape[1]
+    kt, vt, b = np.empty((count, D)), np.empty((count, D)), np.empty(count)
+    for c in range(count):
+        toks = layout.tile_tokens(first + c)
+        x = scale * (k[toks] @ anchor)
+        m = x.max()
+        e = np.exp(x - m)
+        w = e / e.sum()
+        kt[c] = w @ k[toks]
+        vt[c] = w @ v[toks]
+        b[c] = m + math.log(e.mean()) - scale * float(anchor @ kt[c])
+    return kt, vt, b
+
+
+def coarse_branch_reweighted(qbar: np.ndarray, kt: np.ndarray, vt: np.ndarray, bias: np.ndarray,
+                             scale: float) -> np.ndarray:
+    """Compressed branch with Spark-Reweight summaries:
+    o_coarse[qt] = sum_c softmax_c(scale * <qbar[qt], K~_c> + b_c) V~_c.
+    Reading: the query side stays the pooled query of the tile, and only the
+    compressed branch changes; the selection keeps the mean-pooled scores."""
+    s = scale * (qbar @ kt.T) + bias[None, :]
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ vt
+
+
 # --------------------------------------------------------------------------- #
 # 3/4. Fine branch
 # --------------------------------------------------------------------------- #
@@ -358,6 +413,7 @@ class Params:
     tau: float = 1.0
     sink: int = SINK_EXACT_KV
     scale: float = 0.0        # 0 -> 1/sqrt(D)
+    coarse: int = COARSE_MEAN
 
 
 @dataclass
@@ -383,7 +439,12 @@ def selection_for_head(q, k, v, layout: Layout, params: Params):
         thr = None
     else:
         sel, thr = select_adaptive(scores, params.tau)
-    o_coarse = coarse_branch(scores, vbar, layout, params.sink)
+    if params.coarse == COARSE_REWEIGHT:
+        anchor = video_query_anchor(q, layout)
+        kt, vt, bias = reweighted_summaries(k, v, anchor, layout, scale, params.sink)
+        o_coarse = coarse_branch_reweighted(qbar, kt, vt, bias, scale)
+    else:
+        o_coarse = coarse_branch(scores, vbar, layout, params.sink)
     return qbar, kbar, vbar, scores, sel, thr, o_coarse, scale
 
 

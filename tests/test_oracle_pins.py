@@ -392,6 +392,76 @@ def test_channel_gate():
     assert np.allclose(d[:, 37], 2.0 * r1.o_coarse[tile][:, 37], atol=1e-14)
 
 
+# ------------------------------------------------------- Spark-Reweight --
+def test_reweight_anchor_query_is_exact_attention_over_full_tiles():
+    """With every candidate tile full, the anchor's reweighted compressed
+    branch equals exact token-level softmax attention of the anchor over all
+    candidate keys (the bias restores each tile's mass, the weights its
+    within-tile distribution); checked against textbook attention."""
+    wl, lay, q, k, v, g = _tiny_case(cond=((W.SEG_TEXT, 64), (W.SEG_REF_IMAGE, 128)))
+    assert all(len(lay.tile_tokens(t)) == 64 for t in range(lay.n_tiles))
+    scale = O.default_scale()
+    a = O.video_query_anchor(q, lay)
+    vid = np.concatenate([lay.tile_tokens(t) for t in range(lay.n_cond_tiles, lay.n_tiles)])
+    assert np.allclose(a, q[vid].mean(0), atol=1e-15)
+    for sink, keys in ((O.SINK_EXACT_KV, vid), (O.SINK_OFF, np.arange(lay.seq_len))):
+        kt, vt, b = O.reweighted_summaries(k, v, a, lay, scale, sink)
+        oc = O.coarse_branch_reweighted(a[None], kt, vt, b, scale)
+        ref = O.softmax_attention(a[None], k[keys], v[keys], scale)
+        assert np.allclose(oc, ref, atol=1e-12)
+
+
+def test_reweight_two_token_closed_form():
+    """Hand-worked tile: anchor logits 0 and ln 3 -> weights 1/4, 3/4 and an
+    effective pooled logit ln((1 + 3) / 2) = ln 2."""
+    segs = [O.Segment(O.SEG_VIDEO, 0, 2, (1, 1, 2))]
+    lay = O.build_layout(segs, 2)
+    a = np.zeros(128)
+    a[0] = 1.0
+    k = np.zeros((2, 128))
+    k[1, 0] = math.log(3.0)                 # scale 1: x = (0, ln 3)
+    v = np.zeros((2, 128))
+    v[0, 5], v[1, 5] = 8.0, 4.0
+    kt, vt, b = O.reweighted_summaries(k, v, a, lay, 1.0)
+    assert np.isclose(kt[0, 0], 0.75 * math.log(3.0), atol=1e-15)
+    assert np.isclose(vt[0, 5], 0.25 * 8.0 + 0.75 * 4.0, atol=1e-15)
+    assert np.isclose(float(a @ kt[0]) + b[0], math.log(2.0), atol=1e-15)
+
+
+def test_reweight_tile_constant_equals_mean_pooling():
+    """Tokens of a tile all equal: the weights are uniform, the bias zero, and
+    the reweighted branch is the mean-pooled one."""
+    wl = W.WORKLOADS["tiny"]
+    lay = layout_of(wl)
+    rng = np.random.default_rng(21)
+    qc, kc, vc = (rng.standard_normal((lay.n_tiles, 128)) for _ in range(3))
+    tile = lay.inv // O.TILE
+    q, k, v = qc[tile] + 0.3 * rng.standard_normal((lay.seq_len, 128)), kc[tile], vc[tile]
+    scale = O.default_scale()
+    p_mean = O.Params(keep=0.5)
+    p_rw = O.Params(keep=0.5, coarse=O.COARSE_REWEIGHT)
+    r0 = O.selection_for_head(q, k, v, lay, p_mean)
+    r1 = O.selection_for_head(q, k, v, lay, p_rw)
+    assert np.allclose(r0[6], r1[6], atol=1e-12)          # o_coarse
+    for x, y in zip(r0[4], r1[4]):                        # the selection is unchanged
+        assert np.array_equal(x, y)
+    kt, vt, b = O.reweighted_summaries(k, v, O.video_query_anchor(q, lay), lay, scale)
+    assert np.allclose(b, 0.0, atol=1e-12)
+
+
+def test_reweight_changes_only_the_compressed_branch():
+    wl, lay, q, k, v, g = _tiny_case()
+    r0 = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.5))
+    r1 = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.5, coarse=O.COARSE_REWEIGHT))
+    assert np.array_equal(r0.o_fine, r1.o_fine)
+    assert not np.allclose(r0.o_coarse, r1.o_coarse, atol=1e-6)
+    w = O.reweighted_summaries(k, v, O.video_query_anchor(q, lay), lay, O.default_scale())[1]
+    vid_v = v[np.concatenate([lay.tile_tokens(t) for t in range(lay.n_cond_tiles, lay.n_tiles)])]
+    # convex combinations of the candidate values
+    assert np.all(r1.o_coarse <= vid_v.max(0) + 1e-12) and np.all(r1.o_coarse >= vid_v.min(0) - 1e-12)
+    assert np.all(w <= vid_v.max(0) + 1e-12) and np.all(w >= vid_v.min(0) - 1e-12)
+
+
 # ------------------------------------------------------------- generator --
 def test_generator_is_seeded_and_bf16_rounded():
     import torch
