@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 METRIC = "ms per VSA attention call and effective TFLOP/s (% bf16 peak) at 129k tokens"
 WORKLOAD = "5s"
 SINKS = {"exact_kv": 0, "exact_kv_and_rows": 1, "off": 2}
+COARSES = {"mean": 0, "reweight": 1}
 
 
 def valid_flop_fast(counts, n_cond, idx, cnt, sink_rows, sink_off=False):
@@ -128,7 +129,7 @@ def measured_peaks():
 
 
 # --------------------------------------------------------------- CPU oracle
-def oracle_sample(wl, bits, lay, head, n_tiles, rng_seed=0):
+def oracle_sample(wl, bits, lay, head, n_tiles, rng_seed=0, coarse=0):
     """Times the oracle on one head: its whole selection and the fine branch of
     n_tiles query tiles. Returns (seconds, valid FLOP of the sampled fine work,
     seconds extrapolated to one whole call)."""
@@ -137,7 +138,7 @@ def oracle_sample(wl, bits, lay, head, n_tiles, rng_seed=0):
     q, k, v, g = bits
     t0 = time.perf_counter()
     qh, kh, vh, gh = f(q[0, :, head]), f(k[0, :, head]), f(v[0, :, head]), f(g[0, :, head])
-    p = O.Params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink)
+    p = O.Params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=coarse)
     qb, kb, vb, sc, sel, thr, oc, scale = O.selection_for_head(qh, kh, vh, lay, p)
     t_sel = time.perf_counter() - t0
     tiles = np.random.default_rng(rng_seed).choice(lay.n_tiles, n_tiles, replace=False)
@@ -174,13 +175,17 @@ def run_reference(args):
         wl = wl.with_(sink=SINKS[args.sink])
     lay = O.build_layout([O.Segment(k, s, n, gr) for (k, s, n, gr) in wl.segments()], wl.seq_len)
     bits = W.make_inputs(wl, lay.inv // O.TILE)
+    if args.gate == "channel":
+        bits = bits[:3] + (W.make_channel_gate(wl),)
     n_tiles = args.ref_tiles
     for i in range(args.warmup):
-        oracle_sample(wl, bits, lay, head=i % wl.H, n_tiles=max(2, n_tiles // 4), rng_seed=i)
+        oracle_sample(wl, bits, lay, head=i % wl.H, n_tiles=max(2, n_tiles // 4), rng_seed=i,
+                      coarse=COARSES[args.coarse])
     secs, flops = 0.0, 0.0
     per_call = []
     for i in range(args.steps):
-        s, fl, pc = oracle_sample(wl, bits, lay, head=(i * 7) % wl.H, n_tiles=n_tiles, rng_seed=100 + i)
+        s, fl, pc = oracle_sample(wl, bits, lay, head=(i * 7) % wl.H, n_tiles=n_tiles, rng_seed=100 + i,
+                                  coarse=COARSES[args.coarse])
         secs += s
         flops += fl
         per_call.append(pc)
@@ -191,7 +196,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": describe(wl) + ", %s output" % args.out_dtype, "B": wl.B,
+            "config": {"workload": describe(wl) + ", %s coarse, %s gate, %s output" % (args.coarse, args.gate, args.out_dtype), "B": wl.B,
                        "seq_len": wl.seq_len, "parallelism": "host cores",
                        "l2": "inputs (2.5 GB) larger than L2; no flush"},
             "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
@@ -223,11 +228,13 @@ def run_ours(args):
     lay = vsa.Layout(wl.segments(), wl.seq_len)
     perm, inv, counts, kinds = lay.tables()
     bits = W.make_inputs(wl, inv // vsa.TILE)
+    if args.gate == "channel":
+        bits = bits[:3] + (W.make_channel_gate(wl),)
     to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
     q, k, v, g = (to_dev(x) for x in bits)
     stream = torch.cuda.Stream(device=dev)
     out_dtype = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
-    params = vsa.make_params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink)
+    params = vsa.make_params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=COARSES[args.coarse])
     with torch.cuda.stream(stream):
         fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, out_dtype=out_dtype, stream=stream)
         out = torch.empty(q.shape, dtype=out_dtype, device=dev)
@@ -368,7 +375,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": describe(wl) + ", %s output" % args.out_dtype,
+            "config": {"workload": describe(wl) + ", %s coarse, %s gate, %s output" % (args.coarse, args.gate, args.out_dtype),
                        "B": wl.B, "seq_len": wl.seq_len, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
                        "l2": "inputs (2.5 GB) larger than L2; no flush"},
             "roofline": {"bound": "tensor", "kernel": "vsa_attn_kernel", "achieved": achieved, "peak": peak,
@@ -394,7 +401,8 @@ def run_ours(args):
         if world == 1 and not args.no_cpu_baseline:
             from oracle import vsa_oracle as O
             olay = O.build_layout([O.Segment(k_, s_, n_, g_) for (k_, s_, n_, g_) in wl.segments()], wl.seq_len)
-            secs, fl, per_call = oracle_sample(wl, bits, olay, head=0, n_tiles=args.ref_tiles)
+            secs, fl, per_call = oracle_sample(wl, bits, olay, head=0, n_tiles=args.ref_tiles,
+                                               coarse=COARSES[args.coarse])
             line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
                                     "kind": "oracle", "ms_per_call_extrapolated": per_call * 1e3,
                                     "sample": "head 0: whole selection pro rata + fine branch of %d random "
@@ -414,6 +422,10 @@ def main():
     ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32")
     ap.add_argument("--sink", choices=sorted(SINKS), default=None,
                     help="override the workload's sink_conditioning mode")
+    ap.add_argument("--gate", choices=["token", "channel"], default="token",
+                    help="gate g[B,S,H] (one per token and head) or g[B,S,H,128] (one per channel)")
+    ap.add_argument("--coarse", choices=sorted(COARSES), default="mean",
+                    help="compressed-branch summaries: mean pooling or Spark-Reweight")
     ap.add_argument("--ref-tiles", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the torch SDPA comparator")

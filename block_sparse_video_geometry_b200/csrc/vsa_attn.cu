@@ -294,8 +294,13 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_co
   if (threadIdx.x == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = n;
 }
 
-// 144 registers per thread: two CTAs of 224 threads fit one SM's register file.
-__global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArgs a) {
+// At most 128 registers per thread: each of an SM's four sub-partitions has its
+// own 16K-entry register file, and two CTAs of 7 warps place 4 warps on two of
+// them (4 x 32 x 128 = 16K); a higher count leaves room for one CTA per SM.
+// kChannelGate: one gate per channel (g_sd > 0), a separate instantiation so
+// that the per-token form keeps its register allocation.
+template <bool kChannelGate>
+__global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {          // swizzled tiles need 1024-byte alignment
     if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
@@ -590,7 +595,7 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
       if (row_ok && !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && it.qt < G.n_cond)) {
         gp = a.g + a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh;
         gate = __uint_as_float(static_cast<uint32_t>(gp[0]) << 16);
-        gp = a.g_sd ? gp + 64 * hf * a.g_sd : nullptr;
+        gp = kChannelGate ? gp + 64 * hf * a.g_sd : nullptr;
         oc = a.o_coarse + ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + it.qt) * kHeadDim + 64 * hf;
       }
       // O = O(half of step j0) + O(other half) when the item had two steps or more
@@ -613,15 +618,33 @@ __global__ void __maxnreg__(144) vsa_attn_kernel(const __grid_constant__ AttnArg
         if (row_ok) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] *= inv_l;
-          if (oc && gp) {
+          if (kChannelGate && oc) {
+            // this chunk's 32 gates as bf16 pairs (vector loads when the channels are contiguous)
+            const uint16_t* gc = gp + static_cast<int64_t>(ch) * 32 * a.g_sd;
+            uint32_t gw[16];
+            if (a.g_sd == 1 && (reinterpret_cast<uintptr_t>(gc) & 15u) == 0) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const uint4 t = __ldg(reinterpret_cast<const uint4*>(gc) + u);
+                gw[4 * u] = t.x;
+                gw[4 * u + 1] = t.y;
+                gw[4 * u + 2] = t.z;
+                gw[4 * u + 3] = t.w;
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 16; ++u)
+                gw[u] = static_cast<uint32_t>(__ldg(gc + 2 * u * a.g_sd)) |
+                        (static_cast<uint32_t>(__ldg(gc + (2 * u + 1) * a.g_sd)) << 16);
+            }
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               const float4 cv = *reinterpret_cast<const float4*>(oc + ch * 32 + i);
-              const int64_t d = ch * 32 + i;
-              y[i] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + d * a.g_sd)) << 16), cv.x, y[i]);
-              y[i + 1] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + (d + 1) * a.g_sd)) << 16), cv.y, y[i + 1]);
-              y[i + 2] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + (d + 2) * a.g_sd)) << 16), cv.z, y[i + 2]);
-              y[i + 3] = fmaf(__uint_as_float(static_cast<uint32_t>(__ldg(gp + (d + 3) * a.g_sd)) << 16), cv.w, y[i + 3]);
+              const uint32_t g0 = gw[i / 2], g1 = gw[i / 2 + 1];
+              y[i] = fmaf(__uint_as_float(g0 << 16), cv.x, y[i]);
+              y[i + 1] = fmaf(__uint_as_float(g0 & 0xFFFF0000u), cv.y, y[i + 1]);
+              y[i + 2] = fmaf(__uint_as_float(g1 << 16), cv.z, y[i + 2]);
+              y[i + 3] = fmaf(__uint_as_float(g1 & 0xFFFF0000u), cv.w, y[i + 3]);
             }
           } else if (oc) {
 #pragma unroll
@@ -804,7 +827,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.err = static_cast<int*>(workspace);
   a.stall_ns = g_stall_ns.load(std::memory_order_relaxed);
 
-  cudaError_t e = cudaFuncSetAttribute(vsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto attn_kernel = g_sd > 0 ? vsa_attn_kernel<true> : vsa_attn_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
   e = cudaMemsetAsync(workspace, 0, kAttnHeader, stream);
@@ -825,7 +849,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   for (int b = 0; b < B; ++b) {
     a.b = b;
     a.q = static_cast<const uint16_t*>(q) + b * sb;
-    vsa_attn_kernel<<<grid, kThreads, smem, stream>>>(a);
+    attn_kernel<<<grid, kThreads, smem, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: launch", e);
   }

@@ -103,6 +103,7 @@ vsa_status check_qkv(const void* q, const void* k, const void* v, int64_t sb, in
 // Workspace layout of vsa_coarse_select.
 struct SelectWorkspace {
   size_t pooled, scores, stats, total;
+  size_t anchor, summaries, bias;   // VSA_COARSE_REWEIGHT only: [B,H,128], [2,B,H,Nc,128], [B,H,Nc]
   int32_t n_row_blocks;   // 64-query-tile blocks of the coarse kernel
   int32_t ld_scores;      // score row stride: Nc rounded up to 64
 };

@@ -54,6 +54,7 @@ vsa_status check_params(const vsa_params* p) {
   if (p->mode == VSA_SELECT_ADAPTIVE && !(p->tau >= 0.0f && std::isfinite(p->tau)))
     return VSA_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return VSA_ERR_INVALID_ARG;
+  if (p->coarse != VSA_COARSE_MEAN && p->coarse != VSA_COARSE_REWEIGHT) return VSA_ERR_INVALID_ARG;
   return VSA_OK;
 }
 
@@ -86,6 +87,16 @@ SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H, cons
   off = align_up(off + bh * L->n_tiles * static_cast<size_t>(w.ld_scores) * sizeof(float), 256);
   w.stats = off;
   off = align_up(off + bh * w.n_row_blocks * 2 * sizeof(double), 256);
+  w.anchor = w.summaries = w.bias = off;
+  if (p->coarse == VSA_COARSE_REWEIGHT) {
+    const size_t nc = static_cast<size_t>(candidates(L, p->sink).count);
+    w.anchor = off;
+    off = align_up(off + bh * kHeadDim * sizeof(float), 256);
+    w.summaries = off;
+    off = align_up(off + 2 * bh * nc * kHeadDim * sizeof(float), 256);
+    w.bias = off;
+    off = align_up(off + bh * nc * sizeof(float), 256);
+  }
   w.total = off;
   return w;
 }
@@ -282,7 +293,7 @@ const char* vsa_status_string(vsa_status s) {
   return "unknown status";
 }
 
-int32_t vsa_version(void) { return (1 << 16) | 1; }
+int32_t vsa_version(void) { return (1 << 16) | 2; }
 
 const char* vsa_last_error_detail(void) { return g_detail; }
 

@@ -84,6 +84,93 @@ pool_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restr
   }
 }
 
+// --------------------------------------------------------- Spark-Reweight
+// Anchor of each (batch, head): the mean query of the video tokens, from the
+// pooled tile means weighted by the tiles' token counts (fp64 sums).
+// grid (H, B), 128 threads (one per dim).
+__global__ void __launch_bounds__(kHeadDim) anchor_kernel(DevLayout L, int H, const float* __restrict__ pooled_q,
+                                                          float* __restrict__ anchor) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const size_t bh = static_cast<size_t>(b) * H + h;
+  double acc = 0.0, n = 0.0;
+#pragma unroll 4
+  for (int t = L.n_cond; t < L.n_tiles; ++t) {
+    const double c = static_cast<double>(L.count[t]);
+    acc += c * static_cast<double>(pooled_q[(bh * L.n_tiles + t) * kHeadDim + d]);
+    n += c;
+  }
+  anchor[bh * kHeadDim + d] = static_cast<float>(acc / n);
+}
+
+// Weighted summaries and log-mass bias of every candidate key tile: with the
+// anchor logits x_i = scale <a, k_i> of the tile's valid tokens,
+//   K~ = sum w_i k_i, V~ = sum w_i v_i, w = softmax(x), b = log(mean exp(x)) - scale <a, K~>.
+// grid (n_cand, B), 256 threads; warp w handles heads w, w + 8, ...; lane l
+// handles dims 4l .. 4l + 3 (one 8-byte load per token row and tensor).
+constexpr int kReweightThreads = 256;
+
+__global__ void __launch_bounds__(kReweightThreads)
+reweight_kernel(DevLayout L, int cand0, int n_cand, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+                int64_t sb, int64_t ss, int64_t sh, int H, int B, float scale, const float* __restrict__ anchor,
+                float* __restrict__ summaries, float* __restrict__ bias) {
+  const int c = blockIdx.x, b = blockIdx.y, tile = cand0 + c;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int tok[kTile];
+  __shared__ float xs[kReweightThreads / 32][kTile];
+  for (int i = threadIdx.x; i < kTile; i += kReweightThreads) tok[i] = L.perm[tile * kTile + i];
+  __syncthreads();
+  const float n = static_cast<float>(L.count[tile]);
+  for (int h = warp; h < H; h += kReweightThreads / 32) {
+    const size_t bh = static_cast<size_t>(b) * H + h;
+    const float4 a = reinterpret_cast<const float4*>(anchor + bh * kHeadDim)[lane];
+    const uint16_t* kb = k + b * sb + h * sh + 4 * lane;
+    const uint16_t* vb = v + b * sb + h * sh + 4 * lane;
+    float m = -INFINITY;
+    for (int s = 0; s < kTile; ++s) {
+      const int t = tok[s];
+      float x = -INFINITY;
+      if (t >= 0) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(kb + static_cast<int64_t>(t) * ss));
+        float part = a.x * bf16lo(w.x) + a.y * bf16hi(w.x) + a.z * bf16lo(w.y) + a.w * bf16hi(w.y);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        x = part * scale;
+      }
+      if (lane == 0) xs[warp][s] = x;
+      m = fmaxf(m, x);
+    }
+    __syncwarp();
+    float z = 0.f, ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < kTile; ++s) {
+      const int t = tok[s];
+      if (t < 0) continue;
+      const float e = expf(xs[warp][s] - m);
+      z += e;
+      const uint2 kw = __ldg(reinterpret_cast<const uint2*>(kb + static_cast<int64_t>(t) * ss));
+      const uint2 vw = __ldg(reinterpret_cast<const uint2*>(vb + static_cast<int64_t>(t) * ss));
+      ks[0] = fmaf(e, bf16lo(kw.x), ks[0]); ks[1] = fmaf(e, bf16hi(kw.x), ks[1]);
+      ks[2] = fmaf(e, bf16lo(kw.y), ks[2]); ks[3] = fmaf(e, bf16hi(kw.y), ks[3]);
+      vs[0] = fmaf(e, bf16lo(vw.x), vs[0]); vs[1] = fmaf(e, bf16hi(vw.x), vs[1]);
+      vs[2] = fmaf(e, bf16lo(vw.y), vs[2]); vs[3] = fmaf(e, bf16hi(vw.y), vs[3]);
+    }
+    const float inv = 1.0f / z;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ks[e] *= inv;
+      vs[e] *= inv;
+    }
+    float part = a.x * ks[0] + a.y * ks[1] + a.z * ks[2] + a.w * ks[3];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    const size_t plane = static_cast<size_t>(B) * H * n_cand * kHeadDim;
+    float* kd = summaries + (bh * n_cand + c) * kHeadDim;
+    reinterpret_cast<float4*>(kd)[lane] = make_float4(ks[0], ks[1], ks[2], ks[3]);
+    reinterpret_cast<float4*>(kd + plane)[lane] = make_float4(vs[0], vs[1], vs[2], vs[3]);
+    if (lane == 0) bias[bh * n_cand + c] = m + logf(z / n) - scale * part;
+    __syncwarp();   // xs[warp] is rewritten by the next head
+  }
+}
+
 // ------------------------------------------------------- scores + coarse
 // grid (ceil(n_tiles / 64), H, B), 256 threads. Thread (ty, tx) = (tid / 16,
 // tid % 16) owns query rows 4*ty .. 4*ty+3; in the score block it owns candidate
@@ -94,11 +181,13 @@ struct CoarseSmem {
   float p[kCoarseRows][kCoarseCols + 4];  // probabilities of the chunk
 };
 
-template <bool kStats>
+// With kReweight the selection scores still use the mean-pooled K, and the
+// coarse softmax uses scale <Qbar, K~> + b against V~ (Spark-Reweight).
+template <bool kStats, bool kReweight>
 __global__ void __launch_bounds__(kCoarseThreads, 2)
 coarse_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __restrict__ pooled,
               float scale, float* __restrict__ scores, int ld_scores, float* __restrict__ o_coarse,
-              double* __restrict__ stats) {
+              double* __restrict__ stats, const float* __restrict__ summaries, const float* __restrict__ rbias) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   CoarseSmem& sm = *reinterpret_cast<CoarseSmem*>(smem_raw);
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
@@ -108,6 +197,9 @@ coarse_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __r
   const float* qbar = pooled + bh * n_tiles * kHeadDim;
   const float* kbar = pooled + plane + (bh * n_tiles + cand0) * kHeadDim;
   const float* vbar = pooled + 2 * plane + (bh * n_tiles + cand0) * kHeadDim;
+  const size_t rplane = static_cast<size_t>(B) * H * n_cand * kHeadDim;
+  const float* ktil = kReweight ? summaries + bh * n_cand * kHeadDim : nullptr;
+  const float* vsum = kReweight ? summaries + rplane + bh * n_cand * kHeadDim : vbar;
 
   // pooled Q rows of this block, transposed; rows past n_tiles are zero
   for (int f = tid; f < kCoarseRows * kHeadDim / 4; f += kCoarseThreads) {
@@ -131,35 +223,39 @@ coarse_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __r
   double s1 = 0.0, s2 = 0.0;
 
   for (int c0 = 0; c0 < n_cand; c0 += kCoarseCols) {
-    __syncthreads();  // previous chunk's Vbar / p are consumed
-    for (int f = tid; f < kCoarseCols * kHeadDim / 4; f += kCoarseThreads) {
-      const int c = f % kCoarseCols, d4 = f / kCoarseCols;
-      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + c < n_cand) val = reinterpret_cast<const float4*>(kbar + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
-      sm.kv[(4 * d4 + 0) * kCoarseCols + c] = val.x;
-      sm.kv[(4 * d4 + 1) * kCoarseCols + c] = val.y;
-      sm.kv[(4 * d4 + 2) * kCoarseCols + c] = val.z;
-      sm.kv[(4 * d4 + 3) * kCoarseCols + c] = val.w;
-    }
-    __syncthreads();
-
+    // chunk of key summaries (rows c0 .. c0 + 63 of src) into sm.kv, transposed
+    // [d][c], then acc = Qbar K^T for this thread's 4 x 4 block
     float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < kHeadDim; ++d) {
-      const float4 a = *reinterpret_cast<const float4*>(&sm.qT[d][4 * ty]);
-      const float4 bb = *reinterpret_cast<const float4*>(&sm.kv[d * kCoarseCols + 4 * tx]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+    auto chunk_dots = [&](const float* src) {
+      __syncthreads();  // previous readers of sm.kv are done
+      for (int f = tid; f < kCoarseCols * kHeadDim / 4; f += kCoarseThreads) {
+        const int c = f % kCoarseCols, d4 = f / kCoarseCols;
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c0 + c < n_cand) val = reinterpret_cast<const float4*>(src + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
+        sm.kv[(4 * d4 + 0) * kCoarseCols + c] = val.x;
+        sm.kv[(4 * d4 + 1) * kCoarseCols + c] = val.y;
+        sm.kv[(4 * d4 + 2) * kCoarseCols + c] = val.z;
+        sm.kv[(4 * d4 + 3) * kCoarseCols + c] = val.w;
+      }
+      __syncthreads();
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+      for (int d = 0; d < kHeadDim; ++d) {
+        const float4 a = *reinterpret_cast<const float4*>(&sm.qT[d][4 * ty]);
+        const float4 bb = *reinterpret_cast<const float4*>(&sm.kv[d * kCoarseCols + 4 * tx]);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      }
+    };
+    chunk_dots(kbar);
 
-    // scale, write scores, statistics, online softmax
+    // scale, write the selection scores, statistics
     float s[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -177,6 +273,22 @@ coarse_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __r
         float4* dst = reinterpret_cast<float4*>(scores + (bh * n_tiles + row) * ld_scores + c0 + 4 * tx);
         *dst = make_float4(s[i][0], s[i][1], s[i][2], s[i][3]);
       }
+    }
+    if (kReweight) {
+      // the coarse logits: scale <Qbar, K~> + b
+      chunk_dots(ktil);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int col = c0 + 4 * tx + j;
+        const float bj = col < n_cand ? rbias[bh * n_cand + col] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[i][j] = col < n_cand ? fmaf(acc[i][j], scale, bj) : -INFINITY;
+      }
+    }
+
+    // online softmax of the chunk
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
       float cm = fmaxf(fmaxf(s[i][0], s[i][1]), fmaxf(s[i][2], s[i][3]));
 #pragma unroll
       for (int off = 1; off < 16; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
@@ -197,13 +309,13 @@ coarse_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __r
       for (int e = 0; e < 8; ++e) o[i][e] *= corr;
       *reinterpret_cast<float4*>(&sm.p[4 * ty + i][4 * tx]) = make_float4(pv[0], pv[1], pv[2], pv[3]);
     }
-    __syncthreads();  // scores consumed Kbar; p is complete
+    __syncthreads();  // the dots consumed sm.kv; p is complete
 
-    // Vbar chunk [c][d] into the same buffer
+    // Vbar (or V~) chunk [c][d] into the same buffer
     for (int f = tid; f < kCoarseCols * kHeadDim / 4; f += kCoarseThreads) {
       const int c = f / (kHeadDim / 4), d4 = f % (kHeadDim / 4);
       float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + c < n_cand) val = reinterpret_cast<const float4*>(vbar + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
+      if (c0 + c < n_cand) val = reinterpret_cast<const float4*>(vsum + static_cast<size_t>(c0 + c) * kHeadDim)[d4];
       reinterpret_cast<float4*>(sm.kv)[f] = val;
     }
     __syncthreads();
@@ -456,13 +568,25 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
       D, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
       static_cast<const uint16_t*>(v), sb, ss, sh, H, B, pooled);
 
+  const bool reweight = p->coarse == VSA_COARSE_REWEIGHT;
+  float* anchor = reinterpret_cast<float*>(w + ws.anchor);
+  float* summaries = reinterpret_cast<float*>(w + ws.summaries);
+  float* rbias = reinterpret_cast<float*>(w + ws.bias);
+  if (reweight) {
+    anchor_kernel<<<dim3(H, B), kHeadDim, 0, stream>>>(D, H, pooled, anchor);
+    reweight_kernel<<<dim3(cand.count, B), kReweightThreads, 0, stream>>>(
+        D, cand.first, cand.count, static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), sb, ss, sh, H,
+        B, scale, anchor, summaries, rbias);
+  }
+
   const size_t coarse_smem = sizeof(CoarseSmem);
-  auto ck = adaptive ? coarse_kernel<true> : coarse_kernel<false>;
+  auto ck = adaptive ? (reweight ? coarse_kernel<true, true> : coarse_kernel<true, false>)
+                     : (reweight ? coarse_kernel<false, true> : coarse_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(coarse_smem));
   if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: cudaFuncSetAttribute(coarse)", e);
   ck<<<dim3(ws.n_row_blocks, H, B), kCoarseThreads, coarse_smem, stream>>>(
-      L->n_tiles, cand.first, cand.count, H, B, pooled, scale, scores, ld, o_coarse, stats);
+      L->n_tiles, cand.first, cand.count, H, B, pooled, scale, scores, ld, o_coarse, stats, summaries, rbias);
 
   const size_t sel_smem = rows_per_block * row_bytes + rows_per_block * 256 * sizeof(uint32_t);
   auto sk = adaptive ? select_kernel<true> : select_kernel<false>;

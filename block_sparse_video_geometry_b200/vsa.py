@@ -20,6 +20,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, ERR_TIM
 SEG_TEXT, SEG_REF_IMAGE, SEG_REF_AUDIO, SEG_OTHER_COND, SEG_VIDEO = range(5)
 SELECT_TOPK, SELECT_ADAPTIVE = 0, 1
 SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS, SINK_OFF = 0, 1, 2
+COARSE_MEAN, COARSE_REWEIGHT = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 TILE, HEAD_DIM = 64, 128
 
@@ -40,7 +41,7 @@ class Segment(ctypes.Structure):
 
 class Params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("keep", ctypes.c_float), ("tau", ctypes.c_float),
-                ("sink", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("sink", ctypes.c_int32), ("scale", ctypes.c_float), ("coarse", ctypes.c_int32)]
 
 
 class LayoutInfo(ctypes.Structure):
@@ -108,8 +109,8 @@ def _check(status: int, where: str) -> None:
 
 
 def make_params(mode: int = SELECT_TOPK, keep: float = 0.1, tau: float = 1.0,
-                sink: int = SINK_EXACT_KV, scale: float = 0.0) -> Params:
-    return Params(mode, keep, tau, sink, scale)
+                sink: int = SINK_EXACT_KV, scale: float = 0.0, coarse: int = 0) -> Params:
+    return Params(mode, keep, tau, sink, scale, coarse)
 
 
 def _stream_handle(stream) -> int:

@@ -141,3 +141,20 @@ def make_inputs(wl: Workload, cluster_of_token: np.ndarray, threads: int = 8):
     with ThreadPoolExecutor(max(1, threads)) as ex:
         list(ex.map(fill, jobs))
     return qkv[0], qkv[1], qkv[2], g
+
+
+def make_channel_gate(wl: Workload, threads: int = 8) -> np.ndarray:
+    """A per-channel gate g ~ U(0, 1) on [B, S, H, D] as bf16 bits, drawn per
+    chunk of tokens from PCG64 streams keyed (seed, 5, batch, chunk)."""
+    S, H, D, B = wl.seq_len, wl.H, wl.D, wl.B
+    g = np.empty((B, S, H, D), dtype=np.uint16)
+    n_chunks = -(-S // CHUNK_TOKENS)
+
+    def fill(job):
+        b, ch = job
+        s0, s1 = ch * CHUNK_TOKENS, min(S, (ch + 1) * CHUNK_TOKENS)
+        g[b, s0:s1] = f32_to_bf16_bits(_rng(wl.seed, 5, b, ch).random((s1 - s0, H, D), dtype=np.float32))
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(fill, [(b, ch) for b in range(B) for ch in range(n_chunks)]))
+    return g

@@ -94,6 +94,18 @@ typedef enum { VSA_SINK_EXACT_KV = 0, VSA_SINK_EXACT_KV_AND_ROWS = 1, VSA_SINK_O
 
 typedef enum { VSA_OUT_F32 = 0, VSA_OUT_BF16 = 1 } vsa_out_dtype;
 
+/* Compressed (coarse) branch summaries of the candidate key tiles.
+ * MEAN: mean-pooled K and V ("Spark-H3: atencion dispersa por bloques ...",
+ * "Que cambia Spark-Attn": mean-pooled key/value summary).
+ * REWEIGHT: Spark-Reweight (same section; reading): per (batch, head) the
+ * anchor a is the mean query of the video tokens; each candidate tile is
+ * summarised by the anchor's softmax weights over its tokens,
+ * K~ = sum w_i k_i, V~ = sum w_i v_i with w = softmax_i(scale <a, k_i>), plus
+ * the log-mass bias b = log(mean_i exp(scale <a, k_i>)) - scale <a, K~>; the
+ * branch is o_coarse = softmax_c(scale <Qbar, K~_c> + b_c) V~_c. The
+ * selection always uses the mean-pooled scores. */
+typedef enum { VSA_COARSE_MEAN = 0, VSA_COARSE_REWEIGHT = 1 } vsa_coarse_mode;
+
 /* Selection parameters.
  *  mode  : VSA_SELECT_TOPK keeps k = max(1, ceil(keep * Nc)) candidate key
  *          tiles per query tile (Nc = number of candidate tiles, see
@@ -105,13 +117,15 @@ typedef enum { VSA_OUT_F32 = 0, VSA_OUT_BF16 = 1 } vsa_out_dtype;
  *  keep  : (0, 1], used by TOPK.
  *  tau   : >= 0, used by ADAPTIVE.
  *  sink  : vsa_sink_mode.
- *  scale : softmax scale of both branches; <= 0 selects 1/sqrt(128). */
+ *  scale : softmax scale of both branches; <= 0 selects 1/sqrt(128).
+ *  coarse: vsa_coarse_mode. */
 typedef struct {
   int32_t mode;
   float keep;
   float tau;
   int32_t sink;
   float scale;
+  int32_t coarse;
 } vsa_params;
 
 typedef struct vsa_layout vsa_layout;   /* opaque; owns its host tables */

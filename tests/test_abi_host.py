@@ -86,6 +86,10 @@ def test_sink_off_candidates_are_all_tiles():
         assert lay.kmax(vsa.make_params(keep=keep, sink=vsa.SINK_OFF)) == \
             O.topk_count(keep, O.candidate_tiles(ref, O.SINK_OFF)[1])
     assert lay.kmax(vsa.make_params(mode=vsa.SELECT_ADAPTIVE, sink=vsa.SINK_OFF)) == nt
+    # Spark-Reweight adds its anchor, summaries and biases to the selection workspace
+    rw = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5, coarse=vsa.COARSE_REWEIGHT))
+    on = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5))
+    assert rw >= on + 2 * 2 * lay.info.n_video_tiles * 128 * 4
     # the score matrix spans every tile: the selection workspace grows accordingly
     on = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5))
     off = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5, sink=vsa.SINK_OFF))
@@ -130,7 +134,7 @@ def test_calls_validate_before_any_gpu_work():
     good = vsa.make_params(keep=0.5)
     n = ctypes.c_size_t()
     for bad in [vsa.make_params(keep=0.0), vsa.make_params(keep=1.5), vsa.make_params(mode=3),
-                vsa.make_params(sink=5), vsa.make_params(sink=3), vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=-1.0),
+                vsa.make_params(sink=5), vsa.make_params(sink=3), vsa.make_params(coarse=2), vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=-1.0),
                 vsa.make_params(scale=float("nan"))]:
         assert L.vsa_coarse_select_workspace_size(lay.handle, 1, 2, ctypes.byref(bad), ctypes.byref(n)) == \
             vsa.ERR_INVALID_ARG

@@ -123,6 +123,22 @@ def test_channel_gate(cuda_ok, wl, out_dtype):
     full_check(wl, out_dtype=out_dtype, channel_gate=True)
 
 
+@pytest.mark.parametrize("wl,prm", [
+    (W.WORKLOADS["tiny"], {}),
+    (EDGE_WORKLOADS[0], {}),                                   # partial tiles, two batches
+    (W.WORKLOADS["tiny"], {"sink": O.SINK_OFF}),
+    (W.WORKLOADS["tiny"].with_(mode=O.MODE_ADAPTIVE, tau=1.0), {}),
+], ids=["tiny", "ragged_b2", "tiny_sink_off", "tiny_adaptive"])
+def test_spark_reweight(cuda_ok, wl, prm):
+    """Spark-Reweight compressed branch (weighted summaries + log-mass bias)."""
+    full_check(wl, coarse=O.COARSE_REWEIGHT, **prm)
+
+
+def test_mid_spark_reweight_two_heads(cuda_ok):
+    wl = W.WORKLOADS["mid"].with_(H=4)
+    full_check(wl, heads=(1, 2), out_tiles=lambda lay: range(3, lay.n_tiles, 11), coarse=O.COARSE_REWEIGHT)
+
+
 def test_mid_sink_off_two_heads(cuda_ok):
     wl = W.WORKLOADS["mid"].with_(H=4)
     full_check(wl, heads=(0, 3), out_tiles=lambda lay: range(0, lay.n_tiles, 9), sink=O.SINK_OFF,

@@ -33,13 +33,12 @@ def inputs(wl, lay, channel_gate=False):
     (seeded U(0, 1) per channel) instead of [B, S, H]."""
     q, k, v, g = W.make_inputs(wl, lay.inv // O.TILE)
     if channel_gate:
-        rng = np.random.default_rng(1000 + wl.seed)
-        g = W.f32_to_bf16_bits(rng.uniform(0.0, 1.0, (wl.B, wl.seq_len, wl.H, wl.D)).astype(np.float32))
+        g = W.make_channel_gate(wl)
     return q, k, v, g
 
 
 def params_of(wl, **kw):
-    d = dict(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink)
+    d = dict(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=O.COARSE_MEAN)
     d.update(kw)
     return d
 
@@ -76,7 +75,8 @@ class HeadOracle:
         self.q, self.k, self.v = f(q[b, :, h]), f(k[b, :, h]), f(v[b, :, h])
         self.g = f(g[b, :, h])
         self.lay = lay
-        self.p = O.Params(mode=prm["mode"], keep=prm["keep"], tau=prm["tau"], sink=prm["sink"])
+        self.p = O.Params(mode=prm["mode"], keep=prm["keep"], tau=prm["tau"], sink=prm["sink"],
+                          coarse=prm.get("coarse", O.COARSE_MEAN))
         (self.qbar, self.kbar, self.vbar, self.scores, self.sel, self.thr, self.o_coarse,
          self.scale) = O.selection_for_head(self.q, self.k, self.v, lay, self.p)
 
