@@ -222,7 +222,8 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wl = W.WORKLOADS[args.workload].with_(seed=W.WORKLOADS[args.workload].seed + rank)
+    from block_sparse_video_geometry_b200 import sharding
+    wl = W.WORKLOADS[args.workload].with_(seed=sharding.replica_seed(W.WORKLOADS[args.workload].seed, rank))
     if args.sink is not None:
         wl = wl.with_(sink=SINKS[args.sink])
     lay = vsa.Layout(wl.segments(), wl.seq_len)
@@ -356,10 +357,8 @@ def run_ours(args):
         raise RuntimeError("kernel status %s" % vsa.status_string(st))
     del dev_in, dev_out
 
-    times = torch.tensor([ms_step, ms_e2e, att_ms, sel_ms], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    ms_step, ms_e2e, att_ms, sel_ms = times.tolist()
+    ms_step, ms_e2e, att_ms, sel_ms = sharding.max_over_ranks([ms_step, ms_e2e, att_ms, sel_ms], dist, dev)
+    job_flop, = sharding.sum_over_ranks([flop], dist, dev)   # the work of every replica
 
     if rank == 0:
         peaks, src = measured_peaks()
@@ -370,7 +369,7 @@ def run_ours(args):
         sel_bytes = (3 * q.numel() * 2                                           # Q, K, V read once
                      + 2 * wl.B * wl.H * info.n_tiles * ld * 4                    # scores written + read
                      + 4 * wl.B * wl.H * info.n_tiles * (fwd.kmax + 1 + 128))    # idx, cnt, o_coarse
-        value = world * flop / (ms_step * 1e-3) / 1e12
+        value = job_flop / (ms_step * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -387,11 +386,11 @@ def run_ours(args):
                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": sel_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                           "bytes_per_call": sel_bytes, "ms_per_call": sel_ms},
-            "e2e": {"value": world * flop / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": job_flop / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                     "steps": e2e_steps, "copies": "overlap the neighbouring steps' compute"},
-            # per step: pool, coarse, select; permute, schedule, one attention launch per batch
-            "gpu_launches": (5 + wl.B) * args.steps,
+            # per step and rank: pool, coarse, select; permute, schedule, one attention launch per batch
+            "gpu_launches": (5 + wl.B) * args.steps * world,
             "clocks": clocks.summary(),
             "call_ms": {"p50": call_p50, "p90": call_p90, "samples": len(call_ms)},
             "dense_sdpa": None if dense_ms is None else {
