@@ -23,9 +23,9 @@ def sample_tiles(lay, rng, n_random=6):
     return sorted(fixed | set(rng.choice(nt, n_random, replace=False).tolist()))
 
 
-def run_case(wl, heads, n_random=6, g_zero=False, **prm_over):
+def run_case(wl, heads, n_random=6, g_zero=False, channel_gate=False, **prm_over):
     lay = C.oracle_layout(wl)
-    q, k, v, g = C.inputs(wl, lay)
+    q, k, v, g = C.inputs(wl, lay, channel_gate)
     if g_zero:
         g = np.zeros_like(g)
     prm = C.params_of(wl, **prm_over)
@@ -56,6 +56,17 @@ def test_5s_topk_10pct(cuda_ok):
 def test_10s_ragged_rows_dense(cuda_ok):
     lay, res, kept = run_case(W.WORKLOADS["10s"], heads=(0, 23), n_random=4)
     assert lay.n_video_tiles == 4032 and res["kmax"] == 404
+
+
+def test_5s_sink_off(cuda_ok):
+    """sink_conditioning off at full size: every tile is a candidate."""
+    lay, res, kept = run_case(W.WORKLOADS["5s"], heads=(5,), n_random=4, sink=O.SINK_OFF)
+    assert res["kmax"] == O.topk_count(0.1, lay.n_tiles) == 209
+
+
+def test_5s_spark_reweight_channel_gate(cuda_ok):
+    """Spark-Reweight compressed branch and a per-channel gate at full size."""
+    run_case(W.WORKLOADS["5s"], heads=(7,), n_random=4, channel_gate=True, coarse=O.COARSE_REWEIGHT)
 
 
 @pytest.mark.parametrize("tau", [1.0, 1.5, 2.0])
