@@ -40,6 +40,25 @@ SINKS = {"exact_kv": 0, "exact_kv_and_rows": 1, "off": 2}
 COARSES = {"mean": 0, "reweight": 1}
 
 
+def captured_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary of this
+    workload, or None when there is none or the kernel sources changed since
+    the counters were taken (the summary records their sha256 prefix)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", "vsa_attn_kernel_%s_dram.md" % workload)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    src = b"".join(open(os.path.join(ROOT, "block_sparse_video_geometry_b200", "csrc", f), "rb").read()
+                   for f in ("vsa_attn.cu", "sm100.cuh"))
+    m = re.search(r"sha256 prefix: ([0-9a-f]{16})", text)
+    t = re.search(r"traffic per launch \(read \+ write\) \| ([0-9,]+) B", text)
+    if not m or not t or m.group(1) != hashlib.sha256(src).hexdigest()[:16]:
+        return None
+    return int(t.group(1).replace(",", ""))
+
+
 def valid_flop_fast(counts, n_cond, idx, cnt, sink_rows, sink_off=False):
     """Valid fine-branch FLOP of one call: 4 * 128 per attended (valid query,
     valid key) pair; keys of a query tile = conditioning tokens + tokens of its
@@ -378,7 +397,10 @@ def run_ours(args):
                        "B": wl.B, "seq_len": wl.seq_len, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
                        "l2": "inputs (2.5 GB) larger than L2; no flush"},
             "roofline": {"bound": "tensor", "kernel": "vsa_attn_kernel", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": (captured_traffic(args.workload) if args.sink is None and args.coarse == "mean"
+                                     and args.gate == "token" and args.out_dtype == "f32" else None),
+                         "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "peak_source": "%s bf16_tflops_sustained" % src,
                          "frac_of_burst": achieved / peaks["bf16_tflops"],
                          "flop_per_launch": flop, "ms_per_launch": att_ms},
