@@ -386,6 +386,32 @@ def key_tokens_for_tile(layout: Layout, qt: int, selected: np.ndarray, sink: int
     return np.concatenate(parts)
 
 
+def extra_tokens_for_tile(qbar_qt: np.ndarray, k: np.ndarray, layout: Layout, selected: np.ndarray,
+                          n_extra: int, scale: float, sink: int = SINK_EXACT_KV) -> np.ndarray:
+    """extra_tokens ("ComfyUI Agrega Nodo Central de Atencion Dispersa y
+    Compilador Comfy", "Atencion dispersa por bloques": the highest-scoring
+    tokens beyond the selected blocks are added, to stay closer to dense).
+
+    Reading: the candidates are the valid tokens of the candidate key tiles
+    that query tile qt did not select (tokens it attends anyway are not
+    candidates); a token's score is scale * <qbar[qt], k_token>, the tile
+    score taken at token resolution; the n_extra highest are added to the
+    exact key set of every query of the tile (ties: lower token index).
+    Returns the added tokens in ascending order.
+    """
+    if n_extra <= 0:
+        return np.zeros(0, dtype=np.int64)
+    first, count = candidate_tiles(layout, sink)
+    chosen = set(int(c) for c in selected)
+    cand = [layout.tile_tokens(first + c) for c in range(count) if c not in chosen]
+    if not cand:
+        return np.zeros(0, dtype=np.int64)
+    toks = np.concatenate(cand)
+    sc = scale * (np.asarray(k, dtype=np.float64)[toks] @ qbar_qt)
+    order = np.lexsort((toks, -sc))             # score descending, then token index
+    return np.sort(toks[order[:n_extra]])
+
+
 def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
     """Textbook softmax(q k^T * scale) v, row by row, in float64."""
     s = scale * (q @ k.T)
@@ -414,6 +440,7 @@ class Params:
     sink: int = SINK_EXACT_KV
     scale: float = 0.0        # 0 -> 1/sqrt(D)
     coarse: int = COARSE_MEAN
+    extra_tokens: int = 0     # extra key tokens per query tile (0: none)
 
 
 @dataclass
@@ -459,6 +486,10 @@ def output_rows_for_tile(q, k, v, g, layout: Layout, params: Params, qt: int,
     Returns (tokens, o_fine, out).
     """
     keys = key_tokens_for_tile(layout, qt, selected, params.sink)
+    if params.extra_tokens > 0 and not (params.sink == SINK_EXACT_KV_AND_ROWS and qt < layout.n_cond_tiles):
+        qbar_qt = np.asarray(q, dtype=np.float64)[layout.tile_tokens(qt)].mean(axis=0)
+        extra = extra_tokens_for_tile(qbar_qt, k, layout, selected, params.extra_tokens, scale, params.sink)
+        keys = np.concatenate([keys, extra])
     of = fine_branch_tile(q, k, v, layout, qt, keys, scale)
     toks = layout.tile_tokens(qt)
     if params.sink == SINK_EXACT_KV_AND_ROWS and qt < layout.n_cond_tiles:

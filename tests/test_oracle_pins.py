@@ -462,6 +462,45 @@ def test_reweight_changes_only_the_compressed_branch():
     assert np.all(w <= vid_v.max(0) + 1e-12) and np.all(w >= vid_v.min(0) - 1e-12)
 
 
+# --------------------------------------------------------- extra tokens --
+def test_extra_tokens_brute_force():
+    """The added tokens are the E best by pooled-query score among the tokens
+    of the unselected video tiles, found here by a plain sort over tokens."""
+    wl, lay, q, k, v, g = _tiny_case()
+    E = 7
+    res = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.25, extra_tokens=E))
+    tile = lay.inv // O.TILE
+    scale = O.default_scale()
+    S = lay.seq_len
+    cond = np.zeros(S, bool)
+    cond[lay.cond_tokens()] = True
+    mask = np.zeros((S, S), bool)
+    for qt in range(lay.n_tiles):
+        rows = np.nonzero(tile == qt)[0]
+        qbar = q[rows].mean(0)
+        sel_tiles = {lay.n_cond_tiles + int(c) for c in res.selected[qt]}
+        cands = [i for i in range(S) if tile[i] >= lay.n_cond_tiles and tile[i] not in sel_tiles]
+        best = sorted(cands, key=lambda i: (-scale * float(k[i] @ qbar), i))[:E]
+        for r in rows:
+            mask[r, cond] = True
+            mask[r, [i for i in range(S) if tile[i] in sel_tiles]] = True
+            mask[r, best] = True
+    ref = O.dense_attention_masked(q, k, v, mask, scale)
+    assert np.allclose(res.o_fine, ref, atol=1e-12)
+    # E = 0 is the method without extra tokens
+    r0 = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.25))
+    r00 = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.25, extra_tokens=0))
+    assert np.array_equal(r0.out, r00.out)
+
+
+def test_extra_tokens_covering_everything_is_dense():
+    """With E at least the number of unselected video tokens every key is
+    attended: the fine branch is textbook dense attention."""
+    wl, lay, q, k, v, g = _tiny_case()
+    res = O.vsa_forward_head(q, k, v, g, lay, O.Params(keep=0.25, extra_tokens=lay.seq_len))
+    assert np.allclose(res.o_fine, O.softmax_attention(q, k, v, O.default_scale()), atol=1e-12)
+
+
 # ------------------------------------------------------------- generator --
 def test_generator_is_seeded_and_bf16_rounded():
     import torch
