@@ -554,3 +554,75 @@ def test_planted_mistakes_fail_a_pin(monkeypatch):
     bad = O.vsa_forward_head(q2, k2, v2, g2, lay2, O.Params(keep=1.0))
     dense = O.softmax_attention(q2, k2, v2, O.default_scale())
     assert not np.allclose(bad.o_fine, dense, atol=1e-6)
+
+
+# ------------------------------------------------------------- backward --
+def _bwd_case(seed=3, **kw):
+    wl, lay, q, k, v, g = _tiny_case(**kw)
+    rng = np.random.default_rng(seed)
+    dout = rng.standard_normal(q.shape)
+    return wl, lay, q, k, v, g, dout
+
+
+def test_backward_forward_restatement_matches_oracle():
+    """The torch restatement used for the gradients computes the oracle's forward."""
+    import torch
+    from oracle import vsa_backward_oracle as BO
+    wl, lay, q, k, v, g, dout = _bwd_case()
+    for p in (O.Params(keep=0.25), O.Params(keep=0.25, sink=O.SINK_OFF, coarse=O.COARSE_REWEIGHT),
+              O.Params(keep=0.5, sink=O.SINK_EXACT_KV_AND_ROWS, extra_tokens=5)):
+        ref = O.vsa_forward_head(q, k, v, g, lay, p).out
+        sel = O.selection_for_head(q, k, v, lay, p)[4]
+        got = BO.forward_torch(*(torch.tensor(x) for x in (q, k, v, g)), lay, p, sel).numpy()
+        assert np.allclose(got, ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("params", [
+    O.Params(keep=0.25),
+    O.Params(keep=0.5, sink=O.SINK_EXACT_KV_AND_ROWS),
+    O.Params(keep=0.25, sink=O.SINK_OFF, coarse=O.COARSE_REWEIGHT, extra_tokens=3),
+], ids=["exact_kv", "rows_dense", "off_reweight_extra"])
+def test_backward_matches_finite_differences(params):
+    """Directional derivatives of the numpy forward (central differences, the
+    selection unchanged at both points) equal <grad, direction>."""
+    from oracle import vsa_backward_oracle as BO
+    wl, lay, q, k, v, g, dout = _bwd_case()
+    grads = BO.vsa_backward_head(q, k, v, g, dout, lay, params)
+    rng = np.random.default_rng(5)
+    base = (q, k, v, g)
+    sel0 = O.selection_for_head(q, k, v, lay, params)[4]
+    eps = 1e-5
+    for which in range(4):
+        u = rng.standard_normal(base[which].shape)
+        xs_p = list(base)
+        xs_m = list(base)
+        xs_p[which] = base[which] + eps * u
+        xs_m[which] = base[which] - eps * u
+        for xs in (xs_p, xs_m):
+            sel = O.selection_for_head(xs[0], xs[1], xs[2], lay, params)[4]
+            assert all(np.array_equal(a, b) for a, b in zip(sel, sel0))
+        lp = float((O.vsa_forward_head(*xs_p, lay, params).out * dout).sum())
+        lm = float((O.vsa_forward_head(*xs_m, lay, params).out * dout).sum())
+        fd = (lp - lm) / (2 * eps)
+        an = float((grads[which] * u).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (which, fd, an)
+
+
+def test_backward_keep_all_gate_zero_is_textbook_attention_backward():
+    """keep = 100% and g = 0: the gradients of dense attention in closed form
+    (dV = P^T dO, dS = P * (dP - rowsum(dP * P)), dQ = c dS K, dK = c dS^T Q)."""
+    from oracle import vsa_backward_oracle as BO
+    wl, lay, q, k, v, g, dout = _bwd_case(keep=1.0)
+    dq, dk, dv, dg = BO.vsa_backward_head(q, k, v, np.zeros_like(g), dout, lay, O.Params(keep=1.0))
+    c = O.default_scale()
+    s = c * q @ k.T
+    P = np.exp(s - s.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    dP = dout @ v.T
+    dS = P * (dP - (dP * P).sum(1, keepdims=True))
+    assert np.allclose(dv, P.T @ dout, atol=1e-10)
+    assert np.allclose(dq, c * dS @ k, atol=1e-10)
+    assert np.allclose(dk, c * dS.T @ q, atol=1e-10)
+    # dg = <dout, o_coarse[tile]> row by row
+    res = O.vsa_forward_head(q, k, v, np.zeros_like(g), lay, O.Params(keep=1.0))
+    assert np.allclose(dg, (dout * res.o_coarse[lay.inv // O.TILE]).sum(1), atol=1e-10)
