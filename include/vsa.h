@@ -192,7 +192,8 @@ void vsa_layout_free(vsa_layout* layout);
 /* Coarse branch + selection                                                 */
 /* ------------------------------------------------------------------------ */
 
-/* kmax: the row length of the index list (k for TOPK, Nv for ADAPTIVE). */
+/* kmax: the row length of the index list (k for TOPK, Nc for ADAPTIVE; Nc =
+ * number of candidate key tiles of the sink mode). */
 vsa_status vsa_select_kmax(const vsa_layout* layout, const vsa_params* params, int32_t* kmax);
 
 vsa_status vsa_coarse_select_workspace_size(const vsa_layout* layout, int32_t B, int32_t H,
@@ -207,12 +208,15 @@ vsa_status vsa_coarse_select_workspace_size(const vsa_layout* layout, int32_t B,
  *                   stride_s, stride_h); 16-byte aligned, strides multiples
  *                   of 8.
  *  idx            : int32 [B, H, n_tiles, kmax] out: per query tile the
- *                   selected video tiles as video ordinals in [0, Nv),
- *                   ascending; entries past cnt are left unspecified.
+ *                   selected candidate key tiles as candidate ordinals in
+ *                   [0, Nc) (see vsa_sink_mode), ascending; entries past cnt
+ *                   are left unspecified.
  *  cnt            : int32 [B, H, n_tiles] out: list lengths.
- *  o_coarse       : float [B, H, n_tiles, 128] out:
- *                   sum_v softmax_v(s[qt, v]) * mean(V of video tile v), with
- *                   s[qt, v] = scale * <mean Q of tile qt, mean K of video tile v>.
+ *  o_coarse       : float [B, H, n_tiles, 128] out, with COARSE_MEAN:
+ *                   sum_c softmax_c(s[qt, c]) * mean(V of candidate tile c),
+ *                   s[qt, c] = scale * <mean Q of tile qt, mean K of tile c>
+ *                   (the scores the selection uses); with COARSE_REWEIGHT the
+ *                   Spark-Reweight form of vsa_coarse_mode.
  *  workspace      : device scratch of vsa_coarse_select_workspace_size bytes,
  *                   256-byte aligned. Its first 3*B*H*n_tiles*128 floats hold
  *                   the pooled means [3 (q,k,v), B, H, n_tiles, 128] after
