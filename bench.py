@@ -44,19 +44,30 @@ def captured_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary of this
     workload, or None when there is none or the kernel sources changed since
     the counters were taken (the summary records their sha256 prefix)."""
-    import hashlib
     import re
     path = os.path.join(ROOT, "profiles", "vsa_attn_kernel_%s_dram.md" % workload)
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    src = b"".join(open(os.path.join(ROOT, "block_sparse_video_geometry_b200", "csrc", f), "rb").read()
-                   for f in ("vsa_attn.cu", "sm100.cuh"))
     m = re.search(r"sha256 prefix: ([0-9a-f]{16})", text)
     t = re.search(r"traffic per launch \(read \+ write\) \| ([0-9,]+) B", text)
-    if not m or not t or m.group(1) != hashlib.sha256(src).hexdigest()[:16]:
+    if not m or not t or m.group(1) != kernel_code_hash():
         return None
     return int(t.group(1).replace(",", ""))
+
+
+def kernel_code_hash() -> str:
+    """sha256 prefix of the attention kernel's code (vsa_attn.cu + sm100.cuh)
+    with comments and whitespace removed, so that comment edits keep a capture."""
+    import hashlib
+    import re
+    code = ""
+    for f in ("vsa_attn.cu", "sm100.cuh"):
+        text = open(os.path.join(ROOT, "block_sparse_video_geometry_b200", "csrc", f)).read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        code += " ".join(text.split()) + "\n"
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def valid_flop_fast(counts, n_cond, idx, cnt, sink_rows, sink_off=False):

@@ -21,18 +21,21 @@
 //    every item's key-tile sequence as records, so that the copy warps only
 //    stream records (a copy warp shares its scheduler with a softmax warp, and
 //    every instruction it needs per step delays the copies).
-//  * Two CTAs per SM, each with 256 TMEM columns: O (128) and two 64-column
-//    score buffers, all M = 64 accumulators (rows in the first 16 lanes of each
-//    lane quadrant); P of a step is written as bf16 pairs over the first 32
-//    columns of its own score buffer and is the TMEM operand of O += P V. Q and
-//    two K and two V stages sit in shared memory.
+//  * Two CTAs per SM, each with 256 TMEM columns used in both 16-lane halves of
+//    every lane quadrant (an M = 64 operand or accumulator takes 16 lanes of
+//    each quadrant): even steps run in lanes 0-15, odd steps in lanes 16-31,
+//    each half with a copy of Q (the A operand of S = Q K^T), its own O and its
+//    own 64-column score buffer, which P of the step overwrites as bf16 pairs
+//    (the A operand of O += P V). An MMA with A in TMEM needs A and D in the
+//    same lanes, which each half keeps; the output is O(half 0) + O(half 1).
+//    Two K and two V stages sit in shared memory.
 //  * One warp issues every MMA, in the order ..., O += P(j - 1) V, S(j + 1),
 //    O += P(j) V, S(j + 2), ...; MMAs from one thread run in issue order, so
 //    S(j + 2) cannot overwrite P(j) early, and no issue waits for a completion.
 //    A K (V) stage is free again once S (O += P V) of its previous step has
 //    completed.
 //  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues the
-//    MMAs; 3-6 load each item's Q into shared memory, run the fp32 online
+//    MMAs; 3-6 write each item's Q into both TMEM halves, run the fp32 online
 //    softmax and the epilogue: two threads per row (the 16x32bx2 TMEM shape
 //    gives the two half-warps the same 16 lanes at two column offsets), 32 keys
 //    each per step, exp2. P is computed against the running max; the exact row
