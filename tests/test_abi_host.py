@@ -172,3 +172,22 @@ def test_calls_validate_before_any_gpu_work():
                                  ws - 16, None) == vsa.ERR_WORKSPACE_TOO_SMALL
     assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
                                  ws, None) == vsa.ERR_NOT_UPLOADED
+
+
+def test_layout_matches_oracle_on_random_descriptors():
+    """Random segment layouts (conditioning before and after the video, ragged
+    grids, one-token segments): the library's tables equal the oracle's."""
+    rng = np.random.default_rng(2024)
+    for _ in range(60):
+        before = [(int(rng.integers(0, 4)), int(rng.integers(1, 200))) for _ in range(int(rng.integers(0, 4)))]
+        after = [(int(rng.integers(0, 4)), int(rng.integers(1, 150))) for _ in range(int(rng.integers(0, 2)))]
+        grid = tuple(int(x) for x in rng.integers(1, 14, size=3))
+        segs, S = _segments(before, grid, after)
+        lay = vsa.Layout(segs, S)
+        ref = O.build_layout([O.Segment(k, s, n, g) for (k, s, n, g) in segs], S)
+        perm, inv, cnt, kind = lay.tables()
+        assert np.array_equal(perm, ref.perm) and np.array_equal(inv, ref.inv)
+        assert np.array_equal(cnt, (ref.perm >= 0).sum(1)) and np.array_equal(kind, ref.tile_kind)
+        # every token sits in exactly one slot
+        flat = perm[perm >= 0]
+        assert np.array_equal(np.sort(flat), np.arange(S))
