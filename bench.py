@@ -41,19 +41,19 @@ COARSES = {"mean": 0, "reweight": 1}
 
 
 def captured_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary of this
-    workload, or None when there is none or the kernel sources changed since
-    the counters were taken (the summary records their sha256 prefix)."""
-    import re
-    path = os.path.join(ROOT, "profiles", "vsa_attn_kernel_%s_dram.md" % workload)
-    if not os.path.exists(path):
+    """DRAM bytes per attention launch from the committed counter capture of
+    this workload (profiles/vsa_attn_kernel_<workload>_dram.json), or None when
+    there is none or the kernel code changed since the counters were taken
+    (the capture records the code hash of kernel_code_hash())."""
+    path = os.path.join(ROOT, "profiles", "vsa_attn_kernel_%s_dram.json" % workload)
+    try:
+        with open(path) as f:
+            cap = json.load(f)
+    except (OSError, ValueError):
         return None
-    text = open(path).read()
-    m = re.search(r"sha256 prefix: ([0-9a-f]{16})", text)
-    t = re.search(r"traffic per launch \(read \+ write\) \| ([0-9,]+) B", text)
-    if not m or not t or m.group(1) != kernel_code_hash():
+    if cap.get("kernel_code_sha256_16") != kernel_code_hash():
         return None
-    return int(t.group(1).replace(",", ""))
+    return int(cap["dram_bytes_read"]) + int(cap["dram_bytes_write"])
 
 
 def kernel_code_hash() -> str:
@@ -237,6 +237,97 @@ def run_reference(args):
 
 
 # -------------------------------------------------------------- GPU arm
+def time_calls(stream, select_fn, attn_fn, n):
+    """Median ms of the selection call and of the attention call over n calls
+    (CUDA events on the launching stream), plus the sorted whole-call times."""
+    import torch
+    sel, att = [], []
+    for _ in range(n):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        select_fn()
+        e[1].record(stream)
+        attn_fn()
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        sel.append(e[0].elapsed_time(e[1]))
+        att.append(e[1].elapsed_time(e[2]))
+    calls = sorted(a + b for a, b in zip(sel, att))
+    return statistics.median(sel), statistics.median(att), calls
+
+
+def dense_sdpa_ms(stream, q, k, v, n=3):
+    """torch scaled_dot_product_attention on the same Q, K, V (a library kernel,
+    timed for context: the method replaces it); None if it cannot run."""
+    import torch
+    try:
+        qd, kd, vd = (x.transpose(1, 2) for x in (q, k, v))      # [B, H, S, 128] views
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+            d_ms = []
+            for _ in range(n):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                d_ms.append(e0.elapsed_time(e1))
+        return statistics.median(d_ms)
+    except RuntimeError as ex:   # e.g. out of memory on a smaller GPU
+        print("dense comparator skipped: %s" % ex, file=sys.stderr)
+        return None
+    finally:
+        torch.cuda.empty_cache()
+
+
+def check_failures(fwd, stream, where):
+    from block_sparse_video_geometry_b200 import vsa
+    n = vsa.sparse_attn_failed_calls(fwd.ws_attn, stream)
+    if n:
+        raise RuntimeError("%s: %d attention call(s) reported a kernel error" % (where, n))
+
+
+def measure_config(name, wl, params, q, k, v, g, dev, stream, out_dtype, peak, n_calls, dense=None,
+                   inputs_note=None):
+    """One extra workload of the same run: ms per call (selection + attention),
+    valid TFLOP/s, the attention kernel's fraction of the burst bf16 peak, the
+    kept fraction of candidate tiles, and the dense comparator where given."""
+    import torch
+    from block_sparse_video_geometry_b200 import vsa
+    lay = vsa.Layout(wl.segments(), wl.seq_len)
+    perm, inv, counts, kinds = lay.tables()
+    with torch.cuda.stream(stream):
+        fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, out_dtype=out_dtype, stream=stream)
+        out = torch.empty(q.shape, dtype=out_dtype, device=dev)
+    sel_fn = lambda: vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
+    att_fn = lambda: vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
+                                         fwd.ws_attn, stream)
+    for _ in range(3):
+        sel_fn()
+        att_fn()
+    torch.cuda.synchronize()
+    idx, cnt = fwd.idx.cpu().numpy(), fwd.cnt.cpu().numpy()
+    flop = valid_flop_fast(counts, lay.info.n_cond_tiles, idx, cnt, wl.sink == vsa.SINK_EXACT_KV_AND_ROWS,
+                           wl.sink == vsa.SINK_OFF)
+    sel_ms, att_ms, calls = time_calls(stream, sel_fn, att_fn, n_calls)
+    check_failures(fwd, stream, name)
+    call_ms = statistics.median(calls)
+    n_cand = lay.info.n_tiles if wl.sink == vsa.SINK_OFF else lay.info.n_video_tiles
+    res = {"workload": describe(wl), "ms_per_call": call_ms, "select_ms": sel_ms, "attn_ms": att_ms,
+           "valid_tflop": flop / 1e12, "tflops_per_call": flop / (call_ms * 1e-3) / 1e12,
+           "attn_tflops": flop / (att_ms * 1e-3) / 1e12, "attn_frac_of_burst": flop / (att_ms * 1e-3) / 1e12 / peak,
+           "kept_fraction": float(cnt.mean()) / n_cand, "calls": n_calls}
+    if inputs_note:
+        res["inputs"] = inputs_note
+    if dense is not None:
+        res["dense_sdpa_ms"] = dense
+        res["speedup_vs_dense"] = dense / call_ms
+    del fwd, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     from block_sparse_video_geometry_b200 import vsa, workloads as W
@@ -270,17 +361,23 @@ def run_ours(args):
         fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, out_dtype=out_dtype, stream=stream)
         out = torch.empty(q.shape, dtype=out_dtype, device=dev)
     torch.cuda.synchronize()
+    peaks, src = measured_peaks()
+    peak = peaks["bf16_tflops"]
 
-    def step():
+    def select():
         vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
+
+    def attend():
         vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
                             fwd.ws_attn, stream)
 
+    def step():
+        select()
+        attend()
+
     for _ in range(args.warmup):
         step()
-    st = vsa.sparse_attn_status(fwd.ws_attn, stream)
-    if st != vsa.OK:
-        raise RuntimeError("kernel status %s" % vsa.status_string(st))
+    check_failures(fwd, stream, "warm-up")
     flop = valid_flop_fast(counts, lay.info.n_cond_tiles, fwd.idx.cpu().numpy(), fwd.cnt.cpu().numpy(),
                            wl.sink == vsa.SINK_EXACT_KV_AND_ROWS, wl.sink == vsa.SINK_OFF)
 
@@ -299,47 +396,15 @@ def run_ours(args):
         ev1.record(stream)
         barrier()
     ms_step = ev0.elapsed_time(ev1) / args.steps
+    check_failures(fwd, stream, "timed steps")
 
     # ---- per-kernel split: selection call vs attention call, events on the same stream
-    sel_ms, att_ms = [], []
-    for _ in range(max(3, min(args.steps, 10))):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        e[0].record(stream)
-        vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
-        e[1].record(stream)
-        vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
-                            fwd.ws_attn, stream)
-        e[2].record(stream)
-        torch.cuda.synchronize()
-        sel_ms.append(e[0].elapsed_time(e[1]))
-        att_ms.append(e[1].elapsed_time(e[2]))
-    call_ms = sorted(a_ + s_ for a_, s_ in zip(att_ms, sel_ms))
+    sel_ms, att_ms, call_ms = time_calls(stream, select, attend, max(3, min(args.steps, 10)))
+    check_failures(fwd, stream, "per-call timing")
     call_p50 = statistics.median(call_ms)
     call_p90 = call_ms[min(len(call_ms) - 1, int(round(0.9 * (len(call_ms) - 1))))]
-    sel_ms, att_ms = statistics.median(sel_ms), statistics.median(att_ms)
 
-    # ---- dense comparator: torch scaled_dot_product_attention on the same Q, K, V (a library
-    # kernel, timed for context; the method replaces it)
-    dense_ms = None
-    if not args.no_dense:
-        try:
-            qd, kd, vd = (x.transpose(1, 2) for x in (q, k, v))      # [B, H, S, 128] views
-            with torch.cuda.stream(stream):
-                for _ in range(2):
-                    torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
-                d_ms = []
-                for _ in range(3):
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
-                    e1.record(stream)
-                    torch.cuda.synchronize()
-                    d_ms.append(e0.elapsed_time(e1))
-            dense_ms = statistics.median(d_ms)
-        except RuntimeError as ex:   # e.g. out of memory on a smaller GPU
-            dense_ms = None
-            print("dense comparator skipped: %s" % ex, file=sys.stderr)
-        torch.cuda.empty_cache()
+    dense_ms = None if args.no_dense else dense_sdpa_ms(stream, q, k, v)
 
     # ---- end to end through the public API with host buffers. Every step copies its inputs host ->
     # device and reads its output back inside the timed region; the copies overlap the neighbouring
@@ -382,23 +447,49 @@ def run_ours(args):
     e2e_end.record(s_out)
     barrier()
     ms_e2e = e2e_start.elapsed_time(e2e_end) / e2e_steps
-    st = vsa.sparse_attn_status(fwd.ws_attn, stream)
-    if st != vsa.OK:
-        raise RuntimeError("kernel status %s" % vsa.status_string(st))
-    del dev_in, dev_out
+    check_failures(fwd, stream, "end-to-end steps")
+    del dev_in, dev_out, host_in, host_out
+
+    # ---- the other configurations of the same shapes, measured in the same run (rank 0, one GPU)
+    configs = None
+    if world == 1 and not args.no_configs and args.workload == "5s" and args.sink is None \
+            and args.coarse == "mean" and args.gate == "token":
+        configs = {}
+        n = args.config_calls
+        mk = lambda **kw: vsa.make_params(**dict(dict(mode=0, keep=0.1, tau=1.0, sink=0, coarse=0), **kw))
+        note = "the 5 s inputs of this run (seed %d)" % wl.seed
+        for tau in (1.0, 1.5, 2.0):
+            configs["5s_adaptive_tau%g" % tau] = measure_config(
+                "adaptive tau %g" % tau, wl.with_(mode=vsa.SELECT_ADAPTIVE, tau=tau),
+                mk(mode=vsa.SELECT_ADAPTIVE, tau=tau), q, k, v, g, dev, stream, out_dtype, peak, n,
+                inputs_note=note)
+        configs["5s_keep100"] = measure_config("keep 100%", wl.with_(keep=1.0), mk(keep=1.0), q, k, v, g, dev,
+                                               stream, out_dtype, peak, max(3, n // 2), dense=dense_ms,
+                                               inputs_note=note)
+        del q, k, v, g, out
+        fwd = None
+        torch.cuda.empty_cache()
+        w10 = W.WORKLOADS["10s"]
+        lay10 = vsa.Layout(w10.segments(), w10.seq_len)
+        b10 = W.make_inputs(w10, lay10.tables()[1] // vsa.TILE)
+        q10, k10, v10, g10 = (to_dev(x) for x in b10)
+        del b10
+        d10 = None if args.no_dense else dense_sdpa_ms(stream, q10, k10, v10, n=2)
+        configs["10s_ragged_rows_dense"] = measure_config(
+            "10 s", w10, mk(sink=vsa.SINK_EXACT_KV_AND_ROWS), q10, k10, v10, g10, dev, stream, out_dtype, peak,
+            max(3, n // 2), dense=d10)
+        del q10, k10, v10, g10
+        torch.cuda.empty_cache()
 
     ms_step, ms_e2e, att_ms, sel_ms = sharding.max_over_ranks([ms_step, ms_e2e, att_ms, sel_ms], dist, dev)
     job_flop, = sharding.sum_over_ranks([flop], dist, dev)   # the work of every replica
 
     if rank == 0:
-        peaks, src = measured_peaks()
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         achieved = flop / (att_ms * 1e-3) / 1e12
         info = lay.info
-        ld = (info.n_video_tiles + 63) // 64 * 64
-        sel_bytes = (3 * q.numel() * 2                                           # Q, K, V read once
-                     + 2 * wl.B * wl.H * info.n_tiles * ld * 4                    # scores written + read
-                     + 4 * wl.B * wl.H * info.n_tiles * (fwd.kmax + 1 + 128))    # idx, cnt, o_coarse
+        # algorithmic bytes of the selection call: Q, K, V read once, idx, cnt and o_coarse written
+        sel_bytes = 3 * wl.B * wl.seq_len * wl.H * 128 * 2 + 4 * wl.B * wl.H * info.n_tiles * (
+            lay.kmax(params) + 1 + 128)
         value = job_flop / (ms_step * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -412,8 +503,8 @@ def run_ours(args):
                          "traffic": (captured_traffic(args.workload) if args.sink is None and args.coarse == "mean"
                                      and args.gate == "token" and args.out_dtype == "f32" else None),
                          "traffic_unit": "bytes per launch (ncu dram read + write)",
-                         "peak_source": "%s bf16_tflops_sustained" % src,
-                         "frac_of_burst": achieved / peaks["bf16_tflops"],
+                         "peak_source": "%s bf16_tflops (burst: the kernel is timed alone, once per call)" % src,
+                         "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
                          "flop_per_launch": flop, "ms_per_launch": att_ms},
             "selection": {"bound": "hbm", "achieved": sel_bytes / (sel_ms * 1e-3) / 1e9,
                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -422,14 +513,15 @@ def run_ours(args):
             "e2e": {"value": job_flop / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                     "steps": e2e_steps, "copies": "overlap the neighbouring steps' compute"},
-            # per step and rank: pool, coarse, select; permute, schedule, one attention launch per batch
-            "gpu_launches": (5 + wl.B) * args.steps * world,
+            "gpu_launches": launches_per_call(wl.B, args.coarse) * args.steps * world,
             "clocks": clocks.summary(),
             "call_ms": {"p50": call_p50, "p90": call_p90, "samples": len(call_ms)},
             "dense_sdpa": None if dense_ms is None else {
                 "ms": dense_ms, "call_speedup": dense_ms / call_p50,
                 "what": "torch scaled_dot_product_attention, bf16, same Q, K, V, no mask"},
         }
+        if configs:
+            line["configs"] = configs
         if world == 1 and not args.no_cpu_baseline:
             from oracle import vsa_oracle as O
             olay = O.build_layout([O.Segment(k_, s_, n_, g_) for (k_, s_, n_, g_) in wl.segments()], wl.seq_len)
@@ -442,6 +534,13 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
+
+
+def launches_per_call(B: int, coarse: str) -> int:
+    """Kernels this library launches per call: selection (pool, coarse, select;
+    anchor and reweight with Spark-Reweight) and attention (permute, schedule,
+    one attention launch per batch)."""
+    return 3 + (2 if coarse == "reweight" else 0) + 2 + B
 
 
 def main():
@@ -461,6 +560,9 @@ def main():
     ap.add_argument("--ref-tiles", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the torch SDPA comparator")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations (5 s adaptive tau, keep 100%%, 10 s ragged)")
+    ap.add_argument("--config-calls", type=int, default=10, help="timed calls per extra configuration")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

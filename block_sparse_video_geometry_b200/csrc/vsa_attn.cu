@@ -203,8 +203,15 @@ __device__ __forceinline__ int64_t tile_token(const AttnSmem& sm, const Geom& G,
   return G.video_start + (static_cast<int64_t>(t) * G.Hg + h) * G.W + w;
 }
 
+// err[0]: status of the current call (cleared by each call); err[1]: failed
+// calls since the caller last ran vsa_sparse_attn_workspace_init (the first
+// block of a call to record an error counts the call).
+__device__ __forceinline__ void record_error(int* err, int status) {
+  if (atomicExch(err, status) == 0) atomicAdd(err + 1, 1);
+}
+
 __device__ __forceinline__ void raise_abort(AttnSmem& sm, int* err) {
-  atomicExch(err, VSA_ERR_TIMEOUT);
+  record_error(err, VSA_ERR_TIMEOUT);
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
@@ -306,7 +313,7 @@ template <bool kChannelGate>
 __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {          // swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
+    if (threadIdx.x == 0) record_error(a.err, VSA_ERR_UNSUPPORTED);
     return;
   }
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
@@ -834,7 +841,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
-  e = cudaMemsetAsync(workspace, 0, kAttnHeader, stream);
+  e = cudaMemsetAsync(workspace, 0, sizeof(int), stream);   // this call's status word only
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaMemsetAsync", e);
   const int grid = std::max(1, std::min(a.n_items, 2 * n_sm));   // two CTAs per SM, 256 TMEM columns each
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
@@ -861,6 +868,22 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
 
 vsa_status vsa_debug_inject_wait_timeout(uint64_t timeout_ns) {
   g_stall_ns.store(timeout_ns, std::memory_order_relaxed);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_workspace_init(void* workspace, cudaStream_t stream) {
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kAttnHeader, stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_workspace_init: cudaMemsetAsync", e);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_failed_calls(const void* workspace, cudaStream_t stream, uint32_t* count) {
+  if (!workspace || !count) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_failed_calls: cudaStreamSynchronize", e);
+  e = cudaMemcpy(count, static_cast<const int*>(workspace) + 1, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_failed_calls: cudaMemcpy", e);
   return VSA_OK;
 }
 

@@ -72,6 +72,8 @@ _SIGNATURES = {
                                    _P, _I64, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64,
                                    _I64, _P, _SZ, _P]),
     "vsa_sparse_attn_status": (_I32, [_P, _P]),
+    "vsa_sparse_attn_workspace_init": (_I32, [_P, _P]),
+    "vsa_sparse_attn_failed_calls": (_I32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "vsa_debug_inject_wait_timeout": (_I32, [ctypes.c_uint64]),
     "vsa_status_string": (ctypes.c_char_p, [_I32]),
     "vsa_version": (_I32, []),
@@ -246,6 +248,20 @@ def sparse_attn_status(workspace, stream=None) -> int:
     return lib().vsa_sparse_attn_status(workspace.data_ptr(), _stream_handle(stream))
 
 
+def sparse_attn_workspace_init(workspace, stream=None) -> None:
+    """Zeroes the attention workspace header (and its count of failed calls)."""
+    _check(lib().vsa_sparse_attn_workspace_init(workspace.data_ptr(), _stream_handle(stream)),
+           "vsa_sparse_attn_workspace_init")
+
+
+def sparse_attn_failed_calls(workspace, stream=None) -> int:
+    """Synchronises the stream; number of calls that recorded an error since the header was zeroed."""
+    n = ctypes.c_uint32()
+    _check(lib().vsa_sparse_attn_failed_calls(workspace.data_ptr(), _stream_handle(stream), ctypes.byref(n)),
+           "vsa_sparse_attn_failed_calls")
+    return n.value
+
+
 def debug_inject_wait_timeout(timeout_ns):
     """Test hook: while timeout_ns > 0, each sparse_attn_fwd runs into a bounded
     wait that nothing completes and reports ERR_TIMEOUT (see vsa.h); 0 disarms."""
@@ -272,6 +288,7 @@ class Forward:
                                      device=device)
         self.ws_attn = torch.empty(layout.sparse_attn_workspace_size(B, H, params), dtype=torch.uint8,
                                    device=device)
+        sparse_attn_workspace_init(self.ws_attn, stream)
         self.out_dtype = out_dtype or torch.float32
         self.stream = stream
 

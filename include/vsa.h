@@ -286,12 +286,15 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* layout, int32_t B, i
  *  out              : [B, S, H, 128] of out_dtype (vsa_out_dtype) at element
  *                     strides out_stride_*, head_dim contiguous; every valid
  *                     token row is written.
- *  workspace        : vsa_sparse_attn_workspace_size bytes, 256-byte aligned,
- *                     all written by the call before use: an error word; a
- *                     tile-major copy of K and V (32 KB per (batch, head,
- *                     tile); 1.64 GB for the 24-head 133,696-token shape); the
- *                     key-tile schedule of every pair of query tiles (8 bytes
- *                     per key tile; about 0.1 GB for that shape).
+ *  workspace        : vsa_sparse_attn_workspace_size bytes, 256-byte aligned.
+ *                     A 256-byte header holds this call's status word
+ *                     (cleared by the call) and a count of failed calls
+ *                     (see vsa_sparse_attn_workspace_init); the rest is
+ *                     written by the call before use: a tile-major copy of K
+ *                     and V (32 KB per (batch, head, tile); 1.64 GB for the
+ *                     24-head 133,696-token shape) and the key-tile schedule
+ *                     of every query tile (8 bytes per key tile; about 0.1 GB
+ *                     for that shape).
  * Softmax statistics and accumulation are fp32; the probabilities enter the
  * second tensor-core product as bf16. A kernel wait that runs out is recorded
  * in the workspace and reported by vsa_sparse_attn_status. */
@@ -306,6 +309,18 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* layout, const vsa_params* param
                                void* out, int32_t out_dtype, int64_t out_stride_b,
                                int64_t out_stride_s, int64_t out_stride_h,
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Zeroes the workspace header, including the count of failed calls that
+ * vsa_sparse_attn_failed_calls reads (enqueued on `stream`). Call it once
+ * after allocating a workspace; the count is meaningless until then. No
+ * counterpart on the pages (error reporting of this library). */
+vsa_status vsa_sparse_attn_workspace_init(void* workspace, cudaStream_t stream);
+
+/* Synchronises `stream` and reads, into *count, how many vsa_sparse_attn_fwd
+ * calls on this workspace recorded an error (a bounded wait that ran out)
+ * since vsa_sparse_attn_workspace_init. Unlike vsa_sparse_attn_status it sees
+ * a failure of any earlier call, not only the latest one. */
+vsa_status vsa_sparse_attn_failed_calls(const void* workspace, cudaStream_t stream, uint32_t* count);
 
 /* Synchronises `stream` and reads the error word a previous
  * vsa_sparse_attn_fwd left in `workspace`: VSA_OK, VSA_ERR_TIMEOUT (a bounded

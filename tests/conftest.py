@@ -19,3 +19,12 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_terminal_summary(terminalreporter):
+    try:
+        import vsa_cases
+    except ImportError:
+        return
+    n = vsa_cases.NEAR_TIE_ROWS[0]
+    terminalreporter.write_line("near-tie query tiles checked on the GPU's own list: %d" % n)

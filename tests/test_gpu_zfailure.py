@@ -37,9 +37,12 @@ def test_injected_wait_timeout_is_reported_and_recoverable(cuda_ok):
         vsa.debug_inject_wait_timeout(0)
     assert st == vsa.ERR_TIMEOUT
     assert elapsed < 5.0
-    # the context is still usable and the next call is correct
+    assert vsa.sparse_attn_failed_calls(fwd.ws_attn) == 1
+    # the context is still usable and the next call is correct; the failure
+    # stays counted after a good call overwrote the per-call status
     out = fwd(q, k, v, g)
     assert vsa.sparse_attn_status(fwd.ws_attn) == vsa.OK
+    assert vsa.sparse_attn_failed_calls(fwd.ws_attn) == 1
     assert torch.isfinite(out).all()
 
 

@@ -5,8 +5,10 @@ comparison rules.
 Tolerances (stated here once, used by every parity test):
 * layout and selected tile indices: bit-exact, except rows whose oracle
   scores have a near-tie (gap < 1e-4) at the selection boundary; in such a
-  row the two sets may differ only by tiles within 1e-4 of the boundary, and
-  the row's outputs are left out of the comparison;
+  row the two sets may differ only by tiles within 1e-4 of the boundary (and
+  top-k lists keep their length). Both sets are then valid results of the
+  method, so the row's outputs are compared with the oracle's fine branch
+  evaluated on the GPU's own list: no query tile is left out;
 * fp32 output: max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle;
 * bf16 output: the same bounds plus the bf16 rounding of the output itself
   (half an ulp of the reference value per element, a quarter ulp on average);
@@ -22,6 +24,14 @@ from oracle import vsa_oracle as O
 
 GAP = 1e-4
 OUT_MAX_ABS, OUT_MEAN_ABS = 2e-2, 2e-3
+
+# rows whose GPU list differed from the oracle's at a near-tie (and were
+# checked on the GPU's list); the session summary prints the total
+NEAR_TIE_ROWS = [0]
+
+
+def note_near_ties(n: int) -> None:
+    NEAR_TIE_ROWS[0] += int(n)
 
 
 def oracle_layout(wl):
@@ -80,34 +90,42 @@ class HeadOracle:
         (self.qbar, self.kbar, self.vbar, self.scores, self.sel, self.thr, self.o_coarse,
          self.scale) = O.selection_for_head(self.q, self.k, self.v, lay, self.p)
 
-    def tile_out(self, qt):
+    def tile_out(self, qt, selected=None):
+        """Oracle rows of query tile qt; `selected` replaces the oracle's own
+        list (a near-tie row is checked on the list the GPU chose)."""
+        sel = self.sel[qt] if selected is None else np.asarray(selected, dtype=np.int64)
         return O.output_rows_for_tile(self.q, self.k, self.v, self.g, self.lay, self.p, qt,
-                                      self.sel[qt], self.o_coarse, self.scale)
+                                      sel, self.o_coarse, self.scale)
 
 
 def check_lists_valid(res, lay, sink=O.SINK_EXACT_KV):
-    """Every list is ascending, in range (candidate ordinals) and as long as cnt says."""
+    """Every list of every (batch, head, query tile) is strictly ascending, in
+    range (candidate ordinals) and 1 <= cnt <= kmax."""
     idx, cnt = res["idx"], res["cnt"]
     nv = O.candidate_tiles(lay, sink)[1]
     assert cnt.min() >= 1 and cnt.max() <= res["kmax"]
-    B, H, Nt, _ = idx.shape
-    for b in range(B):
-        for h in range(H):
-            for qt in range(Nt):
-                row = idx[b, h, qt, : cnt[b, h, qt]]
-                assert row.min() >= 0 and row.max() < nv
-                assert np.all(np.diff(row) > 0)
+    live = np.arange(idx.shape[-1])[None, None, None, :] < cnt[..., None]
+    assert np.all(np.where(live, idx, 0) >= 0) and np.all(np.where(live, idx, 0) < nv)
+    both = live[..., 1:]
+    assert np.all(np.where(both, idx[..., 1:] > idx[..., :-1], True))
 
 
 def compare_selection(ho: HeadOracle, gpu_idx, gpu_cnt):
-    """Returns the set of query tiles left out for a near-tie; asserts the rest."""
-    excluded = set()
+    """Checks the GPU's lists of one (batch, head) against the oracle's.
+
+    Returns {query tile: GPU list} for the rows that differ at a near-tie;
+    asserts that every other row is identical. A near-tie row may differ only
+    by tiles whose oracle score lies within GAP of the selection boundary, and
+    under top-k it must keep the oracle's length k."""
+    near_tie = {}
     for qt, want in enumerate(ho.sel):
         got = gpu_idx[qt, : gpu_cnt[qt]]
         if got.size == want.size and np.array_equal(got, want):
             continue
         row = ho.scores[qt]
         if ho.p.mode == O.MODE_TOPK:
+            assert got.size == want.size, "query tile %d: top-k list of length %d, want %d" % (
+                qt, got.size, want.size)
             srt = np.sort(row)[::-1]
             kk = want.size
             edge = srt[kk - 1]
@@ -117,8 +135,8 @@ def compare_selection(ho: HeadOracle, gpu_idx, gpu_cnt):
             edge = ho.thr
         diff = np.setxor1d(got, want)
         assert np.all(np.abs(row[diff] - edge) < GAP), "query tile %d: differs away from the boundary" % qt
-        excluded.add(qt)
-    return excluded
+        near_tie[qt] = got.copy()
+    return near_tie
 
 
 def out_error(got, want, bf16: bool):
@@ -130,11 +148,14 @@ def out_error(got, want, bf16: bool):
     return float((err - half_ulp).max()), float(err.mean()), OUT_MEAN_ABS + float((half_ulp / 2).mean())
 
 
-def compare_outputs(ho: HeadOracle, res, b, h, tiles, bf16=False):
-    """Compares the GPU output rows of the given query tiles with the oracle."""
+def compare_outputs(ho: HeadOracle, res, b, h, tiles, bf16=False, near_tie=None):
+    """Compares the GPU output rows of the given query tiles with the oracle.
+    Rows in `near_tie` (from compare_selection) are compared with the oracle
+    evaluated on the GPU's list for that tile."""
+    near_tie = near_tie or {}
     errs, means, bounds = [], [], []
     for qt in tiles:
-        toks, of, want = ho.tile_out(qt)
+        toks, of, want = ho.tile_out(qt, near_tie.get(qt))
         got = res["out"][b, toks, h]
         mx, mean, bound = out_error(got, want, bf16)
         errs.append(mx)
