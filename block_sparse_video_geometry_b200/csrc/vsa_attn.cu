@@ -7,41 +7,45 @@
 // Sparse Attention"); with exact_kv_and_rows the conditioning query tiles
 // attend the whole sequence. The epilogue writes o_fine + g * o_coarse.
 //
-// Design (B200):
-//  * Work item = one 64-token query tile of one (batch, head), computed with
-//    M = 64 tcgen05 MMAs; its key tiles are the dense part (all conditioning
-//    tiles, or all tiles for dense conditioning rows) followed by its own
-//    selection list. (Stacking two query tiles into one M = 128 tile needs the
-//    union of their lists; the selections of neighbouring tiles barely overlap,
-//    so most of that work would be masked.)
-//  * permute_kv_kernel first rewrites K and V tile-major into the workspace,
-//    each 64-token tile of each head one contiguous 16 KB block already in the
-//    128-byte-swizzled layout of the UMMA descriptors, padding slots zero, so
-//    a step's K or V tile arrives with one bulk copy. schedule_kernel writes
-//    every item's key-tile sequence as records, so that the copy warps only
-//    stream records (a copy warp shares its scheduler with a softmax warp, and
-//    every instruction it needs per step delays the copies).
-//  * Two CTAs per SM, each with 256 TMEM columns used in both 16-lane halves of
-//    every lane quadrant (an M = 64 operand or accumulator takes 16 lanes of
-//    each quadrant): even steps run in lanes 0-15, odd steps in lanes 16-31,
-//    each half with a copy of Q (the A operand of S = Q K^T), its own O and its
-//    own 64-column score buffer, which P of the step overwrites as bf16 pairs
-//    (the A operand of O += P V). An MMA with A in TMEM needs A and D in the
-//    same lanes, which each half keeps; the output is O(half 0) + O(half 1).
-//    Two K and two V stages sit in shared memory.
-//  * One warp issues every MMA, in the order ..., O += P(j - 1) V, S(j + 1),
-//    O += P(j) V, S(j + 2), ...; MMAs from one thread run in issue order, so
-//    S(j + 2) cannot overwrite P(j) early, and no issue waits for a completion.
-//    A K (V) stage is free again once S (O += P V) of its previous step has
-//    completed.
-//  * Warps: 0 and 1 copy K (and publish per-step tile info) and V; 2 issues the
-//    MMAs; 3-6 write each item's Q into both TMEM halves, run the fp32 online
-//    softmax and the epilogue: two threads per row (the 16x32bx2 TMEM shape
-//    gives the two half-warps the same 16 lanes at two column offsets), 32 keys
-//    each per step, exp2. P is computed against the running max; the exact row
-//    max of a step is only formed when a row's sum of P exceeds 2^8 (then O
-//    and the sum are rescaled and P recomputed), which keeps every P at most
-//    2^8.
+// Design (B200). One call runs four kernels:
+//  * permute_qkv_kernel rewrites K and V (and, for the pair pass, Q)
+//    tile-major into the workspace, each 64-token tile of each head one
+//    contiguous 16 KB block already in the 128-byte-swizzled layout of the UMMA
+//    descriptors, padding slots zero, so that a step's K or V tile arrives with
+//    one bulk copy. schedule_kernel writes every sparse item's key-tile
+//    sequence as records, so that the copy warps only stream records (a copy
+//    warp shares its scheduler with a softmax warp, and every instruction it
+//    needs per step delays the copies).
+//  * The pair pass (pairpass::pair_attn_kernel) runs the key tiles that every
+//    query tile of a head attends: the conditioning prefix, and for dense
+//    conditioning rows the whole sequence. Its work item is a PAIR of query
+//    tiles stacked into one M = 128 MMA (full tensor rate, each key tile copied
+//    once per two query tiles); it leaves the partial output over the
+//    conditioning keys, normalised, with its log-sum-exp (dense rows: the
+//    final output).
+//  * The sparse pass (vsa_attn_kernel) runs each query tile's own selection
+//    list with M = 64 MMAs (the lists of neighbouring query tiles barely
+//    overlap, so stacking them would mostly compute masked work) and merges the
+//    pair pass's partial result in its epilogue, exactly: the softmax over a
+//    union of key sets is the log-sum-exp-weighted combination of the
+//    softmaxes over the parts. Two CTAs per SM, each with 256 TMEM columns used
+//    in both 16-lane halves of every lane quadrant (an M = 64 operand or
+//    accumulator takes 16 lanes of each quadrant): even steps run in lanes
+//    0-15, odd steps in lanes 16-31, each half with a copy of Q (the A operand
+//    of S = Q K^T), its own O and its own 64-column score buffer, which P of the
+//    step overwrites as bf16 pairs (the A operand of O += P V). An MMA with A in
+//    TMEM needs A and D in the same lanes, which each half keeps; the output is
+//    O(half 0) + O(half 1). Two K and two V stages sit in shared memory.
+//  * Sparse pass warps: 0 and 1 copy K (and publish per-step tile info) and V;
+//    2 issues the MMAs in the order ..., O += P(j - 1) V, S(j + 1), O += P(j) V,
+//    S(j + 2), ... (MMAs from one thread run in issue order, so S(j + 2) cannot
+//    overwrite P(j) early, and no issue waits for a completion); 3-6 write each
+//    item's Q into both TMEM halves, run the fp32 online softmax and the
+//    epilogue: two threads per row (the 16x32bx2 TMEM shape gives the two
+//    half-warps the same 16 lanes at two column offsets), 32 keys each per
+//    step, exp2. P is computed against the running max; the exact row max of a
+//    step is only formed when a row's sum of P exceeds 2^8 (then O and the sum
+//    are rescaled and P recomputed), which keeps every P at most 2^8.
 //  * Every wait is bounded: a wait that runs out sets an error word in the
 //    workspace, raises an abort flag that ends the other roles' loops, drains
 //    in-flight copies and MMAs and frees TMEM before the block exits.
@@ -124,16 +128,18 @@ struct AttnArgs {
   const uint16_t* q;         // batch base of Q, element strides q_ss, q_sh
   int64_t q_ss, q_sh;
   int32_t H, b, sink, kmax;
-  int32_t c0;                // first query tile of the sparse item range
-  int32_t n_fixed;           // key tiles every sparse item attends first (conditioning tiles, or none)
+  int32_t c0;                // first query tile of the item range (the rest are dense rows of the pair pass)
   int32_t cand0, n_cand;     // candidate key tiles: tile ids cand0 .. cand0 + n_cand - 1
-  int32_t nq_dense, nq_sparse, n_dense_items, n_items;   // query tiles per head: dense rows, sparse rows
+  int32_t nq, n_items;       // query tiles per head in this pass; items = nq * H
   const int32_t* idx;         // selection lists (read by schedule_kernel)
   const int32_t* cnt;
   const unsigned long long* valid;   // per-tile slot masks
   int2* sched;               // step records: [b][item][max_steps]
   int32_t* nsteps;           // steps per (b, item)
   int32_t max_steps;
+  int32_t merge_prefix;      // merge the pair pass's partial output over the conditioning keys
+  const float* part_o;       // [B, H, n_tiles, 64, 128] normalised partial output
+  const float* part_lse;     // [B, H, n_tiles, 64] its log2-sum-exp2 (scaled log2 domain)
   const float* o_coarse;
   const uint16_t* g;
   int64_t g_sb, g_ss, g_sh, g_sd;   // g_sd = 0: one gate per (token, head)
@@ -147,21 +153,13 @@ struct AttnArgs {
 
 // Work item = one query tile of one (batch, head).
 struct Item {
-  int h, qt, dense;
+  int h, qt;
 };
 
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item) {
   Item it;
-  if (item < a.n_dense_items) {
-    it.h = item / a.nq_dense;
-    it.qt = item % a.nq_dense;
-    it.dense = 1;
-  } else {
-    const int r = item - a.n_dense_items;
-    it.h = r / a.nq_sparse;
-    it.qt = a.c0 + r % a.nq_sparse;
-    it.dense = 0;
-  }
+  it.h = item / a.nq;
+  it.qt = a.c0 + (item - it.h * a.nq);
   return it;
 }
 
@@ -210,14 +208,15 @@ __device__ __forceinline__ void record_error(int* err, int status) {
   if (atomicExch(err, status) == 0) atomicAdd(err + 1, 1);
 }
 
-__device__ __forceinline__ void raise_abort(AttnSmem& sm, int* err) {
+template <class Smem>
+__device__ __forceinline__ void raise_abort(Smem& sm, int* err) {
   record_error(err, VSA_ERR_TIMEOUT);
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
 // Lane 0 waits; the result is broadcast so the warp leaves a loop together.
-__device__ __forceinline__ bool warp_wait(AttnSmem& sm, uint64_t& bar, uint32_t parity, int lane,
-                                          int* err) {
+template <class Smem>
+__device__ __forceinline__ bool warp_wait(Smem& sm, uint64_t& bar, uint32_t parity, int lane, int* err) {
   int ok = 1;
   if (lane == 0) {
     ok = mbar_wait(smem_u32(&bar), parity, &sm.abort, kTimeoutNs) ? 1 : 0;
@@ -241,61 +240,59 @@ __device__ __forceinline__ float exp_pass(const float (&x)[32], float c, float m
   return (ps[0] + ps[1]) + (ps[2] + ps[3]);
 }
 
-// K and V into tile-major order for the attention kernel:
-//   kv[((b * H + h) * n_tiles + tile) * 32 KB + which * 16 KB + j * 8 KB + r * 128 B + 16 * (c ^ (r & 7))]
-// holds 16-byte chunk c of d-half j of slot r (which = 0 for K, 1 for V), i.e.
-// each 16 KB block is the 128-byte-swizzled K-major layout the UMMA
-// descriptors read; padding slots are zero. Consecutive threads write
-// consecutive 16-byte chunks and read the chunks of one 128-byte row.
+// Q, K and V into tile-major order for the attention kernels:
+//   qtm[((b * H + h) * n_tiles + tile) * 16 KB + j * 8 KB + r * 128 B + 16 * (c ^ (r & 7))]
+//   kv [((b * H + h) * n_tiles + tile) * 32 KB + which * 16 KB + (same)]   (which = 0: K, 1: V)
+// hold 16-byte chunk c of d-half j of slot r, i.e. each 16 KB block is the
+// 128-byte-swizzled K-major layout the UMMA descriptors read; padding slots are
+// zero. Consecutive threads write consecutive 16-byte chunks and read the
+// chunks of one 128-byte row. The tile-major Q feeds the pair pass only (the
+// sparse pass loads Q rows straight into tensor memory).
 __global__ void __launch_bounds__(256)
-permute_kv_kernel(DevLayout L, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int64_t sb,
-                  int64_t ss, int64_t sh, int H, uint8_t* __restrict__ kv) {
+permute_qkv_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                   const uint16_t* __restrict__ v, int64_t sb, int64_t ss, int64_t sh, int H, int with_q,
+                   uint8_t* __restrict__ qtm, uint8_t* __restrict__ kv) {
   const int tile = blockIdx.x, b = blockIdx.y;
   __shared__ int tok[kTile];
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
   __syncthreads();
-  const int n = H * 2048;   // (head, tensor, d-half, row, chunk)
+  const int n_t = with_q ? 3 : 2;
+  const int n = H * n_t * 1024;   // (head, tensor, d-half, row, chunk)
   for (int w = threadIdx.x; w < n; w += blockDim.x) {
-    const int pc = w & 7, r = (w >> 3) & 63, j = (w >> 9) & 1, which = (w >> 10) & 1, h = w >> 11;
+    const int pc = w & 7, r = (w >> 3) & 63, j = (w >> 9) & 1, rest = w >> 10;
+    const int which = rest % n_t + (with_q ? 0 : 1), h = rest / n_t;     // 0: Q, 1: K, 2: V
     const int t = tok[r];
     uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    const uint16_t* srcb = which == 0 ? q : (which == 1 ? k : v);
     if (t >= 0) {
-      const uint16_t* src = (which ? v : k) + b * sb + static_cast<int64_t>(t) * ss + h * sh + j * 64 +
-                            ((pc ^ (r & 7)) << 3);
+      const uint16_t* src = srcb + b * sb + static_cast<int64_t>(t) * ss + h * sh + j * 64 + ((pc ^ (r & 7)) << 3);
       val = __ldg(reinterpret_cast<const uint4*>(src));
     }
-    uint8_t* dst = kv + ((static_cast<size_t>(b) * H + h) * L.n_tiles + tile) * 32768u + which * 16384 +
-                   j * 8192 + r * 128 + pc * 16;
-    *reinterpret_cast<uint4*>(dst) = val;
+    const size_t th = (static_cast<size_t>(b) * H + h) * L.n_tiles + tile;
+    uint8_t* dst = which == 0 ? qtm + th * 16384u : kv + th * 32768u + (which - 1) * 16384;
+    *reinterpret_cast<uint4*>(dst + j * 8192 + r * 128 + pc * 16) = val;
   }
 }
 
 // Step schedule of each work item, built once per call so that the copy warps
 // of the attention kernel only stream records. Record = (key tile, flags): bit 4
-// last step of the item, bit 5 the key tile has padding slots. Key tiles come in
-// the item's order: the dense part (the conditioning tiles unless the sink mode
-// is off, or all tiles for dense rows), then the query tile's selection list
-// (ascending candidate ordinals).
+// last step of the item, bit 5 the key tile has padding slots. Key tiles are the
+// query tile's selection list (ascending candidate ordinals); the conditioning
+// keys every query attends are the pair pass's.
 constexpr int kSchedThreads = 128;
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_constant__ AttnArgs a) {
   const int item = blockIdx.x, b = blockIdx.y;
   const Geom& G = a.G;
   const Item it = decode_item(a, item);
-  const int n_dense = it.dense ? G.n_tiles : a.n_fixed;
   const size_t row = (static_cast<size_t>(b) * a.H + it.h) * G.n_tiles + it.qt;
-  const int n_sel = it.dense ? 0 : min(max(a.cnt[row], 0), a.kmax);
-  const int n = n_dense + n_sel;
+  // lists from vsa_coarse_select hold 1..kmax entries; anything else is clamped
+  const int n = min(max(a.cnt[row], 1), a.kmax);
   int2* rec = a.sched + (static_cast<size_t>(b) * a.n_items + item) * a.max_steps;
   for (int r = threadIdx.x; r < n; r += kSchedThreads) {
-    int t;
-    if (r < n_dense) {
-      t = r;
-    } else {
-      // entries outside [0, n_cand) (never written by vsa_coarse_select) are clamped: memory stays in bounds
-      const int c = a.idx[row * a.kmax + (r - n_dense)];
-      t = a.cand0 + min(max(c, 0), a.n_cand - 1);
-    }
+    // entries outside [0, n_cand) (never written by vsa_coarse_select) are clamped: memory stays in bounds
+    const int c = a.idx[row * a.kmax + r];
+    const int t = a.cand0 + min(max(c, 0), a.n_cand - 1);
     uint32_t fl = 0u;
     if (r == n - 1) fl |= 16u;
     if (a.valid[t] != ~0ull) fl |= 32u;
@@ -595,14 +592,24 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         ++j;
       }
       if (!ok) break;
-      // epilogue: out = O / l + g * o_coarse over this thread's half row (64 columns)
+      // epilogue: out = o_fine + g * o_coarse over this thread's half row (64
+      // columns). o_fine merges this pass's O / l with the pair pass's partial
+      // output over the conditioning keys, weighted 2^(ms - M) and 2^(lse - M)
+      // (the softmax over a union of key sets from the softmaxes of the parts).
       if (!(ok = warp_wait(sm, sm.o_full, it_n & 1, lane, a.err))) break;
       tc_fence_after();
-      const float inv_l = 1.0f / (l + __shfl_xor_sync(0xffffffffu, l, 16));
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      const size_t prow = ((static_cast<size_t>(a.b) * a.H + it.h) * G.n_tiles + it.qt) * kTile + r;
+      const float lse_c = (a.merge_prefix && row_ok) ? a.part_lse[prow] : -INFINITY;
+      const float mx = fmaxf(ms, lse_c);
+      const float wf = ex2_approx(ms - mx), wc = lse_c != -INFINITY ? ex2_approx(lse_c - mx) : 0.f;
+      const float inv_l = 1.0f / (l_row * wf + wc);
+      const float af = wf * inv_l, ac = wc * inv_l;
+      const float* pc = a.part_o + prow * kHeadDim + 64 * hf;
       float gate = 0.f;
       const float* oc = nullptr;
       const uint16_t* gp = nullptr;          // per-channel gate of this row (g_sd > 0)
-      if (row_ok && !(a.sink == VSA_SINK_EXACT_KV_AND_ROWS && it.qt < G.n_cond)) {
+      if (row_ok) {
         gp = a.g + a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh;
         gate = __uint_as_float(static_cast<uint32_t>(gp[0]) << 16);
         gp = kChannelGate ? gp + 64 * hf * a.g_sd : nullptr;
@@ -627,7 +634,17 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         }
         if (row_ok) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] *= inv_l;
+          for (int i = 0; i < 32; ++i) y[i] *= af;
+          if (ac != 0.f) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 t = *reinterpret_cast<const float4*>(pc + ch * 32 + i);
+              y[i] = fmaf(t.x, ac, y[i]);
+              y[i + 1] = fmaf(t.y, ac, y[i + 1]);
+              y[i + 2] = fmaf(t.z, ac, y[i + 2]);
+              y[i + 3] = fmaf(t.w, ac, y[i + 3]);
+            }
+          }
           if (kChannelGate && oc) {
             // this chunk's 32 gates as bf16 pairs (vector loads when the channels are contiguous)
             const uint16_t* gc = gp + static_cast<int64_t>(ch) * 32 * a.g_sd;
@@ -692,6 +709,411 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
   }
 }
 
+// ------------------------------------------------------------------ pair pass
+// The key tiles that every query tile of a head attends (the conditioning
+// prefix, and for dense conditioning rows the whole sequence) are run for
+// PAIRS of query tiles stacked into one M = 128 MMA: the tensor pipe runs at
+// its full rate (an M = 64 MMA takes as long as an M = 128 one) and each key
+// tile is copied once per two query tiles. Dense rows are final output; for
+// the others the pass leaves the normalised partial output and its log2-sum-
+// exp2 for the sparse pass to merge. Same roles as the sparse pass: warps 0
+// and 1 copy K and V tiles (warp 0 also the pair's Q, bulk-copied from the
+// tile-major copy as the M = 128 A operand), warp 2 issues the MMAs (S from
+// shared memory, P V with P in tensor memory), warps 3-10 run the softmax of
+// 16 rows each (two threads per row) and the epilogue. Tensor memory: O in
+// columns 0-127, two score slots in 128-255; two CTAs per SM.
+namespace pairpass {
+
+constexpr int kThreads = 352;
+constexpr int kWarpK = 0, kWarpV = 1, kWarpMma = 2, kWarpSoftmax = 3;
+constexpr int kInfoSlots = 8;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 0, kColS = 128;
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // S = Q K^T: Q and K K-major in shared memory
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // O += P V: P in TMEM, V MN-major
+
+struct Info {
+  int32_t flags;                    // bit 0: first step of the item, bit 1: last step
+  unsigned long long valid;         // slot mask of the key tile
+};
+
+struct Smem {
+  uint8_t q[2 * kTileBytes];        // the pair's Q: [d half][128 rows][128 B], rows 64-127 the second tile
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
+  Info info[kInfoSlots];
+  uint64_t k_full[2], v_full[2], s_full[2], p_full[2], pv_done[2];
+  uint64_t info_full[kInfoSlots];
+  uint64_t q_full, q_empty, o_full, drain, never;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct Args {
+  int32_t n_cond, n_tiles;
+  const int32_t* perm;              // token of (tile, slot), -1 for padding
+  const unsigned long long* valid;  // slot mask of each tile
+  const uint8_t* qtm;               // tile-major Q: ((b * H + h) * n_tiles + tile) * 16 KB
+  const uint8_t* kv;                // tile-major K, V: ((b * H + h) * n_tiles + tile) * 32 KB
+  int32_t H, b;
+  int32_t c0;                       // first query tile of the prefix pairs
+  int32_t n_dpairs, n_ppairs;       // pairs per head: dense rows (all key tiles), prefix (conditioning key tiles)
+  int32_t n_items;
+  float* part_o;                    // [B, H, n_tiles, 64, 128] normalised partial output
+  float* part_lse;                  // [B, H, n_tiles, 64] its log2-sum-exp2 (scaled log2 domain)
+  void* out;
+  int32_t out_bf16;
+  int64_t o_sb, o_ss, o_sh;
+  float scale_log2;
+  int* err;
+  uint64_t stall_ns;                // > 0: the MMA warp first waits this long on a barrier nothing arrives on
+};
+
+struct PItem {
+  int h, qa, qb;                    // query tiles of rows 0-63 and 64-127 (qb < 0: none)
+  int n;                            // key tiles 0 .. n - 1
+  int dense;
+};
+
+__device__ __forceinline__ PItem decode(const Args& a, int item) {
+  PItem it;
+  const int nd = a.H * a.n_dpairs;
+  if (item < nd) {
+    it.h = item / a.n_dpairs;
+    const int p = item - it.h * a.n_dpairs;
+    it.qa = 2 * p;
+    it.qb = 2 * p + 1 < a.n_cond ? 2 * p + 1 : -1;
+    it.n = a.n_tiles;
+    it.dense = 1;
+  } else {
+    const int r = item - nd;
+    it.h = r / a.n_ppairs;
+    const int p = r - it.h * a.n_ppairs;
+    it.qa = a.c0 + 2 * p;
+    it.qb = it.qa + 1 < a.n_tiles ? it.qa + 1 : -1;
+    it.n = a.n_cond;
+    it.dense = 0;
+  }
+  return it;
+}
+
+__global__ void __maxnreg__(80) pair_attn_kernel(const __grid_constant__ Args a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {          // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) record_error(a.err, VSA_ERR_UNSUPPORTED);
+    return;
+  }
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.k_full[i]), 1);
+      mbar_init(smem_u32(&sm.v_full[i]), 1);
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.p_full[i]), 8);      // one arrival per softmax warp
+      mbar_init(smem_u32(&sm.pv_done[i]), 1);
+    }
+    for (int s = 0; s < kInfoSlots; ++s) mbar_init(smem_u32(&sm.info_full[s]), 1);
+    mbar_init(smem_u32(&sm.q_full), 1);
+    mbar_init(smem_u32(&sm.q_empty), 1);
+    mbar_init(smem_u32(&sm.o_full), 1);
+    mbar_init(smem_u32(&sm.drain), 1);
+    mbar_init(smem_u32(&sm.never), 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const size_t head0 = static_cast<size_t>(a.b) * a.H;
+
+  if (warp == kWarpK || warp == kWarpV) {
+    // ----------------------------------------------------------- producers
+    // Key tiles 0 .. n - 1 of every item into stage j & 1: a K stage is free
+    // again once S of its previous step completed (s_full), a V stage once
+    // O += P V of it did (pv_done). The K warp also copies each pair's Q (once
+    // the previous pair's S completed) and publishes per-step tile info.
+    const bool is_k = warp == kWarpK;
+    uint64_t* full = is_k ? sm.k_full : sm.v_full;
+    uint64_t* freed = is_k ? sm.s_full : sm.pv_done;
+    uint32_t step = 0;
+    int it_n = 0, q_last = -1;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
+      const PItem it = decode(a, item);
+      const uint8_t* head_kv = a.kv + (head0 + it.h) * a.n_tiles * 32768u + (is_k ? 0u : 16384u);
+      if (is_k) {
+        if (it_n >= 1 && !(ok = warp_wait(sm, sm.q_empty, (it_n - 1) & 1, lane, a.err))) break;
+        if (lane == 0) {
+          const uint8_t* qa = a.qtm + ((head0 + it.h) * a.n_tiles + it.qa) * kTileBytes;
+          const uint8_t* qb = a.qtm + ((head0 + it.h) * a.n_tiles + (it.qb >= 0 ? it.qb : it.qa)) * kTileBytes;
+          const uint32_t bar = smem_u32(&sm.q_full);
+          mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+          bulk_load(smem_u32(sm.q), qa, 8192, bar);
+          bulk_load(smem_u32(sm.q) + 8192, qb, 8192, bar);
+          bulk_load(smem_u32(sm.q) + 16384, qa + 8192, 8192, bar);
+          bulk_load(smem_u32(sm.q) + 24576, qb + 8192, 8192, bar);
+        }
+        q_last = it_n;
+        __syncwarp();
+      }
+      unsigned long long v_cur = 0ull;       // slot masks of key tiles jj .. jj + 31, one per lane
+      for (int jj = 0; jj < it.n; ++jj) {
+        if (is_k && (jj & 31) == 0) v_cur = jj + lane < it.n ? a.valid[jj + lane] : 0ull;
+        const unsigned long long vm = __shfl_sync(0xffffffffu, v_cur, jj & 31);
+        const int st = step & 1;
+        if (step >= 2 && !(ok = warp_wait(sm, freed[st], ((step >> 1) - 1) & 1, lane, a.err))) break;
+        if (lane == 0) {
+          if (is_k) {
+            Info& inf = sm.info[step % kInfoSlots];
+            inf.flags = (jj == 0 ? 1 : 0) | (jj == it.n - 1 ? 2 : 0);
+            inf.valid = vm;
+            mbar_arrive(smem_u32(&sm.info_full[step % kInfoSlots]));
+          }
+          const uint32_t bar = smem_u32(&full[st]);
+          mbar_arrive_expect_tx(bar, kTileBytes);
+          bulk_load(smem_u32(is_k ? sm.k[st] : sm.v[st]), head_kv + static_cast<size_t>(jj) * 32768u, kTileBytes,
+                    bar);
+        }
+        __syncwarp();
+        ++step;
+      }
+    }
+    if (!ok && lane == 0) {
+      // let every issued copy land before the block can exit
+      for (uint32_t i = (step > 2u ? step - 2u : 0u); i < step; ++i)
+        mbar_wait(smem_u32(&full[i & 1]), (i >> 1) & 1, nullptr, kDrainNs);
+      if (is_k && q_last >= 0) mbar_wait(smem_u32(&sm.q_full), q_last & 1, nullptr, kDrainNs);
+    }
+  } else if (warp == kWarpMma) {
+    // ----------------------------------------------------------------- MMA
+    // S(j) once O += P(j - 2) V was issued (its score slot is free: MMAs from
+    // one thread run in issue order), the pair's Q and K(j) have landed;
+    // O += P(j) V once all softmax warps wrote P(j) and V(j) has landed. The
+    // thread issues whichever is ready, S first.
+    bool ok = true;
+    if (lane == 0) {
+      if (a.stall_ns) ok = mbar_wait(smem_u32(&sm.never), 0, &sm.abort, a.stall_ns);   // injected failure
+      uint32_t ns = 0, np = 0, ring = 0;
+      int s_item = blockIdx.x, s_it = 0;
+      bool s_done = s_item >= a.n_items;
+      uint64_t t_idle = globaltimer_ns();
+      uint32_t spins = 0;
+      const uint64_t qd = smem_desc_sw128(smem_u32(sm.q), 16, 1024);
+      while (ok) {
+        bool progress = false;
+        if (!s_done && ns < np + 2 && mbar_test_wait(smem_u32(&sm.k_full[ns & 1]), (ns >> 1) & 1) &&
+            (!(sm.info[ns % kInfoSlots].flags & 1) || mbar_test_wait(smem_u32(&sm.q_full), s_it & 1))) {
+          tc_fence_after();
+          const int fl = sm.info[ns % kInfoSlots].flags;
+          // 16 d per K step: 32 B inside a swizzle row of the d half kk / 4
+          // (descriptor addresses count 16-byte units)
+          const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ns & 1]), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + kColS + 64 * (ns & 1), qd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2,
+                    kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdescS, kk > 0 ? 1u : 0u);
+          umma_commit(smem_u32(&sm.s_full[ns & 1]));
+          ring = (ring & ~(3u << (2 * (ns & 3)))) | (static_cast<uint32_t>(fl & 3) << (2 * (ns & 3)));
+          if (fl & 2) {
+            umma_commit(smem_u32(&sm.q_empty));       // the pair's Q may be replaced
+            s_item += gridDim.x;
+            ++s_it;
+            s_done = s_item >= a.n_items;
+          }
+          ++ns;
+          progress = true;
+        }
+        if (np < ns && mbar_test_wait(smem_u32(&sm.p_full[np & 1]), (np >> 1) & 1) &&
+            mbar_test_wait(smem_u32(&sm.v_full[np & 1]), (np >> 1) & 1)) {
+          tc_fence_after();
+          const uint32_t fl = (ring >> (2 * (np & 3))) & 3u;
+          // V as MN-major B: 64-d blocks 8 KB apart, 16 keys = 2 KB per K step;
+          // P (A, over its scores in TMEM): 16 keys = 8 columns of bf16 pairs
+          const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[np & 1]), 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + kColO, tmem + kColS + 64 * (np & 1) + kk * 8, vd + kk * (2048 >> 4), kIdescPV,
+                    ((fl & 1) && kk == 0) ? 0u : 1u);
+          umma_commit(smem_u32(&sm.pv_done[np & 1]));
+          if (fl & 2) umma_commit(smem_u32(&sm.o_full));
+          ++np;
+          progress = true;
+        }
+        if (s_done && np == ns) break;
+        if (progress) {
+          spins = 0;
+        } else if ((++spins & 255u) == 0) {
+          const uint64_t now = globaltimer_ns();
+          if (spins == 256u) t_idle = now;
+          if (*reinterpret_cast<volatile int*>(&sm.abort) || now - t_idle > kTimeoutNs) ok = false;
+        }
+      }
+      if (!ok) raise_abort(sm, a.err);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      umma_commit(smem_u32(&sm.drain));
+      mbar_wait(smem_u32(&sm.drain), 0, nullptr, kDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ softmax / epilogue
+    // Warp w owns TMEM lanes 32 (w & 3) + 16 s .. + 15 (s = (w - 3) / 4), i.e.
+    // rows of the M = 128 pair (row r in lane r: rows 0-63 the first query
+    // tile, 64-127 the second). Thread t handles row t & 15 of them and the key
+    // (or output column) half hf = t >> 4; its partner is thread t ^ 16.
+    const int quad = warp & 3;
+    const int sub = (warp - kWarpSoftmax) >> 2;
+    const int hf = lane >> 4;
+    const int prow = quad * 32 + sub * 16 + (lane & 15);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32 + sub * 16) << 16);
+    const float c = a.scale_log2;
+    uint32_t j = 0;
+    int it_n = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it_n) {
+      const PItem it = decode(a, item);
+      const int qtile = prow < 64 ? it.qa : it.qb;
+      const int slot = prow & 63;
+      const int tok = qtile >= 0 ? a.perm[qtile * kTile + slot] : -1;
+      const bool row_ok = tok >= 0;
+      const uint32_t j0 = j, jend = j + it.n;
+      float ms = -INFINITY, l = 0.f;
+      bool have_next = false, s_ready = false;
+      Info next{};
+      for (; j < jend; ++j) {
+        Info inf;
+        if (have_next) {
+          inf = next;
+        } else {
+          if (!(ok = warp_wait(sm, sm.info_full[j % kInfoSlots], (j / kInfoSlots) & 1, lane, a.err))) break;
+          inf = sm.info[j % kInfoSlots];
+        }
+        if (!s_ready && !(ok = warp_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, lane, a.err))) break;
+        tc_fence_after();
+        const bool more = j + 1 < jend;
+        uint32_t t_info = 0, t_s = 0;
+        if (more) {
+          t_info = mbar_test_wait(smem_u32(&sm.info_full[(j + 1) % kInfoSlots]), ((j + 1) / kInfoSlots) & 1);
+          t_s = mbar_test_wait(smem_u32(&sm.s_full[(j + 1) & 1]), ((j + 1) >> 1) & 1);
+        }
+        const uint32_t scol = lane_addr + kColS + 64 * (j & 1);
+        float x[32];
+        tmem_ld16x2_32f<32>(scol, x);
+        tmem_wait_ld();
+        if (inf.valid != ~0ull) {             // padding slots never attend
+          const uint32_t vm = static_cast<uint32_t>(inf.valid >> (32 * hf));
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = ((vm >> i) & 1u) ? x[i] : -INFINITY;
+        }
+        // exact row max; O and l rescaled when it raises the running max
+        auto exact_max = [&]() -> bool {
+          float m = x[0];
+#pragma unroll
+          for (int i = 1; i < 32; ++i) m = fmaxf(m, x[i]);
+          const float mt = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16)) * c;
+          const bool need = ms != -INFINITY && mt > ms;
+          if (ms == -INFINITY) ms = mt;       // first key tile of the item: O and l are still zero
+          if (__any_sync(0xffffffffu, need)) {
+            // rescale once the last O += P V (of step j - 1) has landed
+            if (j > j0 && !warp_wait(sm, sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lane, a.err)) return false;
+            tc_fence_after();
+            const float f = need ? ex2_approx(ms - mt) : 1.0f;
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint32_t oa = lane_addr + kColO + 16 * ch;
+              float u[16];
+              tmem_ld16x2_16f<64>(oa, u);
+              tmem_wait_ld();
+              uint32_t w[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(u[i] * f);
+              tmem_st16x2_16<64>(oa, w);
+            }
+            tmem_wait_st();
+            if (need) {
+              l *= f;
+              ms = mt;
+            }
+          }
+          return true;
+        };
+        // P against the running max; the exact max only when a row has no
+        // reference yet or its sum of P exceeds 2^8 (every P stays <= 2^8)
+        uint32_t pw[16];
+        if (__any_sync(0xffffffffu, ms == -INFINITY) && !(ok = exact_max())) break;
+        float psum = exp_pass(x, c, ms, pw);
+        if (__any_sync(0xffffffffu, psum + __shfl_xor_sync(0xffffffffu, psum, 16) > kPSumLimit)) {
+          if (!(ok = exact_max())) break;
+          psum = exp_pass(x, c, ms, pw);
+        }
+        l += psum;
+        tmem_st16x2_16<16>(scol, pw);          // P(j) over the first 32 columns of its slot
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[j & 1]));
+        have_next = more && __all_sync(0xffffffffu, t_info);
+        if (have_next) next = sm.info[(j + 1) % kInfoSlots];
+        s_ready = more && __all_sync(0xffffffffu, t_s);
+      }
+      if (!ok) break;
+      // epilogue: dense rows -> out = O / l (no coarse term); prefix rows ->
+      // the normalised partial output and its log2-sum-exp2
+      if (!(ok = warp_wait(sm, sm.o_full, it_n & 1, lane, a.err))) break;
+      tc_fence_after();
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      const float inv_l = 1.0f / l_row;
+      const size_t poff = ((head0 + it.h) * a.n_tiles + (qtile >= 0 ? qtile : 0)) * kTile + slot;
+      if (row_ok && !it.dense && hf == 0) a.part_lse[poff] = ms + __log2f(l_row);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float y[16];
+        tmem_ld16x2_16f<64>(lane_addr + kColO + 16 * ch, y);
+        tmem_wait_ld();
+        if (!row_ok) continue;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] *= inv_l;
+        const int col = 64 * hf + 16 * ch;
+        if (!it.dense) {
+          float4* dst = reinterpret_cast<float4*>(a.part_o + poff * kHeadDim + col);
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) dst[i / 4] = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
+        } else {
+          const int64_t off = a.b * a.o_sb + tok * a.o_ss + it.h * a.o_sh + col;
+          if (a.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + off);
+#pragma unroll
+            for (int i = 0; i < 16; i += 8)
+              dst[i / 8] = make_uint4(pack_bf16x2(y[i], y[i + 1]), pack_bf16x2(y[i + 2], y[i + 3]),
+                                      pack_bf16x2(y[i + 4], y[i + 5]), pack_bf16x2(y[i + 6], y[i + 7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + off);
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) dst[i / 4] = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
+          }
+        }
+      }
+      // the next item's first O += P V overwrites O only after every softmax
+      // warp's P of that step, i.e. after every warp finished reading O here
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace pairpass
+
 // ------------------------------------------------------------------ host side
 int sm_count() {
   int dev = 0, n = 0;
@@ -700,43 +1122,52 @@ int sm_count() {
   return n;
 }
 
-constexpr size_t kAttnHeader = 256;   // error word
+constexpr size_t kAttnHeader = 256;   // status word, failed-call count
 
 std::atomic<uint64_t> g_stall_ns{0};   // vsa_debug_inject_wait_timeout
 constexpr size_t kMaxAttnSmem = 227 * 1024;
 
-// Work decomposition shared by the host and the kernels (see decode_item).
-struct ItemCounts {
-  int32_t c0, nq_dense, nq_sparse, n_dense_items, n_items, n_fixed, max_steps;
+// Work decomposition shared by the host and the kernels (see decode_item and
+// pairpass::decode). The conditioning keys that every query attends go to the
+// pair pass (dense rows: all keys); the sparse pass walks the selection lists.
+struct Passes {
+  int32_t c0, nq, max_steps;           // sparse pass: query tiles [c0, n_tiles); steps per item <= max_steps
+  int32_t n_dpairs, n_ppairs;          // pair pass, per head
+  int32_t merge_prefix;                // the sparse epilogue merges the pair pass's partial output
 };
 
-ItemCounts item_counts(const vsa_layout* L, int H, const vsa_params* p, int32_t kmax) {
-  ItemCounts c{};
+Passes passes(const vsa_layout* L, const vsa_params* p, int32_t kmax) {
+  Passes s{};
   const bool rows = p->sink == VSA_SINK_EXACT_KV_AND_ROWS;
-  c.c0 = rows ? L->n_cond : 0;
-  c.nq_dense = rows ? L->n_cond : 0;
-  c.nq_sparse = L->n_tiles - c.c0;
-  c.n_dense_items = c.nq_dense * H;
-  c.n_items = c.n_dense_items + c.nq_sparse * H;
-  c.n_fixed = p->sink == VSA_SINK_OFF ? 0 : L->n_cond;
-  c.max_steps = std::max(rows ? L->n_tiles : 0, c.n_fixed + std::min(kmax, candidates(L, p->sink).count));
-  return c;
+  s.c0 = rows ? L->n_cond : 0;
+  s.nq = L->n_tiles - s.c0;
+  s.max_steps = std::max(1, std::min(kmax, candidates(L, p->sink).count));
+  s.n_dpairs = rows ? (L->n_cond + 1) / 2 : 0;
+  s.n_ppairs = (p->sink != VSA_SINK_OFF && L->n_cond > 0) ? (s.nq + 1) / 2 : 0;
+  s.merge_prefix = s.n_ppairs > 0;
+  return s;
 }
 
-// [error word][tile-major K/V][step records][steps per item]
+// [header][tile-major K/V][tile-major Q][step records][steps per item][partial output][partial log-sum-exp]
 struct AttnWorkspace {
-  size_t kv, sched, nsteps, total;
+  size_t kv, qtm, sched, nsteps, part_o, part_lse, total;
 };
 
 AttnWorkspace attn_workspace(const vsa_layout* L, int B, int H, const vsa_params* p) {
   int32_t kmax = 0;
   vsa_select_kmax(L, p, &kmax);
-  const ItemCounts c = item_counts(L, H, p, kmax);
+  const Passes s = passes(L, p, kmax);
+  const bool pairs = s.n_dpairs + s.n_ppairs > 0;
+  const size_t tiles = static_cast<size_t>(B) * H * L->n_tiles;
+  const size_t items = static_cast<size_t>(B) * H * s.nq;
   AttnWorkspace w{};
   w.kv = kAttnHeader;
-  w.sched = w.kv + static_cast<size_t>(B) * H * L->n_tiles * 32768u;
-  w.nsteps = w.sched + align_up(static_cast<size_t>(B) * c.n_items * c.max_steps * sizeof(int2), 256);
-  w.total = w.nsteps + align_up(static_cast<size_t>(B) * c.n_items * sizeof(int32_t), 256);
+  w.qtm = w.kv + tiles * 2 * kTileBytes;
+  w.sched = w.qtm + (pairs ? tiles * kTileBytes : 0);
+  w.nsteps = w.sched + align_up(items * s.max_steps * sizeof(int2), 256);
+  w.part_o = w.nsteps + align_up(items * sizeof(int32_t), 256);
+  w.part_lse = w.part_o + (s.merge_prefix ? tiles * kTile * kHeadDim * sizeof(float) : 0);
+  w.total = w.part_lse + align_up(s.merge_prefix ? tiles * kTile * sizeof(float) : 0, 256);
   return w;
 }
 
@@ -808,17 +1239,15 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.H = H;
   a.sink = p->sink;
   a.kmax = kmax;
-  const ItemCounts ic = item_counts(L, H, p, kmax);
-  a.c0 = ic.c0;
-  a.n_fixed = ic.n_fixed;
+  const Passes ps = passes(L, p, kmax);
+  a.c0 = ps.c0;
   const Candidates cand = candidates(L, p->sink);
   a.cand0 = cand.first;
   a.n_cand = cand.count;
-  a.nq_dense = ic.nq_dense;
-  a.nq_sparse = ic.nq_sparse;
-  a.n_dense_items = ic.n_dense_items;
-  a.n_items = ic.n_items;
-  a.max_steps = ic.max_steps;
+  a.nq = ps.nq;
+  a.n_items = ps.nq * H;
+  a.max_steps = ps.max_steps;
+  a.merge_prefix = ps.merge_prefix;
   a.valid = D.valid;
   a.idx = idx;
   a.cnt = cnt;
@@ -837,29 +1266,66 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.err = static_cast<int*>(workspace);
   a.stall_ns = g_stall_ns.load(std::memory_order_relaxed);
 
-  auto attn_kernel = g_sd > 0 ? vsa_attn_kernel<true> : vsa_attn_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
-  e = cudaMemsetAsync(workspace, 0, sizeof(int), stream);   // this call's status word only
-  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaMemsetAsync", e);
-  const int grid = std::max(1, std::min(a.n_items, 2 * n_sm));   // two CTAs per SM, 256 TMEM columns each
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   a.kv = wsb + ws.kv;
   a.sched = reinterpret_cast<int2*>(wsb + ws.sched);
   a.nsteps = reinterpret_cast<int32_t*>(wsb + ws.nsteps);
-  permute_kv_kernel<<<dim3(L->n_tiles, B), 256, 0, stream>>>(D, static_cast<const uint16_t*>(k),
-                                                            static_cast<const uint16_t*>(v), sb, ss, sh, H,
-                                                            wsb + ws.kv);
+  a.part_o = reinterpret_cast<const float*>(wsb + ws.part_o);
+  a.part_lse = reinterpret_cast<const float*>(wsb + ws.part_lse);
+
+  pairpass::Args pa{};
+  pa.n_cond = L->n_cond;
+  pa.n_tiles = L->n_tiles;
+  pa.perm = D.perm;
+  pa.valid = D.valid;
+  pa.qtm = wsb + ws.qtm;
+  pa.kv = wsb + ws.kv;
+  pa.H = H;
+  pa.c0 = ps.c0;
+  pa.n_dpairs = ps.n_dpairs;
+  pa.n_ppairs = ps.n_ppairs;
+  pa.n_items = H * (ps.n_dpairs + ps.n_ppairs);
+  pa.part_o = reinterpret_cast<float*>(wsb + ws.part_o);
+  pa.part_lse = reinterpret_cast<float*>(wsb + ws.part_lse);
+  pa.out = out;
+  pa.out_bf16 = a.out_bf16;
+  pa.o_sb = o_sb;
+  pa.o_ss = o_ss;
+  pa.o_sh = o_sh;
+  pa.scale_log2 = a.scale_log2;
+  pa.err = a.err;
+  pa.stall_ns = a.stall_ns;
+
+  auto attn_kernel = g_sd > 0 ? vsa_attn_kernel<true> : vsa_attn_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute", e);
+  const size_t pair_smem = sizeof(pairpass::Smem);
+  e = cudaFuncSetAttribute(pairpass::pair_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pair_smem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaFuncSetAttribute(pair)", e);
+  e = cudaMemsetAsync(workspace, 0, sizeof(int), stream);   // this call's status word only
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: cudaMemsetAsync", e);
+  permute_qkv_kernel<<<dim3(L->n_tiles, B), 256, 0, stream>>>(
+      D, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), sb, ss,
+      sh, H, pa.n_items > 0 ? 1 : 0, wsb + ws.qtm, wsb + ws.kv);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: permute launch", e);
   schedule_kernel<<<dim3(a.n_items, B), kSchedThreads, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: schedule launch", e);
   for (int b = 0; b < B; ++b) {
+    if (pa.n_items > 0) {
+      pa.b = b;
+      pairpass::pair_attn_kernel<<<std::max(1, std::min(pa.n_items, 2 * n_sm)), pairpass::kThreads, pair_smem,
+                                   stream>>>(pa);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: pair pass launch", e);
+    }
     a.b = b;
     a.q = static_cast<const uint16_t*>(q) + b * sb;
-    attn_kernel<<<grid, kThreads, smem, stream>>>(a);
+    // two CTAs per SM, 256 TMEM columns each
+    attn_kernel<<<std::max(1, std::min(a.n_items, 2 * n_sm)), kThreads, smem, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: launch", e);
   }

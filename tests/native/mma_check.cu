@@ -1,17 +1,18 @@
-// Test harness (not part of libvsa): runs the attention kernel's tcgen05
-// building blocks once on small inputs so that tests can compare each against
-// a torch matmul:
-//   S1 = Q K^T   Q [128 x 128] and K [64 x 128] loaded by the 3-D token map
-//   S2 = Q Kc^T  Kc = one 4x4x4 cube gathered by the 5-D video-grid map
-//   O  = P V     P [128 x 64] written to 128B-swizzled smem by threads,
-//                V [64 x 128] loaded by the 3-D map, used as an MN-major operand
-//   O2 = P V     the same product with P written to TMEM by tcgen05.st
-//                (row i in lane i, bf16 pairs per column) and read as A from TMEM
-// Same descriptors, swizzle and TMEM access pattern as vsa_attn.cu. All waits
-// are bounded; a wait that runs out writes 1 to *err.
-#include <cuda.h>
+// Test-only check of the tcgen05 building blocks the attention kernels use, in
+// the same forms (one CTA, 4 warps):
+//  * bulk copies of 16 KB tile-major operand tiles ([d half][64 rows][128 B],
+//    128-byte swizzled) and of a query-tile pair as four 8 KB pieces into the
+//    [d half][128 rows][128 B] layout;
+//  * S = Q K^T with M = 64 (Q and K from shared memory) into TMEM lane half 0
+//    and lane half 1 (address lane field 0 and 16), and with M = 128 on a pair;
+//  * P written into TMEM as bf16 pairs with the 16x32bx2 store shape, then
+//    O = P V with P as the A operand in TMEM and V MN-major from shared memory,
+//    for M = 64 in lane half 1 and for M = 128;
+//  * every read-back with the 16x32bx2 load shape.
+// Results go to global memory for the host to compare with plain matmuls.
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
+
+#include <cstdint>
 
 #include "sm100.cuh"
 
@@ -19,180 +20,165 @@ using namespace vsa::sm100;
 
 namespace {
 
-struct __align__(1024) CheckSmem {
-  uint8_t q[2][128 * 128];
-  uint8_t k[2][64 * 128];
-  uint8_t kc[2][64 * 128];
-  uint8_t v[2][64 * 128];
-  uint8_t p[128 * 128];
-  uint64_t bar_load, bar_mma, bar_ts;
-  uint32_t tmem_base;
+constexpr uint32_t kCols = 512;
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+struct Smem {
+  uint8_t q[16384];
+  uint8_t qp[32768];
+  uint8_t k[16384];
+  uint8_t v[16384];
+  uint64_t bar_load, bar_mma;
+  uint32_t tmem;
+  int fail;
 };
 
-constexpr uint64_t kTimeout = 2000000000ull;
+// bf16 bits of a row-major [rows, 64] P (keys 32 hf .. + 31 of row r) as 16 pairs
+__device__ void load_p_pairs(const uint16_t* p, int r, int hf, uint32_t (&w)[16]) {
+  const uint16_t* src = p + r * 64 + 32 * hf;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = static_cast<uint32_t>(src[2 * i]) | (static_cast<uint32_t>(src[2 * i + 1]) << 16);
+}
+
+// rows (lanes base .. base + 15 of warp w) x 64 fp32 columns from TMEM, split 32
+__device__ void store_rows64(uint32_t taddr, float* out, int row0, int ld) {
+  const int lane = threadIdx.x & 31;
+  float x[32];
+  tmem_ld16x2_32f<32>(taddr, x);
+  tmem_wait_ld();
+  float* dst = out + (row0 + (lane & 15)) * ld + 32 * (lane >> 4);
+  for (int i = 0; i < 32; ++i) dst[i] = x[i];
+}
+
+// same rows x 128 fp32 columns, split 64 (two loads of 32)
+__device__ void store_rows128(uint32_t taddr, float* out, int row0) {
+  const int lane = threadIdx.x & 31;
+  for (int ch = 0; ch < 2; ++ch) {
+    float x[32];
+    tmem_ld16x2_32f<64>(taddr + 32 * ch, x);
+    tmem_wait_ld();
+    float* dst = out + (row0 + (lane & 15)) * 128 + 64 * (lane >> 4) + 32 * ch;
+    for (int i = 0; i < 32; ++i) dst[i] = x[i];
+  }
+}
 
 __global__ void __launch_bounds__(128, 1)
-check_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tgrid,
-             int cube_t0, int cube_h0, int cube_w0, int cube_head, const uint16_t* p_in,
-             float* s1_out, float* s2_out, float* o_out, float* o2_out, int* err) {
-  extern __shared__ uint8_t raw[];
-  CheckSmem& sm = *reinterpret_cast<CheckSmem*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
+mma_check_kernel(const uint8_t* q, const uint8_t* qa, const uint8_t* qb, const uint8_t* k, const uint8_t* v,
+                 const uint16_t* p64, const uint16_t* p128, float* s64_0, float* s64_1, float* s128, float* o64,
+                 float* o128, int* err) {
+  extern __shared__ __align__(1024) uint8_t raw[];
+  if (smem_u32(raw) & 1023u) {
+    if (threadIdx.x == 0) *err = 99;
+    return;
+  }
+  Smem& sm = *reinterpret_cast<Smem*>(raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.bar_load), 1);
     mbar_init(smem_u32(&sm.bar_mma), 1);
-    mbar_init(smem_u32(&sm.bar_ts), 1);
+    sm.fail = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_alloc(smem_u32(&sm.tmem), kCols);
     tmem_relinquish();
   }
-  // P: row r = thread, 64 bf16, written in the 128B-swizzled K-major layout
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(p_in + tid * 64);
-    for (int ch = 0; ch < 8; ++ch)
-      *reinterpret_cast<uint4*>(sm.p + tid * 128 + ((ch ^ (tid & 7)) << 4)) = src[ch];
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  bool ok = true;
-  if (tid == 0) {
+  const uint32_t tm = sm.tmem;
+
+  if (threadIdx.x == 0) {
     const uint32_t bar = smem_u32(&sm.bar_load);
-    mbar_arrive_expect_tx(bar, 32768 + 16384 * 3);
-    tma_load_3d(smem_u32(sm.q[0]), &tq, bar, 0, 0, 0);
-    tma_load_3d(smem_u32(sm.q[0] + 8192), &tq, bar, 0, 0, 64);
-    tma_load_3d(smem_u32(sm.q[1]), &tq, bar, 64, 0, 0);
-    tma_load_3d(smem_u32(sm.q[1] + 8192), &tq, bar, 64, 0, 64);
-    tma_load_3d(smem_u32(sm.k[0]), &tk, bar, 0, 0, 0);
-    tma_load_3d(smem_u32(sm.k[1]), &tk, bar, 64, 0, 0);
-    tma_load_3d(smem_u32(sm.v[0]), &tv, bar, 0, 0, 0);
-    tma_load_3d(smem_u32(sm.v[1]), &tv, bar, 64, 0, 0);
-    tma_load_5d(smem_u32(sm.kc[0]), &tgrid, bar, 0, cube_head, cube_w0, cube_h0, cube_t0);
-    tma_load_5d(smem_u32(sm.kc[1]), &tgrid, bar, 64, cube_head, cube_w0, cube_h0, cube_t0);
-    ok = mbar_wait(bar, 0, nullptr, kTimeout);
-    if (ok) {
-      tc_fence_after();
-      const uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
+    mbar_arrive_expect_tx(bar, 16384u * 5);
+    bulk_load(smem_u32(sm.q), q, 16384, bar);
+    bulk_load(smem_u32(sm.qp), qa, 8192, bar);
+    bulk_load(smem_u32(sm.qp) + 8192, qb, 8192, bar);
+    bulk_load(smem_u32(sm.qp) + 16384, qa + 8192, 8192, bar);
+    bulk_load(smem_u32(sm.qp) + 24576, qb + 8192, 8192, bar);
+    bulk_load(smem_u32(sm.k), k, 16384, bar);
+    bulk_load(smem_u32(sm.v), v, 16384, bar);
+    if (!mbar_wait(bar, 0, nullptr, kWaitNs)) sm.fail = 1;
+    tc_fence_after();
+    if (!sm.fail) {
+      const uint64_t qd = smem_desc_sw128(smem_u32(sm.q), 16, 1024);
+      const uint64_t pd = smem_desc_sw128(smem_u32(sm.qp), 16, 1024);
+      const uint64_t kd = smem_desc_sw128(smem_u32(sm.k), 16, 1024);
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk & 3) * 32;
-        const uint64_t ad = smem_desc_sw128(smem_u32(sm.q[0]) + (kk >> 2) * 16384 + off, 16, 1024);
-        umma_ss(tmem + 128, ad, smem_desc_sw128(smem_u32(sm.k[0]) + (kk >> 2) * 8192 + off, 16, 1024),
-                idS, kk > 0);
-        umma_ss(tmem + 192, ad, smem_desc_sw128(smem_u32(sm.kc[0]) + (kk >> 2) * 8192 + off, 16, 1024),
-                idS, kk > 0);
+        const uint64_t ko = (kk >> 2) * (8192 >> 4) + (kk & 3) * 2;
+        umma_ss(tm + 0, qd + ko, kd + ko, idesc_bf16_f32(64, 64, 0, 0), kk > 0);                     // half 0, cols 0-63
+        umma_ss(tm + (16u << 16) + 64, qd + ko, kd + ko, idesc_bf16_f32(64, 64, 0, 0), kk > 0);      // half 1, cols 64-127
+        umma_ss(tm + 128, pd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2, kd + ko, idesc_bf16_f32(128, 64, 0, 0),
+                kk > 0);                                                                                // M = 128, cols 128-191
       }
-      for (int kk = 0; kk < 4; ++kk)
-        umma_ss(tmem, smem_desc_sw128(smem_u32(sm.p) + kk * 32, 16, 1024),
-                smem_desc_sw128(smem_u32(sm.v[0]) + kk * 2048, 8192, 1024), idPV, kk > 0);
       umma_commit(smem_u32(&sm.bar_mma));
-      ok = mbar_wait(smem_u32(&sm.bar_mma), 0, nullptr, kTimeout);
+      if (!mbar_wait(smem_u32(&sm.bar_mma), 0, nullptr, kWaitNs)) sm.fail = 2;
     }
-    if (!ok) *err = 1;
   }
   __syncthreads();
-  ok = *reinterpret_cast<volatile int*>(err) == 0;
-  const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  if (ok) {
-    // P into TMEM columns 384..415 of this thread's lane, then O2 = P V from TMEM
-    tc_fence_after();
-    uint32_t w[32];
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(p_in + tid * 64);
-    for (int c = 0; c < 32; ++c) w[c] = src[c];
-    tmem_st32(la + 384, w);
+  tc_fence_after();
+  if (sm.fail) {
+    if (threadIdx.x == 0) *err = sm.fail;
+  } else {
+    const uint32_t q0 = tm + (static_cast<uint32_t>(warp * 32) << 16);
+    store_rows64(q0 + 0, s64_0, 16 * warp, 64);                        // M = 64: rows 16 w .. in lanes 32 w ..
+    store_rows64(q0 + (16u << 16) + 64, s64_1, 16 * warp, 64);
+    store_rows64(q0 + 128, s128, 32 * warp, 64);                       // M = 128: row r in lane r
+    store_rows64(q0 + (16u << 16) + 128, s128, 32 * warp + 16, 64);
+    // P into TMEM: M = 64 in lane half 1 at columns 256-287, M = 128 at 320-351
+    uint32_t w[16];
+    load_p_pairs(p64, 16 * warp + (lane & 15), lane >> 4, w);
+    tmem_st16x2_16<16>(q0 + (16u << 16) + 256, w);
+    load_p_pairs(p128, 32 * warp + (lane & 15), lane >> 4, w);
+    tmem_st16x2_16<16>(q0 + 320, w);
+    load_p_pairs(p128, 32 * warp + 16 + (lane & 15), lane >> 4, w);
+    tmem_st16x2_16<16>(q0 + (16u << 16) + 320, w);
     tmem_wait_st();
   }
   tc_fence_before();
   __syncthreads();
-  if (ok && tid == 0) {
-    tc_fence_after();
-    const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
-    for (int kk = 0; kk < 4; ++kk)
-      umma_ts(tmem + 256, tmem + 384 + kk * 8, smem_desc_sw128(smem_u32(sm.v[0]) + kk * 2048, 8192, 1024),
-              idPV, kk > 0);
-    umma_commit(smem_u32(&sm.bar_ts));
-    if (!mbar_wait(smem_u32(&sm.bar_ts), 0, nullptr, kTimeout)) *err = 1;
+  tc_fence_after();
+  if (threadIdx.x == 0 && !sm.fail) {
+    const uint64_t vd = smem_desc_sw128(smem_u32(sm.v), 8192, 1024);
+    for (int kk = 0; kk < 4; ++kk) {
+      umma_ts(tm + (16u << 16) + 384, tm + (16u << 16) + 256 + kk * 8, vd + kk * (2048 >> 4),
+              idesc_bf16_f32(64, 128, 0, 1), kk > 0);                                   // O64, lane half 1, cols 384-511
+      umma_ts(tm + 0, tm + 320 + kk * 8, vd + kk * (2048 >> 4), idesc_bf16_f32(128, 128, 0, 1), kk > 0);   // O128, cols 0-127
+    }
+    umma_commit(smem_u32(&sm.bar_mma));
+    if (!mbar_wait(smem_u32(&sm.bar_mma), 1, nullptr, kWaitNs)) sm.fail = 3;
   }
   __syncthreads();
-  ok = *reinterpret_cast<volatile int*>(err) == 0;
-  if (ok) {
-    tc_fence_after();
-    uint32_t u[32];
-    for (int ch = 0; ch < 2; ++ch) {
-      tmem_ld32(la + 128 + ch * 32, u);
-      tmem_wait_ld();
-      for (int c = 0; c < 32; ++c) s1_out[tid * 64 + ch * 32 + c] = __uint_as_float(u[c]);
-      tmem_ld32(la + 192 + ch * 32, u);
-      tmem_wait_ld();
-      for (int c = 0; c < 32; ++c) s2_out[tid * 64 + ch * 32 + c] = __uint_as_float(u[c]);
-    }
-    for (int ch = 0; ch < 4; ++ch) {
-      tmem_ld32(la + ch * 32, u);
-      tmem_wait_ld();
-      for (int c = 0; c < 32; ++c) o_out[tid * 128 + ch * 32 + c] = __uint_as_float(u[c]);
-      tmem_ld32(la + 256 + ch * 32, u);
-      tmem_wait_ld();
-      for (int c = 0; c < 32; ++c) o2_out[tid * 128 + ch * 32 + c] = __uint_as_float(u[c]);
-    }
+  tc_fence_after();
+  if (sm.fail) {
+    if (threadIdx.x == 0) *err = sm.fail;
+  } else {
+    const uint32_t q0 = tm + (static_cast<uint32_t>(warp * 32) << 16);
+    store_rows128(q0 + (16u << 16) + 384, o64, 16 * warp);
+    store_rows128(q0 + 0, o128, 32 * warp);
+    store_rows128(q0 + (16u << 16) + 0, o128, 32 * warp + 16);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tm, kCols);
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  void* p = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-      q != cudaDriverEntryPointSuccess)
-    return nullptr;
-  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-}
-
-bool encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box) {
-  auto enc = encoder();
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return enc && enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
-                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-// q [128, 128], k [64, 128], v [64, 128], p [128, 64] bf16 row-major;
-// grid [T, Hg, W, 2 heads, 128] bf16; outputs fp32 s1 [128, 64], s2 [128, 64], o and o2 [128, 128].
-// Returns 0 on success, 1 for a wait that ran out, 2 for a CUDA error.
-extern "C" int mma_check_run(const void* q, const void* k, const void* v, const void* p, const void* grid,
-                             int T, int Hg, int W, int cube_t0, int cube_h0, int cube_w0, int cube_head,
-                             float* s1, float* s2, float* o, float* o2, int* err_dev) {
-  CUtensorMap tq, tk, tv, tg;
-  const cuuint32_t box3[3] = {64, 1, 64};
-  const cuuint64_t dq[3] = {128, 1, 128}, dk[3] = {128, 1, 64};
-  const cuuint64_t st3[2] = {256, 256};
-  if (!encode(&tq, 3, q, dq, st3, box3) || !encode(&tk, 3, k, dk, st3, box3) || !encode(&tv, 3, v, dk, st3, box3))
-    return 2;
-  const cuuint64_t dg[5] = {128, 2, static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(Hg), static_cast<cuuint64_t>(T)};
-  const cuuint64_t sg[4] = {256, 512, 512ull * W, 512ull * W * Hg};
-  const cuuint32_t box5[5] = {64, 1, 4, 4, 4};
-  if (!encode(&tg, 5, grid, dg, sg, box5)) return 2;
-  const size_t smem = sizeof(CheckSmem) + 1024;
-  if (cudaFuncSetAttribute(check_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
-    return 2;
-  cudaMemset(err_dev, 0, sizeof(int));
-  check_kernel<<<1, 128, smem>>>(tq, tk, tv, tg, cube_t0, cube_h0, cube_w0, cube_head,
-                                 static_cast<const uint16_t*>(p), s1, s2, o, o2, err_dev);
-  if (cudaDeviceSynchronize() != cudaSuccess) return 2;
-  int err = 0;
-  cudaMemcpy(&err, err_dev, sizeof(int), cudaMemcpyDeviceToHost);
-  return err;
+extern "C" int mma_check_run(const void* q, const void* qa, const void* qb, const void* k, const void* v,
+                             const void* p64, const void* p128, float* s64_0, float* s64_1, float* s128, float* o64,
+                             float* o128, int* err) {
+  const int smem = static_cast<int>(sizeof(Smem));
+  if (cudaFuncSetAttribute(mma_check_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return 1;
+  mma_check_kernel<<<1, 128, smem>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(qa),
+                                     static_cast<const uint8_t*>(qb), static_cast<const uint8_t*>(k),
+                                     static_cast<const uint8_t*>(v), static_cast<const uint16_t*>(p64),
+                                     static_cast<const uint16_t*>(p128), s64_0, s64_1, s128, o64, o128, err);
+  if (cudaGetLastError() != cudaSuccess) return 2;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 3;
+  return 0;
 }

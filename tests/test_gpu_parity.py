@@ -18,32 +18,43 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 # --------------------------------------------- tcgen05 building blocks ----
+def swizzled_tile(x):
+    """bf16 bits [64, 128] -> the 16 KB tile-major block the kernels copy:
+    d-half j, row r, 16-byte chunk c stored at j * 8 KB + r * 128 B + 16 (c ^ (r & 7))."""
+    x = np.ascontiguousarray(x).reshape(64, 2, 8, 8)          # (row, d half, chunk, element)
+    out = np.empty((2, 64, 8, 8), dtype=np.uint16)
+    for r in range(64):
+        out[:, r, np.arange(8) ^ (r & 7), :] = x[r]
+    return out.reshape(-1)
+
+
 def test_tcgen05_building_blocks(cuda_ok):
-    """One S = Q K^T (3-D and 5-D TMA maps), one O = P V (swizzled P, MN-major V),
-    and O = P V with P in TMEM."""
+    """S = Q K^T at M = 64 into both TMEM lane halves and at M = 128 on a query
+    pair (bulk-copied swizzled tiles), and O = P V with P written into TMEM
+    (M = 64 in lane half 1, and M = 128), against fp32 matmuls."""
     import torch
     lib = ctypes.CDLL(os.path.join(ROOT, "tests", "native", "libmma_check.so"))
     lib.mma_check_run.restype = ctypes.c_int
-    g = torch.Generator().manual_seed(0)
-    r = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16).cuda()
-    q, k, v, p = r(128, 128), r(64, 128), r(64, 128), r(128, 64)
-    T, Hg, Wd = 6, 5, 9
-    grid = r(T, Hg, Wd, 2, 128)
-    s1, s2, o, o2 = (torch.zeros(128, n, device="cuda") for n in (64, 64, 128, 128))
+    rng = np.random.default_rng(0)
+    bf = lambda *s: W.f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32))
+    q, qa, qb, k, v = bf(64, 128), bf(64, 128), bf(64, 128), bf(64, 128), bf(64, 128)
+    p64, p128 = W.f32_to_bf16_bits(rng.random((64, 64)).astype(np.float32)), \
+        W.f32_to_bf16_bits(rng.random((128, 64)).astype(np.float32))
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).cuda()
+    tq, tqa, tqb, tk, tv = (dev(swizzled_tile(x)) for x in (q, qa, qb, k, v))
+    tp64, tp128 = dev(p64), dev(p128)
+    outs = [torch.full(sh, float("nan"), device="cuda") for sh in ((64, 64), (64, 64), (128, 64), (64, 128),
+                                                                     (128, 128))]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    t0, h0, w0, head = 4, 4, 8, 1           # a cube cut by all three grid edges
-    rc = lib.mma_check_run(*(ctypes.c_void_p(x.data_ptr()) for x in (q, k, v, p, grid)),
-                           T, Hg, Wd, t0, h0, w0, head,
-                           *(ctypes.c_void_p(x.data_ptr()) for x in (s1, s2, o, o2, err)))
-    assert rc == 0
-    f = lambda x: x.float().cpu()
-    assert torch.allclose(f(s1), f(q) @ f(k).T, atol=1e-2, rtol=1e-3)
-    cube = torch.zeros(4, 4, 4, 128)
-    gc = f(grid)[t0:t0 + 4, h0:h0 + 4, w0:w0 + 4, head]
-    cube[: gc.shape[0], : gc.shape[1], : gc.shape[2]] = gc
-    assert torch.allclose(f(s2), f(q) @ cube.reshape(64, 128).T, atol=1e-2, rtol=1e-3)
-    assert torch.allclose(f(o), f(p) @ f(v), atol=1e-2, rtol=1e-3)
-    assert torch.allclose(f(o2), f(p) @ f(v), atol=1e-2, rtol=1e-3)     # A operand read from TMEM
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    rc = lib.mma_check_run(*(ptr(t) for t in (tq, tqa, tqb, tk, tv, tp64, tp128)), *(ptr(t) for t in outs), ptr(err))
+    assert rc == 0 and int(err.item()) == 0
+    f = lambda x: torch.from_numpy(O.bf16_bits_to_f64(x)).float()
+    s64_0, s64_1, s128, o64, o128 = (t.cpu() for t in outs)
+    ok = lambda got, want: torch.allclose(got, want, atol=1e-2, rtol=1e-3)
+    assert ok(s64_0, f(q) @ f(k).T) and ok(s64_1, f(q) @ f(k).T)
+    assert ok(s128, torch.cat([f(qa), f(qb)]) @ f(k).T)
+    assert ok(o64, f(p64) @ f(v)) and ok(o128, f(p128) @ f(v))
 
 
 # --------------------------------------------------------- full checks ----
