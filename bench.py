@@ -300,9 +300,7 @@ def measure_config(name, wl, params, q, k, v, g, dev, stream, out_dtype, peak, n
     with torch.cuda.stream(stream):
         fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, out_dtype=out_dtype, stream=stream)
         out = torch.empty(q.shape, dtype=out_dtype, device=dev)
-    sel_fn = lambda: vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
-    att_fn = lambda: vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
-                                         fwd.ws_attn, stream)
+    sel_fn, att_fn = call_fns(vsa, lay, params, fwd, q, k, v, g, out, stream)
     for _ in range(3):
         sel_fn()
         att_fn()
@@ -310,6 +308,9 @@ def measure_config(name, wl, params, q, k, v, g, dev, stream, out_dtype, peak, n
     idx, cnt = fwd.idx.cpu().numpy(), fwd.cnt.cpu().numpy()
     flop = valid_flop_fast(counts, lay.info.n_cond_tiles, idx, cnt, wl.sink == vsa.SINK_EXACT_KV_AND_ROWS,
                            wl.sink == vsa.SINK_OFF)
+    if params.extra_tokens > 0:
+        flop += valid_flop_extra(counts, fwd.extra_cnt.cpu().numpy(), wl.sink == vsa.SINK_EXACT_KV_AND_ROWS,
+                                 lay.info.n_cond_tiles)
     sel_ms, att_ms, calls = time_calls(stream, sel_fn, att_fn, n_calls)
     check_failures(fwd, stream, name)
     call_ms = statistics.median(calls)
@@ -326,6 +327,29 @@ def measure_config(name, wl, params, q, k, v, g, dev, stream, out_dtype, peak, n
     del fwd, out
     torch.cuda.empty_cache()
     return res
+
+
+def call_fns(vsa, lay, params, fwd, q, k, v, g, out, stream):
+    """The two timed halves of one call: selection (plus the extra-token
+    choice when params.extra_tokens > 0) and attention."""
+    def select():
+        vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
+        if params.extra_tokens > 0:
+            vsa.extra_tokens_select(lay, params, q, k, fwd.idx, fwd.cnt, fwd.kmax, fwd.extra_idx, fwd.extra_cnt,
+                                    fwd.ws_extra, stream)
+
+    def attend():
+        vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out, fwd.ws_attn,
+                            stream, fwd.extra_idx, fwd.extra_cnt)
+    return select, attend
+
+
+def valid_flop_extra(counts, extra_cnt, rows_dense, n_cond):
+    """FLOP of the extra-token key step: 4 * 128 per (valid query, extra token)."""
+    e = extra_cnt.astype(np.float64)
+    if rows_dense:
+        e[:, :, :n_cond] = 0
+    return 4.0 * 128.0 * float((e * counts[None, None, :].astype(np.float64)).sum())
 
 
 def run_ours(args):
@@ -356,20 +380,15 @@ def run_ours(args):
     q, k, v, g = (to_dev(x) for x in bits)
     stream = torch.cuda.Stream(device=dev)
     out_dtype = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
-    params = vsa.make_params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=COARSES[args.coarse])
+    params = vsa.make_params(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=COARSES[args.coarse],
+                             extra_tokens=args.extra_tokens)
     with torch.cuda.stream(stream):
         fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, out_dtype=out_dtype, stream=stream)
         out = torch.empty(q.shape, dtype=out_dtype, device=dev)
     torch.cuda.synchronize()
     peaks, src = measured_peaks()
     peak = peaks["bf16_tflops"]
-
-    def select():
-        vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
-
-    def attend():
-        vsa.sparse_attn_fwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, out,
-                            fwd.ws_attn, stream)
+    select, attend = call_fns(vsa, lay, params, fwd, q, k, v, g, out, stream)
 
     def step():
         select()
@@ -380,6 +399,9 @@ def run_ours(args):
     check_failures(fwd, stream, "warm-up")
     flop = valid_flop_fast(counts, lay.info.n_cond_tiles, fwd.idx.cpu().numpy(), fwd.cnt.cpu().numpy(),
                            wl.sink == vsa.SINK_EXACT_KV_AND_ROWS, wl.sink == vsa.SINK_OFF)
+    if args.extra_tokens > 0:
+        flop += valid_flop_extra(counts, fwd.extra_cnt.cpu().numpy(), wl.sink == vsa.SINK_EXACT_KV_AND_ROWS,
+                                 lay.info.n_cond_tiles)
 
     def barrier():
         torch.cuda.synchronize()
@@ -436,9 +458,9 @@ def run_ours(args):
         if i >= 2:
             stream.wait_event(ev_out[bsel])              # the output of step i - 2 has been read back
         qq, kk, vv, gg = dev_in[bsel]
-        vsa.coarse_select(lay, params, qq, kk, vv, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
-        vsa.sparse_attn_fwd(lay, params, qq, kk, vv, gg, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, dev_out[bsel],
-                            fwd.ws_attn, stream)
+        s_fn, a_fn = call_fns(vsa, lay, params, fwd, qq, kk, vv, gg, dev_out[bsel], stream)
+        s_fn()
+        a_fn()
         ev_done[bsel].record(stream)
         s_out.wait_event(ev_done[bsel])
         with torch.cuda.stream(s_out):
@@ -453,16 +475,20 @@ def run_ours(args):
     # ---- the other configurations of the same shapes, measured in the same run (rank 0, one GPU)
     configs = None
     if world == 1 and not args.no_configs and args.workload == "5s" and args.sink is None \
-            and args.coarse == "mean" and args.gate == "token":
+            and args.coarse == "mean" and args.gate == "token" and args.extra_tokens == 0:
         configs = {}
         n = args.config_calls
-        mk = lambda **kw: vsa.make_params(**dict(dict(mode=0, keep=0.1, tau=1.0, sink=0, coarse=0), **kw))
+        mk = lambda **kw: vsa.make_params(**dict(dict(mode=0, keep=0.1, tau=1.0, sink=0, coarse=0, extra_tokens=0),
+                                                 **kw))
         note = "the 5 s inputs of this run (seed %d)" % wl.seed
         for tau in (1.0, 1.5, 2.0):
             configs["5s_adaptive_tau%g" % tau] = measure_config(
                 "adaptive tau %g" % tau, wl.with_(mode=vsa.SELECT_ADAPTIVE, tau=tau),
                 mk(mode=vsa.SELECT_ADAPTIVE, tau=tau), q, k, v, g, dev, stream, out_dtype, peak, n,
                 inputs_note=note)
+        configs["5s_extra_tokens16"] = measure_config(
+            "extra tokens 16", wl, mk(extra_tokens=16), q, k, v, g, dev, stream, out_dtype, peak, max(3, n // 2),
+            inputs_note=note)
         configs["5s_keep100"] = measure_config("keep 100%", wl.with_(keep=1.0), mk(keep=1.0), q, k, v, g, dev,
                                                stream, out_dtype, peak, max(3, n // 2), dense=dense_ms,
                                                inputs_note=note)
@@ -495,7 +521,9 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": describe(wl) + ", %s coarse, %s gate, %s output" % (args.coarse, args.gate, args.out_dtype),
+            "config": {"workload": describe(wl) + ", %s coarse, %s gate, %s output%s" % (
+                args.coarse, args.gate, args.out_dtype,
+                ", %d extra tokens" % args.extra_tokens if args.extra_tokens else ""),
                        "B": wl.B, "seq_len": wl.seq_len, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
                        "l2": "inputs (2.5 GB) larger than L2; no flush"},
             "roofline": {"bound": "tensor", "kernel": "vsa_attn_kernel", "achieved": achieved, "peak": peak,
@@ -513,7 +541,8 @@ def run_ours(args):
             "e2e": {"value": job_flop / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                     "steps": e2e_steps, "copies": "overlap the neighbouring steps' compute"},
-            "gpu_launches": launches_per_call(wl.B, args.coarse) * args.steps * world,
+            "gpu_launches": launches_per_call(wl.B, args.coarse, wl.sink != vsa.SINK_OFF and lay.info.n_cond_tiles > 0,
+                                              args.extra_tokens > 0) * args.steps * world,
             "clocks": clocks.summary(),
             "call_ms": {"p50": call_p50, "p90": call_p90, "samples": len(call_ms)},
             "dense_sdpa": None if dense_ms is None else {
@@ -536,11 +565,13 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def launches_per_call(B: int, coarse: str) -> int:
+def launches_per_call(B: int, coarse: str, pair_pass: bool, extra: bool) -> int:
     """Kernels this library launches per call: selection (pool, coarse, select;
-    anchor and reweight with Spark-Reweight) and attention (permute, schedule,
-    one attention launch per batch)."""
-    return 3 + (2 if coarse == "reweight" else 0) + 2 + B
+    anchor and reweight with Spark-Reweight; permute K, pool Q and the token
+    ranking with extra tokens) and attention (permute, schedule, the pair pass
+    and the sparse pass per batch, plus the extra-token gather)."""
+    sel = 3 + (2 if coarse == "reweight" else 0) + (3 if extra else 0)
+    return sel + 2 + (1 if extra else 0) + B * (2 if pair_pass else 1)
 
 
 def main():
@@ -557,6 +588,8 @@ def main():
                     help="gate g[B,S,H] (one per token and head) or g[B,S,H,128] (one per channel)")
     ap.add_argument("--coarse", choices=sorted(COARSES), default="mean",
                     help="compressed-branch summaries: mean pooling or Spark-Reweight")
+    ap.add_argument("--extra-tokens", type=int, default=0,
+                    help="extra_tokens E (0..64): the E best tokens beyond each query tile's selected tiles")
     ap.add_argument("--ref-tiles", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the torch SDPA comparator")

@@ -137,6 +137,9 @@ struct AttnArgs {
   int2* sched;               // step records: [b][item][max_steps]
   int32_t* nsteps;           // steps per (b, item)
   int32_t max_steps;
+  int32_t n_extra;           // extra_tokens E (0: none)
+  const int32_t* extra_cnt;  // [B, H, n_tiles] tokens chosen per query tile
+  const uint8_t* extra_kv;   // their K and V as one tile-major tile per (b, h, query tile), 32 KB
   int32_t merge_prefix;      // merge the pair pass's partial output over the conditioning keys
   const float* part_o;       // [B, H, n_tiles, 64, 128] normalised partial output
   const float* part_lse;     // [B, H, n_tiles, 64] its log2-sum-exp2 (scaled log2 domain)
@@ -274,6 +277,36 @@ permute_qkv_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* 
   }
 }
 
+// The extra tokens of each sparsely attended query tile gathered into one
+// tile-major K/V tile (same layout as permute_qkv_kernel's; slots past the
+// token count zero): extra_kv[((b * H + h) * n_tiles + qt) * 32 KB + ...].
+// grid (query tiles from c0, H, B). Token indices outside [0, S) are skipped.
+__global__ void __launch_bounds__(256)
+gather_extra_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int64_t sb, int64_t ss,
+                    int64_t sh, int H, int n_tiles, int c0, int64_t seq_len, const int32_t* __restrict__ extra_idx,
+                    const int32_t* __restrict__ extra_cnt, int E, uint8_t* __restrict__ extra_kv) {
+  const int qt = c0 + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t row = (static_cast<size_t>(b) * H + h) * n_tiles + qt;
+  __shared__ int tok[kTile];
+  const int n = min(max(extra_cnt[row], 0), E);
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) {
+    const int t = i < n ? extra_idx[row * E + i] : -1;
+    tok[i] = (t >= 0 && t < seq_len) ? t : -1;
+  }
+  __syncthreads();
+  for (int w = threadIdx.x; w < 2048; w += blockDim.x) {   // (tensor, d-half, row, chunk)
+    const int pc = w & 7, r = (w >> 3) & 63, j = (w >> 9) & 1, which = w >> 10;
+    const int t = tok[r];
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= 0) {
+      const uint16_t* src = (which ? v : k) + b * sb + static_cast<int64_t>(t) * ss + h * sh + j * 64 +
+                            ((pc ^ (r & 7)) << 3);
+      val = __ldg(reinterpret_cast<const uint4*>(src));
+    }
+    *reinterpret_cast<uint4*>(extra_kv + row * 32768u + which * 16384 + j * 8192 + r * 128 + pc * 16) = val;
+  }
+}
+
 // Step schedule of each work item, built once per call so that the copy warps
 // of the attention kernel only stream records. Record = (key tile, flags): bit 4
 // last step of the item, bit 5 the key tile has padding slots. Key tiles are the
@@ -288,17 +321,26 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const __grid_co
   const size_t row = (static_cast<size_t>(b) * a.H + it.h) * G.n_tiles + it.qt;
   // lists from vsa_coarse_select hold 1..kmax entries; anything else is clamped
   const int n = min(max(a.cnt[row], 1), a.kmax);
+  // extra tokens: one more step over the query tile's gathered tile, whose
+  // record holds the token count instead of a tile (flag bit 6)
+  const int n_e = a.n_extra > 0 ? min(max(a.extra_cnt[row], 0), a.n_extra) : 0;
+  const int total = n + (n_e > 0 ? 1 : 0);
   int2* rec = a.sched + (static_cast<size_t>(b) * a.n_items + item) * a.max_steps;
-  for (int r = threadIdx.x; r < n; r += kSchedThreads) {
-    // entries outside [0, n_cand) (never written by vsa_coarse_select) are clamped: memory stays in bounds
-    const int c = a.idx[row * a.kmax + r];
-    const int t = a.cand0 + min(max(c, 0), a.n_cand - 1);
-    uint32_t fl = 0u;
-    if (r == n - 1) fl |= 16u;
-    if (a.valid[t] != ~0ull) fl |= 32u;
+  for (int r = threadIdx.x; r < total; r += kSchedThreads) {
+    uint32_t fl = r == total - 1 ? 16u : 0u;
+    int t;
+    if (r < n) {
+      // entries outside [0, n_cand) (never written by vsa_coarse_select) are clamped: memory stays in bounds
+      const int c = a.idx[row * a.kmax + r];
+      t = a.cand0 + min(max(c, 0), a.n_cand - 1);
+      if (a.valid[t] != ~0ull) fl |= 32u;
+    } else {
+      t = n_e;
+      fl |= 64u;
+    }
     rec[r] = make_int2(t, static_cast<int>(fl));
   }
-  if (threadIdx.x == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = n;
+  if (threadIdx.x == 0) a.nsteps[static_cast<size_t>(b) * a.n_items + item] = total;
 }
 
 // At most 128 registers per thread: each of an SM's four sub-partitions has its
@@ -360,8 +402,12 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
       const size_t bi = static_cast<size_t>(a.b) * a.n_items + item;
       const int2* rec = a.sched + bi * a.max_steps;
       const int n = a.nsteps[bi];
-      const int h = decode_item(a, item).h;
+      const Item itm = decode_item(a, item);
+      const int h = itm.h;
       const uint8_t* head_kv = a.kv + (static_cast<size_t>(a.b) * a.H + h) * G.n_tiles * 32768u + (is_k ? 0u : 16384u);
+      const uint8_t* extra_kv = a.n_extra > 0 ? a.extra_kv + ((static_cast<size_t>(a.b) * a.H + h) * G.n_tiles + itm.qt) *
+                                                                 32768u + (is_k ? 0u : 16384u)
+                                              : nullptr;
       // records 32 at a time, one per lane, the next 32 prefetched
       int2 cur = lane < n ? rec[lane] : make_int2(0, 0);
       int2 nxt = 32 + lane < n ? rec[32 + lane] : make_int2(0, 0);
@@ -375,17 +421,18 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
         const int st = step & 1;
         if (step >= 2 && !(ok = warp_wait(sm, freed[st], ((step >> 1) - 1) & 1, lane, a.err))) break;
         if (lane == 0) {
+          const bool extra = (fl & 64) != 0;     // the gathered extra-token tile; `tile` is its token count
           if (is_k) {
             StageInfo& inf = sm.info[step % kInfoSlots];
             inf.tile = tile;
             inf.last = (fl >> 4) & 1;
-            inf.valid = (fl & 32) ? a.valid[tile] : ~0ull;
+            inf.valid = extra ? (tile >= 64 ? ~0ull : ((1ull << tile) - 1ull)) : ((fl & 32) ? a.valid[tile] : ~0ull);
             mbar_arrive(smem_u32(&sm.info_full[step % kInfoSlots]));
           }
           const uint32_t bar = smem_u32(&full[st]);
           mbar_arrive_expect_tx(bar, kTileBytes);
-          bulk_load(smem_u32(is_k ? sm.k[st] : sm.v[st]), head_kv + static_cast<size_t>(tile) * 32768u, kTileBytes,
-                    bar);
+          bulk_load(smem_u32(is_k ? sm.k[st] : sm.v[st]),
+                    extra ? extra_kv : head_kv + static_cast<size_t>(tile) * 32768u, kTileBytes, bar);
         }
         __syncwarp();
         ++issued;
@@ -1141,7 +1188,7 @@ Passes passes(const vsa_layout* L, const vsa_params* p, int32_t kmax) {
   const bool rows = p->sink == VSA_SINK_EXACT_KV_AND_ROWS;
   s.c0 = rows ? L->n_cond : 0;
   s.nq = L->n_tiles - s.c0;
-  s.max_steps = std::max(1, std::min(kmax, candidates(L, p->sink).count));
+  s.max_steps = std::max(1, std::min(kmax, candidates(L, p->sink).count)) + (p->extra_tokens > 0 ? 1 : 0);
   s.n_dpairs = rows ? (L->n_cond + 1) / 2 : 0;
   s.n_ppairs = (p->sink != VSA_SINK_OFF && L->n_cond > 0) ? (s.nq + 1) / 2 : 0;
   s.merge_prefix = s.n_ppairs > 0;
@@ -1149,8 +1196,9 @@ Passes passes(const vsa_layout* L, const vsa_params* p, int32_t kmax) {
 }
 
 // [header][tile-major K/V][tile-major Q][step records][steps per item][partial output][partial log-sum-exp]
+// [extra-token tiles]
 struct AttnWorkspace {
-  size_t kv, qtm, sched, nsteps, part_o, part_lse, total;
+  size_t kv, qtm, sched, nsteps, part_o, part_lse, extra_kv, total;
 };
 
 AttnWorkspace attn_workspace(const vsa_layout* L, int B, int H, const vsa_params* p) {
@@ -1167,7 +1215,8 @@ AttnWorkspace attn_workspace(const vsa_layout* L, int B, int H, const vsa_params
   w.nsteps = w.sched + align_up(items * s.max_steps * sizeof(int2), 256);
   w.part_o = w.nsteps + align_up(items * sizeof(int32_t), 256);
   w.part_lse = w.part_o + (s.merge_prefix ? tiles * kTile * kHeadDim * sizeof(float) : 0);
-  w.total = w.part_lse + align_up(s.merge_prefix ? tiles * kTile * sizeof(float) : 0, 256);
+  w.extra_kv = w.part_lse + align_up(s.merge_prefix ? tiles * kTile * sizeof(float) : 0, 256);
+  w.total = w.extra_kv + (p->extra_tokens > 0 ? tiles * 2 * kTileBytes : 0);
   return w;
 }
 
@@ -1191,7 +1240,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
                                const void* q, const void* k, const void* v, int64_t sb, int64_t ss,
                                int64_t sh, const void* g, int64_t g_sb, int64_t g_ss, int64_t g_sh,
                                int64_t g_sd, const int32_t* idx, const int32_t* cnt, int32_t kmax,
-                               const float* o_coarse, void* out, int32_t out_dtype, int64_t o_sb,
+                               const float* o_coarse, const int32_t* extra_idx, const int32_t* extra_cnt,
+                               void* out, int32_t out_dtype, int64_t o_sb,
                                int64_t o_ss, int64_t o_sh, void* workspace, size_t workspace_bytes,
                                cudaStream_t stream) {
   if (!L) return VSA_ERR_INVALID_ARG;
@@ -1200,6 +1250,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   st = check_qkv(q, k, v, sb, ss, sh, B, H);
   if (st != VSA_OK) return st;
   if (!g || !idx || !cnt || !o_coarse || !out || !workspace) return VSA_ERR_INVALID_ARG;
+  if (p->extra_tokens > 0 && (!extra_idx || !extra_cnt)) return VSA_ERR_INVALID_ARG;
   if (out_dtype != VSA_OUT_F32 && out_dtype != VSA_OUT_BF16) return VSA_ERR_INVALID_ARG;
   if (g_sb < 0 || g_ss <= 0 || g_sh <= 0 || g_sd < 0 || o_sb < 0 || o_ss <= 0 || o_sh <= 0)
     return VSA_ERR_INVALID_ARG;
@@ -1248,6 +1299,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.n_items = ps.nq * H;
   a.max_steps = ps.max_steps;
   a.merge_prefix = ps.merge_prefix;
+  a.n_extra = p->extra_tokens;
+  a.extra_cnt = extra_cnt;
   a.valid = D.valid;
   a.idx = idx;
   a.cnt = cnt;
@@ -1272,6 +1325,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.nsteps = reinterpret_cast<int32_t*>(wsb + ws.nsteps);
   a.part_o = reinterpret_cast<const float*>(wsb + ws.part_o);
   a.part_lse = reinterpret_cast<const float*>(wsb + ws.part_lse);
+  a.extra_kv = wsb + ws.extra_kv;
 
   pairpass::Args pa{};
   pa.n_cond = L->n_cond;
@@ -1311,6 +1365,13 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
       sh, H, pa.n_items > 0 ? 1 : 0, wsb + ws.qtm, wsb + ws.kv);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: permute launch", e);
+  if (a.n_extra > 0 && ps.nq > 0) {
+    gather_extra_kernel<<<dim3(ps.nq, H, B), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), sb, ss, sh, H, L->n_tiles, ps.c0,
+        L->seq_len, extra_idx, extra_cnt, a.n_extra, wsb + ws.extra_kv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: extra-token gather launch", e);
+  }
   schedule_kernel<<<dim3(a.n_items, B), kSchedThreads, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: schedule launch", e);

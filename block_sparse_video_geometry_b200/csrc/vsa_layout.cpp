@@ -55,6 +55,7 @@ vsa_status check_params(const vsa_params* p) {
     return VSA_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return VSA_ERR_INVALID_ARG;
   if (p->coarse != VSA_COARSE_MEAN && p->coarse != VSA_COARSE_REWEIGHT) return VSA_ERR_INVALID_ARG;
+  if (p->extra_tokens < 0 || p->extra_tokens > VSA_MAX_EXTRA_TOKENS) return VSA_ERR_INVALID_ARG;
   return VSA_OK;
 }
 
@@ -293,7 +294,7 @@ const char* vsa_status_string(vsa_status s) {
   return "unknown status";
 }
 
-int32_t vsa_version(void) { return (1 << 16) | 2; }
+int32_t vsa_version(void) { return (1 << 16) | 3; }
 
 const char* vsa_last_error_detail(void) { return g_detail; }
 

@@ -23,6 +23,7 @@ SINK_EXACT_KV, SINK_EXACT_KV_AND_ROWS, SINK_OFF = 0, 1, 2
 COARSE_MEAN, COARSE_REWEIGHT = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 TILE, HEAD_DIM = 64, 128
+MAX_EXTRA_TOKENS = 64
 
 
 class VSAError(RuntimeError):
@@ -41,7 +42,8 @@ class Segment(ctypes.Structure):
 
 class Params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("keep", ctypes.c_float), ("tau", ctypes.c_float),
-                ("sink", ctypes.c_int32), ("scale", ctypes.c_float), ("coarse", ctypes.c_int32)]
+                ("sink", ctypes.c_int32), ("scale", ctypes.c_float), ("coarse", ctypes.c_int32),
+                ("extra_tokens", ctypes.c_int32)]
 
 
 class LayoutInfo(ctypes.Structure):
@@ -69,8 +71,12 @@ _SIGNATURES = {
                                          _P, _P, _P, _P]),
     "vsa_sparse_attn_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
     "vsa_sparse_attn_fwd": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
-                                   _P, _I64, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _I64, _I64,
+                                   _P, _I64, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _P, _P, _I32, _I64, _I64,
                                    _I64, _P, _SZ, _P]),
+    "vsa_extra_tokens_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
+    "vsa_extra_tokens_select": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _I64, _I64, _I64,
+                                       _P, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "vsa_extra_tokens_status": (_I32, [_P, _P]),
     "vsa_sparse_attn_status": (_I32, [_P, _P]),
     "vsa_sparse_attn_workspace_init": (_I32, [_P, _P]),
     "vsa_sparse_attn_failed_calls": (_I32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -111,8 +117,8 @@ def _check(status: int, where: str) -> None:
 
 
 def make_params(mode: int = SELECT_TOPK, keep: float = 0.1, tau: float = 1.0,
-                sink: int = SINK_EXACT_KV, scale: float = 0.0, coarse: int = 0) -> Params:
-    return Params(mode, keep, tau, sink, scale, coarse)
+                sink: int = SINK_EXACT_KV, scale: float = 0.0, coarse: int = 0, extra_tokens: int = 0) -> Params:
+    return Params(mode, keep, tau, sink, scale, coarse, extra_tokens)
 
 
 def _stream_handle(stream) -> int:
@@ -179,6 +185,12 @@ class Layout:
                "vsa_coarse_select_workspace_size")
         return n.value
 
+    def extra_tokens_workspace_size(self, B: int, H: int, params: Params) -> int:
+        n = _SZ()
+        _check(lib().vsa_extra_tokens_workspace_size(self._h, B, H, ctypes.byref(params), ctypes.byref(n)),
+               "vsa_extra_tokens_workspace_size")
+        return n.value
+
     def sparse_attn_workspace_size(self, B: int, H: int, params: Params) -> int:
         n = _SZ()
         _check(lib().vsa_sparse_attn_workspace_size(self._h, B, H, ctypes.byref(params), ctypes.byref(n)),
@@ -216,10 +228,28 @@ def coarse_select_noalloc(layout: Layout, params: Params, q, k, v, idx, cnt, o_c
            "vsa_coarse_select_noalloc")
 
 
+def extra_tokens_select(layout: Layout, params: Params, q, k, idx, cnt, kmax: int, extra_idx, extra_cnt,
+                        workspace, stream=None) -> None:
+    """vsa_extra_tokens_select: extra_idx int32 [B, H, n_tiles, E], extra_cnt int32 [B, H, n_tiles] out."""
+    B, S, H, _ = q.shape
+    sb, ss, sh = _qkv_strides(q, k, k)
+    _check(lib().vsa_extra_tokens_select(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
+                                         sb, ss, sh, idx.data_ptr(), cnt.data_ptr(), kmax, extra_idx.data_ptr(),
+                                         extra_cnt.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel() * workspace.element_size(), _stream_handle(stream)),
+           "vsa_extra_tokens_select")
+
+
+def extra_tokens_status(workspace, stream=None) -> int:
+    """Synchronises the stream; the status word of the extra-token selection (OK or ERR_TIMEOUT)."""
+    return lib().vsa_extra_tokens_status(workspace.data_ptr(), _stream_handle(stream))
+
+
 def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: int, o_coarse, out,
-                    workspace, stream=None) -> None:
+                    workspace, stream=None, extra_idx=None, extra_cnt=None) -> None:
     """vsa_sparse_attn_fwd on torch tensors; out is float32 or bfloat16 [B, S, H, 128];
-    g is bf16 [B, S, H] (one gate per token and head) or [B, S, H, 128] (one per channel)."""
+    g is bf16 [B, S, H] (one gate per token and head) or [B, S, H, 128] (one per channel);
+    extra_idx / extra_cnt from extra_tokens_select when params.extra_tokens > 0."""
     import torch
     B, S, H, _ = q.shape
     if g.dim() == 3:
@@ -238,6 +268,8 @@ def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: 
     _check(lib().vsa_sparse_attn_fwd(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
                                      v.data_ptr(), sb, ss, sh, g.data_ptr(), g.stride(0), g.stride(1),
                                      g.stride(2), g_sd, idx.data_ptr(), cnt.data_ptr(), kmax, o_coarse.data_ptr(),
+                                     None if extra_idx is None else extra_idx.data_ptr(),
+                                     None if extra_cnt is None else extra_cnt.data_ptr(),
                                      out.data_ptr(), od, out.stride(0), out.stride(1), out.stride(2),
                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                      _stream_handle(stream)), "vsa_sparse_attn_fwd")
@@ -291,6 +323,12 @@ class Forward:
         sparse_attn_workspace_init(self.ws_attn, stream)
         self.out_dtype = out_dtype or torch.float32
         self.stream = stream
+        self.extra_idx = self.extra_cnt = self.ws_extra = None
+        if params.extra_tokens > 0:
+            self.extra_idx = torch.empty((B, H, info.n_tiles, params.extra_tokens), dtype=torch.int32, device=device)
+            self.extra_cnt = torch.empty((B, H, info.n_tiles), dtype=torch.int32, device=device)
+            self.ws_extra = torch.empty(layout.extra_tokens_workspace_size(B, H, params), dtype=torch.uint8,
+                                        device=device)
 
     def __call__(self, q, k, v, g, out=None):
         import torch
@@ -298,8 +336,11 @@ class Forward:
             out = torch.empty(q.shape, dtype=self.out_dtype, device=q.device)
         coarse_select(self.layout, self.params, q, k, v, self.idx, self.cnt, self.o_coarse, self.ws_select,
                       self.stream)
+        if self.params.extra_tokens > 0:
+            extra_tokens_select(self.layout, self.params, q, k, self.idx, self.cnt, self.kmax, self.extra_idx,
+                                self.extra_cnt, self.ws_extra, self.stream)
         sparse_attn_fwd(self.layout, self.params, q, k, v, g, self.idx, self.cnt, self.kmax, self.o_coarse,
-                        out, self.ws_attn, self.stream)
+                        out, self.ws_attn, self.stream, self.extra_idx, self.extra_cnt)
         return out
 
     def pooled(self):

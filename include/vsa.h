@@ -46,6 +46,7 @@ extern "C" {
 #define VSA_TILE 64
 #define VSA_HEAD_DIM 128
 #define VSA_MAX_SEGMENTS 64
+#define VSA_MAX_EXTRA_TOKENS 64
 
 typedef enum {
   VSA_OK = 0,
@@ -118,7 +119,10 @@ typedef enum { VSA_COARSE_MEAN = 0, VSA_COARSE_REWEIGHT = 1 } vsa_coarse_mode;
  *  tau   : >= 0, used by ADAPTIVE.
  *  sink  : vsa_sink_mode.
  *  scale : softmax scale of both branches; <= 0 selects 1/sqrt(128).
- *  coarse: vsa_coarse_mode. */
+ *  coarse: vsa_coarse_mode.
+ *  extra_tokens: 0, or E in [1, VSA_MAX_EXTRA_TOKENS]: the E best individual
+ *          tokens outside a query tile's selected tiles join its exact key set
+ *          (see vsa_extra_tokens_select). */
 typedef struct {
   int32_t mode;
   float keep;
@@ -126,6 +130,7 @@ typedef struct {
   int32_t sink;
   float scale;
   int32_t coarse;
+  int32_t extra_tokens;
 } vsa_params;
 
 typedef struct vsa_layout vsa_layout;   /* opaque; owns its host tables */
@@ -260,6 +265,48 @@ vsa_status vsa_coarse_select_noalloc(const vsa_layout* layout, const vsa_params*
                                      cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* extra_tokens                                                              */
+/* ------------------------------------------------------------------------ */
+
+vsa_status vsa_extra_tokens_workspace_size(const vsa_layout* layout, int32_t B, int32_t H,
+                                           const vsa_params* params, size_t* bytes);
+
+/* vsa_extra_tokens_select: the extra key tokens of every query tile
+ * ("ComfyUI Agrega Nodo Central de Atencion Dispersa y Compilador Comfy",
+ * section "Atencion dispersa por bloques": extra_tokens adds the best-scoring
+ * tokens beyond the selected blocks, to stay closer to dense attention).
+ * Reading: for a query tile qt attended sparsely (every tile except dense
+ * conditioning rows under EXACT_KV_AND_ROWS), the candidate tokens are the
+ * valid tokens of the candidate key tiles qt did not select; token i scores
+ * scale * <mean Q of tile qt, k_i>; the E = params->extra_tokens highest, ties
+ * to the lower token index, are chosen (fewer when fewer candidates exist).
+ *
+ *  q, k, strides  : as vsa_coarse_select (v is not read).
+ *  idx, cnt, kmax : the lists of vsa_coarse_select with the same params.
+ *  extra_idx      : int32 [B, H, n_tiles, E] out: token indices, unordered;
+ *                   entries past extra_cnt unspecified.
+ *  extra_cnt      : int32 [B, H, n_tiles] out: number of tokens chosen (0 for
+ *                   dense conditioning rows).
+ *  workspace      : vsa_extra_tokens_workspace_size bytes, 256-byte aligned;
+ *                   its first word is the status that vsa_extra_tokens_status
+ *                   reads (a kernel wait that ran out).
+ * Scores: fp32 accumulation of the exact bf16 keys against the fp32 pooled
+ * query split into three bf16 terms (tensor cores), so the chosen set matches
+ * an fp64 evaluation except where two scores tie within fp32 rounding.
+ * Errors: INVALID_ARG when params->extra_tokens is 0 (nothing to choose). */
+vsa_status vsa_extra_tokens_select(const vsa_layout* layout, const vsa_params* params,
+                                   int32_t B, int32_t H, const void* q, const void* k,
+                                   int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                                   const int32_t* idx, const int32_t* cnt, int32_t kmax,
+                                   int32_t* extra_idx, int32_t* extra_cnt,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream` and reads the status word a previous
+ * vsa_extra_tokens_select left in `workspace`: VSA_OK or VSA_ERR_TIMEOUT. No
+ * counterpart on the pages (error reporting of this library). */
+vsa_status vsa_extra_tokens_status(const void* workspace, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Fine branch + gate combine                                                */
 /* ------------------------------------------------------------------------ */
 
@@ -283,6 +330,9 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* layout, int32_t B, i
  *                     "Technical Architecture").
  *  idx, cnt, kmax   : lists from vsa_coarse_select (same params).
  *  o_coarse         : float [B, H, n_tiles, 128] from vsa_coarse_select.
+ *  extra_idx,       : the lists of vsa_extra_tokens_select (same params) when
+ *  extra_cnt          params->extra_tokens > 0, else NULL; a query tile's
+ *                     extra tokens join its exact key set.
  *  out              : [B, S, H, 128] of out_dtype (vsa_out_dtype) at element
  *                     strides out_stride_*, head_dim contiguous; every valid
  *                     token row is written.
@@ -306,6 +356,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* layout, const vsa_params* param
                                int64_t g_stride_h, int64_t g_stride_d,
                                const int32_t* idx, const int32_t* cnt, int32_t kmax,
                                const float* o_coarse,
+                               const int32_t* extra_idx, const int32_t* extra_cnt,
                                void* out, int32_t out_dtype, int64_t out_stride_b,
                                int64_t out_stride_s, int64_t out_stride_h,
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);

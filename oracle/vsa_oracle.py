@@ -476,20 +476,22 @@ def selection_for_head(q, k, v, layout: Layout, params: Params):
 
 
 def output_rows_for_tile(q, k, v, g, layout: Layout, params: Params, qt: int,
-                         selected: np.ndarray, o_coarse: np.ndarray, scale: float):
+                         selected: np.ndarray, o_coarse: np.ndarray, scale: float, extra=None):
     """o_fine and out for the valid query tokens of tile qt.
 
     out = o_fine + g * o_coarse[qt], g [S] (one gate per token, broadcast over
     the head dimension) or [S, D] (one per channel); under exact_kv_and_rows
     the conditioning query rows get the dense result only (no coarse term;
     reading: they are run dense, and dense attention has no compressed branch).
-    Returns (tokens, o_fine, out).
+    `extra`, if given, is the tile's set of extra tokens (instead of the one
+    extra_tokens_for_tile chooses). Returns (tokens, o_fine, out).
     """
     keys = key_tokens_for_tile(layout, qt, selected, params.sink)
     if params.extra_tokens > 0 and not (params.sink == SINK_EXACT_KV_AND_ROWS and qt < layout.n_cond_tiles):
-        qbar_qt = np.asarray(q, dtype=np.float64)[layout.tile_tokens(qt)].mean(axis=0)
-        extra = extra_tokens_for_tile(qbar_qt, k, layout, selected, params.extra_tokens, scale, params.sink)
-        keys = np.concatenate([keys, extra])
+        if extra is None:
+            qbar_qt = np.asarray(q, dtype=np.float64)[layout.tile_tokens(qt)].mean(axis=0)
+            extra = extra_tokens_for_tile(qbar_qt, k, layout, selected, params.extra_tokens, scale, params.sink)
+        keys = np.concatenate([keys, np.asarray(extra, dtype=np.int64)])
     of = fine_branch_tile(q, k, v, layout, qt, keys, scale)
     toks = layout.tile_tokens(qt)
     if params.sink == SINK_EXACT_KV_AND_ROWS and qt < layout.n_cond_tiles:

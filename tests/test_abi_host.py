@@ -135,7 +135,8 @@ def test_calls_validate_before_any_gpu_work():
     n = ctypes.c_size_t()
     for bad in [vsa.make_params(keep=0.0), vsa.make_params(keep=1.5), vsa.make_params(mode=3),
                 vsa.make_params(sink=5), vsa.make_params(sink=3), vsa.make_params(coarse=2), vsa.make_params(mode=vsa.SELECT_ADAPTIVE, tau=-1.0),
-                vsa.make_params(scale=float("nan"))]:
+                vsa.make_params(scale=float("nan")), vsa.make_params(extra_tokens=-1),
+                vsa.make_params(extra_tokens=vsa.MAX_EXTRA_TOKENS + 1)]:
         assert L.vsa_coarse_select_workspace_size(lay.handle, 1, 2, ctypes.byref(bad), ctypes.byref(n)) == \
             vsa.ERR_INVALID_ARG
     assert L.vsa_coarse_select_workspace_size(lay.handle, 1, 2, ctypes.byref(good), ctypes.byref(n)) == vsa.OK
@@ -159,19 +160,36 @@ def test_calls_validate_before_any_gpu_work():
     common = (lay.handle, ctypes.byref(good), 1, 2, fake, fake, fake, args["sb"], args["ss"], args["sh"],
               fake, 2, 2 * S, 2, 0)
     # wrong kmax, bad out dtype, unaligned out stride, not uploaded
-    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, 7, S * 256, 256, 128, fake, 256,
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, None, None, fake, 7, S * 256, 256, 128, fake, 256,
                                  None) == vsa.ERR_INVALID_ARG
-    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_BF16, S * 256, 256, 129, fake,
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, None, None, fake, vsa.OUT_BF16, S * 256, 256, 129, fake,
                                  256, None) == vsa.ERR_INVALID_ARG
     # negative channel stride of the gate
-    assert L.vsa_sparse_attn_fwd(*common[:-1], -1, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128,
+    assert L.vsa_sparse_attn_fwd(*common[:-1], -1, fake, fake, kmax, fake, None, None, fake, vsa.OUT_F32, S * 256, 256, 128,
                                  fake, 1 << 30, None) == vsa.ERR_INVALID_ARG
     ws = lay.sparse_attn_workspace_size(1, 2, good)
     assert ws >= 256 + 2 * lay.info.n_tiles * 32768          # error word + tile-major K/V
-    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, None, None, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
                                  ws - 16, None) == vsa.ERR_WORKSPACE_TOO_SMALL
-    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
+    assert L.vsa_sparse_attn_fwd(*common, fake, fake, kmax, fake, None, None, fake, vsa.OUT_F32, S * 256, 256, 128, fake,
                                  ws, None) == vsa.ERR_NOT_UPLOADED
+    # extra_tokens: the lists are required when E > 0; the selection needs E > 0
+    ex = vsa.make_params(keep=0.5, extra_tokens=8)
+    ex_common = (lay.handle, ctypes.byref(ex)) + common[2:]
+    ws_x = lay.sparse_attn_workspace_size(1, 2, ex)
+    assert ws_x >= ws + 2 * lay.info.n_tiles * 32768           # one gathered K/V tile per (head, query tile)
+    assert L.vsa_sparse_attn_fwd(*ex_common, fake, fake, kmax, fake, None, None, fake, vsa.OUT_F32, S * 256, 256,
+                                 128, fake, ws_x, None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd(*ex_common, fake, fake, kmax, fake, fake, fake, fake, vsa.OUT_F32, S * 256, 256,
+                                 128, fake, ws_x, None) == vsa.ERR_NOT_UPLOADED
+    xs = lay.extra_tokens_workspace_size(1, 2, ex)
+    assert L.vsa_extra_tokens_select(lay.handle, ctypes.byref(good), 1, 2, fake, fake, args["sb"], args["ss"],
+                                     args["sh"], fake, fake, kmax, fake, fake, fake, xs, None) == vsa.ERR_INVALID_ARG
+    assert L.vsa_extra_tokens_select(lay.handle, ctypes.byref(ex), 1, 2, fake, fake, args["sb"], args["ss"],
+                                     args["sh"], fake, fake, kmax, fake, fake, fake, xs - 16, None) == \
+        vsa.ERR_WORKSPACE_TOO_SMALL
+    assert L.vsa_extra_tokens_select(lay.handle, ctypes.byref(ex), 1, 2, fake, fake, args["sb"], args["ss"],
+                                     args["sh"], fake, fake, kmax, fake, fake, fake, xs, None) == vsa.ERR_NOT_UPLOADED
 
 
 def test_layout_matches_oracle_on_random_descriptors():

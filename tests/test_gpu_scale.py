@@ -92,3 +92,25 @@ def test_5s_keep_all_equals_dense(cuda_ok):
             dense = O.softmax_attention(f(q[0, toks, h]), kk, vv, O.default_scale())
             err = np.abs(res["out"][0, toks, h] - dense)
             assert err.max() <= C.OUT_MAX_ABS and err.mean() <= C.OUT_MEAN_ABS
+
+
+def test_5s_extra_tokens(cuda_ok):
+    """extra_tokens at full size: the chosen sets of sampled query tiles against
+    the oracle's ranking over their ~116k candidate tokens, and their outputs."""
+    wl = W.WORKLOADS["5s"]
+    E = 16
+    lay = C.oracle_layout(wl)
+    q, k, v, g = C.inputs(wl, lay)
+    prm = C.params_of(wl, extra_tokens=E)
+    res = C.gpu_forward(wl, (q, k, v, g), prm)
+    assert res["status"] == vsa.OK and res["extra_status"] == vsa.OK
+    assert res["extra_cnt"].min() == E and res["extra_cnt"].max() == E
+    rng = np.random.default_rng(99)
+    for h in (2, 21):
+        ho = C.HeadOracle(wl, lay, (q, k, v, g), 0, h, prm)
+        near = C.compare_selection(ho, res["idx"][0, h], res["cnt"][0, h])
+        tiles = sorted(set(sample_tiles(lay, rng, 4)) | set(list(near)[:4]))
+        near_x = C.compare_extra(ho, res["extra_idx"][0, h], res["extra_cnt"][0, h], tiles, near)
+        C.note_near_ties(len(near_x))
+        gpu_extra = {qt: res["extra_idx"][0, h, qt, :E] for qt in tiles}
+        C.compare_outputs(ho, res, 0, h, tiles, near_tie=near, extra=gpu_extra)

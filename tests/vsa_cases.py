@@ -48,7 +48,7 @@ def inputs(wl, lay, channel_gate=False):
 
 
 def params_of(wl, **kw):
-    d = dict(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=O.COARSE_MEAN)
+    d = dict(mode=wl.mode, keep=wl.keep, tau=wl.tau, sink=wl.sink, coarse=O.COARSE_MEAN, extra_tokens=0)
     d.update(kw)
     return d
 
@@ -71,6 +71,10 @@ def gpu_forward(wl, bits, prm: dict, out_dtype="f32", layout=None):
     res = dict(status=st, idx=fwd.idx.cpu().numpy(), cnt=fwd.cnt.cpu().numpy(),
                o_coarse=fwd.o_coarse.cpu().numpy(), pooled=fwd.pooled().cpu().numpy(),
                out=out.float().cpu().numpy(), kmax=fwd.kmax)
+    if prm.get("extra_tokens", 0) > 0:
+        res["extra_status"] = vsa.extra_tokens_status(fwd.ws_extra)
+        res["extra_idx"] = fwd.extra_idx.cpu().numpy()
+        res["extra_cnt"] = fwd.extra_cnt.cpu().numpy()
     del fwd, tq, tk, tv, tg, out
     torch.cuda.empty_cache()
     return res
@@ -86,16 +90,27 @@ class HeadOracle:
         self.g = f(g[b, :, h])
         self.lay = lay
         self.p = O.Params(mode=prm["mode"], keep=prm["keep"], tau=prm["tau"], sink=prm["sink"],
-                          coarse=prm.get("coarse", O.COARSE_MEAN))
+                          coarse=prm.get("coarse", O.COARSE_MEAN), extra_tokens=prm.get("extra_tokens", 0))
         (self.qbar, self.kbar, self.vbar, self.scores, self.sel, self.thr, self.o_coarse,
          self.scale) = O.selection_for_head(self.q, self.k, self.v, lay, self.p)
 
-    def tile_out(self, qt, selected=None):
-        """Oracle rows of query tile qt; `selected` replaces the oracle's own
-        list (a near-tie row is checked on the list the GPU chose)."""
+    def tile_out(self, qt, selected=None, extra=None):
+        """Oracle rows of query tile qt; `selected` / `extra` replace the
+        oracle's own list / extra tokens (a near-tie row is checked on the
+        choice the GPU made)."""
         sel = self.sel[qt] if selected is None else np.asarray(selected, dtype=np.int64)
         return O.output_rows_for_tile(self.q, self.k, self.v, self.g, self.lay, self.p, qt,
-                                      sel, self.o_coarse, self.scale)
+                                      sel, self.o_coarse, self.scale, extra=extra)
+
+    def extra_scores(self, qt, selected):
+        """(candidate tokens, oracle scores) of query tile qt's extra-token
+        ranking given its selected tiles."""
+        first, count = O.candidate_tiles(self.lay, self.p.sink)
+        chosen = set(int(c) for c in selected)
+        toks = [self.lay.tile_tokens(first + c) for c in range(count) if c not in chosen]
+        toks = np.concatenate(toks) if toks else np.zeros(0, dtype=np.int64)
+        qbar = self.q[self.lay.tile_tokens(qt)].mean(axis=0)
+        return toks, self.scale * (self.k[toks] @ qbar)
 
 
 def check_lists_valid(res, lay, sink=O.SINK_EXACT_KV):
@@ -139,6 +154,37 @@ def compare_selection(ho: HeadOracle, gpu_idx, gpu_cnt):
     return near_tie
 
 
+def compare_extra(ho: HeadOracle, gpu_idx, gpu_cnt, tiles, near_sel=None):
+    """Checks the GPU's extra-token sets of the given query tiles against the
+    oracle's (ranked given the selection the GPU used). Returns {query tile: GPU
+    set} for sets that differ at a near-tie: same size, and every differing
+    token's oracle score within GAP of the E-th best score."""
+    near_sel = near_sel or {}
+    E = ho.p.extra_tokens
+    rows_dense = ho.p.sink == O.SINK_EXACT_KV_AND_ROWS
+    near = {}
+    for qt in tiles:
+        got = np.sort(gpu_idx[qt, : gpu_cnt[qt]])
+        if rows_dense and qt < ho.lay.n_cond_tiles:
+            assert gpu_cnt[qt] == 0
+            continue
+        sel = near_sel.get(qt, ho.sel[qt])
+        toks, sc = ho.extra_scores(qt, sel)
+        order = np.lexsort((toks, -sc))
+        want = np.sort(toks[order[:E]])
+        assert got.size == want.size, "query tile %d: %d extra tokens, want %d" % (qt, got.size, want.size)
+        if np.array_equal(got, want):
+            continue
+        edge = sc[order[want.size - 1]]
+        diff = np.setxor1d(got, want)
+        pos = {int(t): i for i, t in enumerate(toks)}
+        assert all(int(t) in pos for t in diff), "query tile %d: extra token outside the candidates" % qt
+        gaps = np.abs(sc[[pos[int(t)] for t in diff]] - edge)
+        assert np.all(gaps < GAP), "query tile %d: extra tokens differ away from the boundary" % qt
+        near[qt] = got
+    return near
+
+
 def out_error(got, want, bf16: bool):
     """(max excess over the bound, mean-abs error, mean bound) for one block of rows."""
     err = np.abs(got - want)
@@ -148,14 +194,17 @@ def out_error(got, want, bf16: bool):
     return float((err - half_ulp).max()), float(err.mean()), OUT_MEAN_ABS + float((half_ulp / 2).mean())
 
 
-def compare_outputs(ho: HeadOracle, res, b, h, tiles, bf16=False, near_tie=None):
+def compare_outputs(ho: HeadOracle, res, b, h, tiles, bf16=False, near_tie=None, extra=None):
     """Compares the GPU output rows of the given query tiles with the oracle.
     Rows in `near_tie` (from compare_selection) are compared with the oracle
-    evaluated on the GPU's list for that tile."""
+    evaluated on the GPU's list for that tile; with extra tokens, every row is
+    evaluated on the GPU's extra set (`extra`: {query tile: tokens}), which
+    compare_extra has checked against the oracle's."""
     near_tie = near_tie or {}
+    extra = extra or {}
     errs, means, bounds = [], [], []
     for qt in tiles:
-        toks, of, want = ho.tile_out(qt, near_tie.get(qt))
+        toks, of, want = ho.tile_out(qt, near_tie.get(qt), extra.get(qt))
         got = res["out"][b, toks, h]
         mx, mean, bound = out_error(got, want, bf16)
         errs.append(mx)
