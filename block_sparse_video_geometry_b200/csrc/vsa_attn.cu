@@ -143,6 +143,12 @@ struct AttnArgs {
   int32_t merge_prefix;      // merge the pair pass's partial output over the conditioning keys
   const float* part_o;       // [B, H, n_tiles, 64, 128] normalised partial output
   const float* part_lse;     // [B, H, n_tiles, 64] its log2-sum-exp2 (scaled log2 domain)
+  // statistics mode (the backward pass): instead of the output, write each
+  // query row's log2-sum-exp2 of the fine branch and D = <dO, o_fine>
+  float* st_lse;             // [B, H, n_tiles, 64] (+inf for padding rows), or null
+  float* st_d;               // [B, H, n_tiles, 64]
+  const uint16_t* dout;      // dO [B, S, H, 128] bf16 at element strides d_sb, d_ss, d_sh
+  int64_t d_sb, d_ss, d_sh;
   const float* o_coarse;
   const uint16_t* g;
   int64_t g_sb, g_ss, g_sh, g_sd;   // g_sd = 0: one gate per (token, head)
@@ -653,10 +659,13 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
       const float inv_l = 1.0f / (l_row * wf + wc);
       const float af = wf * inv_l, ac = wc * inv_l;
       const float* pc = a.part_o + prow * kHeadDim + 64 * hf;
+      const bool stats = a.st_lse != nullptr;
+      const uint16_t* drow = stats && row_ok ? a.dout + a.b * a.d_sb + tok * a.d_ss + it.h * a.d_sh + 64 * hf : nullptr;
+      float dsum = 0.f;
       float gate = 0.f;
       const float* oc = nullptr;
       const uint16_t* gp = nullptr;          // per-channel gate of this row (g_sd > 0)
-      if (row_ok) {
+      if (row_ok && !stats) {
         gp = a.g + a.b * a.g_sb + tok * a.g_ss + it.h * a.g_sh;
         gate = __uint_as_float(static_cast<uint32_t>(gp[0]) << 16);
         gp = kChannelGate ? gp + 64 * hf * a.g_sd : nullptr;
@@ -691,6 +700,18 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
               y[i + 2] = fmaf(t.z, ac, y[i + 2]);
               y[i + 3] = fmaf(t.w, ac, y[i + 3]);
             }
+          }
+          if (stats) {                         // D = <dO, o_fine>: this thread's 32 columns of the chunk
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 w = __ldg(reinterpret_cast<const uint4*>(drow + ch * 32) + u);
+              const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dsum = fmaf(__uint_as_float(wv[e] << 16), y[8 * u + 2 * e],
+                            fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), y[8 * u + 2 * e + 1], dsum));
+            }
+            continue;
           }
           if (kChannelGate && oc) {
             // this chunk's 32 gates as bf16 pairs (vector loads when the channels are contiguous)
@@ -742,6 +763,13 @@ __global__ void __maxnreg__(128) vsa_attn_kernel(const __grid_constant__ AttnArg
 #pragma unroll
             for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
           }
+        }
+      }
+      if (stats) {
+        const float d_row = dsum + __shfl_xor_sync(0xffffffffu, dsum, 16);
+        if (hf == 0) {
+          a.st_lse[prow] = row_ok ? mx + __log2f(l_row * wf + wc) : INFINITY;
+          a.st_d[prow] = row_ok ? d_row : 0.f;
         }
       }
       tc_fence_before();
@@ -808,6 +836,10 @@ struct Args {
   int32_t n_items;
   float* part_o;                    // [B, H, n_tiles, 64, 128] normalised partial output
   float* part_lse;                  // [B, H, n_tiles, 64] its log2-sum-exp2 (scaled log2 domain)
+  float* st_lse;                    // statistics mode (see AttnArgs): dense rows' log2-sum-exp2 and D, or null
+  float* st_d;
+  const uint16_t* dout;
+  int64_t d_sb, d_ss, d_sh;
   void* out;
   int32_t out_bf16;
   int64_t o_sb, o_ss, o_sh;
@@ -1117,6 +1149,9 @@ __global__ void __maxnreg__(80) pair_attn_kernel(const __grid_constant__ Args a)
       const float inv_l = 1.0f / l_row;
       const size_t poff = ((head0 + it.h) * a.n_tiles + (qtile >= 0 ? qtile : 0)) * kTile + slot;
       if (row_ok && !it.dense && hf == 0) a.part_lse[poff] = ms + __log2f(l_row);
+      const bool stats = it.dense && a.st_lse != nullptr;
+      const uint16_t* drow = stats && row_ok ? a.dout + a.b * a.d_sb + tok * a.d_ss + it.h * a.d_sh + 64 * hf : nullptr;
+      float dsum = 0.f;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         float y[16];
@@ -1126,7 +1161,17 @@ __global__ void __maxnreg__(80) pair_attn_kernel(const __grid_constant__ Args a)
 #pragma unroll
         for (int i = 0; i < 16; ++i) y[i] *= inv_l;
         const int col = 64 * hf + 16 * ch;
-        if (!it.dense) {
+        if (stats) {                           // D = <dO, o_fine> over this thread's columns
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4*>(drow + 16 * ch) + u);
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dsum = fmaf(__uint_as_float(wv[e] << 16), y[8 * u + 2 * e],
+                          fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), y[8 * u + 2 * e + 1], dsum));
+          }
+        } else if (!it.dense) {
           float4* dst = reinterpret_cast<float4*>(a.part_o + poff * kHeadDim + col);
 #pragma unroll
           for (int i = 0; i < 16; i += 4) dst[i / 4] = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
@@ -1143,6 +1188,13 @@ __global__ void __maxnreg__(80) pair_attn_kernel(const __grid_constant__ Args a)
 #pragma unroll
             for (int i = 0; i < 16; i += 4) dst[i / 4] = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
           }
+        }
+      }
+      if (stats && qtile >= 0) {
+        const float d_row = dsum + __shfl_xor_sync(0xffffffffu, dsum, 16);
+        if (hf == 0) {
+          a.st_lse[poff] = row_ok ? ms + __log2f(l_row) : INFINITY;
+          a.st_d[poff] = row_ok ? d_row : 0.f;
         }
       }
       // the next item's first O += P V overwrites O only after every softmax
@@ -1236,20 +1288,39 @@ vsa_status vsa_sparse_attn_workspace_size(const vsa_layout* L, int32_t B, int32_
   return VSA_OK;
 }
 
-vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H,
-                               const void* q, const void* k, const void* v, int64_t sb, int64_t ss,
-                               int64_t sh, const void* g, int64_t g_sb, int64_t g_ss, int64_t g_sh,
-                               int64_t g_sd, const int32_t* idx, const int32_t* cnt, int32_t kmax,
-                               const float* o_coarse, const int32_t* extra_idx, const int32_t* extra_cnt,
-                               void* out, int32_t out_dtype, int64_t o_sb,
-                               int64_t o_ss, int64_t o_sh, void* workspace, size_t workspace_bytes,
-                               cudaStream_t stream) {
+}  // extern "C"
+
+// The forward call; with `stats` (the backward pass) it writes each query
+// row's log2-sum-exp2 and D = <dO, o_fine> instead of the output (g, o_coarse
+// and out are then not read and may be null).
+vsa_status vsa::attn_forward(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H, const void* q,
+                             const void* k, const void* v, int64_t sb, int64_t ss, int64_t sh, const void* g,
+                             int64_t g_sb, int64_t g_ss, int64_t g_sh, int64_t g_sd, const int32_t* idx,
+                             const int32_t* cnt, int32_t kmax, const float* o_coarse, const int32_t* extra_idx,
+                             const int32_t* extra_cnt, void* out, int32_t out_dtype, int64_t o_sb, int64_t o_ss,
+                             int64_t o_sh, const AttnStats* stats, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
   if (!L) return VSA_ERR_INVALID_ARG;
   vsa_status st = check_params(p);
   if (st != VSA_OK) return st;
   st = check_qkv(q, k, v, sb, ss, sh, B, H);
   if (st != VSA_OK) return st;
-  if (!g || !idx || !cnt || !o_coarse || !out || !workspace) return VSA_ERR_INVALID_ARG;
+  if (!idx || !cnt || !workspace) return VSA_ERR_INVALID_ARG;
+  if (stats) {
+    // only the statistics are written: any aligned non-null stand-ins for the rest
+    static const uint16_t kZero[8] = {0};
+    if (!stats->lse || !stats->d || !stats->dout) return VSA_ERR_INVALID_ARG;
+    g = kZero;
+    g_sb = 0;
+    g_ss = g_sh = 1;
+    g_sd = 0;
+    o_coarse = reinterpret_cast<const float*>(workspace);
+    out = workspace;
+    out_dtype = VSA_OUT_F32;
+    o_sb = 0;
+    o_ss = o_sh = 4;
+  }
+  if (!g || !o_coarse || !out) return VSA_ERR_INVALID_ARG;
   if (p->extra_tokens > 0 && (!extra_idx || !extra_cnt)) return VSA_ERR_INVALID_ARG;
   if (out_dtype != VSA_OUT_F32 && out_dtype != VSA_OUT_BF16) return VSA_ERR_INVALID_ARG;
   if (g_sb < 0 || g_ss <= 0 || g_sh <= 0 || g_sd < 0 || o_sb < 0 || o_ss <= 0 || o_sh <= 0)
@@ -1349,6 +1420,14 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
   pa.scale_log2 = a.scale_log2;
   pa.err = a.err;
   pa.stall_ns = a.stall_ns;
+  if (stats) {
+    a.st_lse = pa.st_lse = stats->lse;
+    a.st_d = pa.st_d = stats->d;
+    a.dout = pa.dout = static_cast<const uint16_t*>(stats->dout);
+    a.d_sb = pa.d_sb = stats->d_sb;
+    a.d_ss = pa.d_ss = stats->d_ss;
+    a.d_sh = pa.d_sh = stats->d_sh;
+  }
 
   auto attn_kernel = g_sd > 0 ? vsa_attn_kernel<true> : vsa_attn_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1391,6 +1470,22 @@ vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t
     if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_fwd: launch", e);
   }
   return VSA_OK;
+}
+
+extern "C" {
+
+vsa_status vsa_sparse_attn_fwd(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H,
+                               const void* q, const void* k, const void* v, int64_t sb, int64_t ss,
+                               int64_t sh, const void* g, int64_t g_sb, int64_t g_ss, int64_t g_sh,
+                               int64_t g_sd, const int32_t* idx, const int32_t* cnt, int32_t kmax,
+                               const float* o_coarse, const int32_t* extra_idx, const int32_t* extra_cnt,
+                               void* out, int32_t out_dtype, int64_t o_sb,
+                               int64_t o_ss, int64_t o_sh, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  if (!g || !o_coarse || !out) return VSA_ERR_INVALID_ARG;
+  return attn_forward(L, p, B, H, q, k, v, sb, ss, sh, g, g_sb, g_ss, g_sh, g_sd, idx, cnt, kmax, o_coarse,
+                      extra_idx, extra_cnt, out, out_dtype, o_sb, o_ss, o_sh, nullptr, workspace, workspace_bytes,
+                      stream);
 }
 
 vsa_status vsa_debug_inject_wait_timeout(uint64_t timeout_ns) {

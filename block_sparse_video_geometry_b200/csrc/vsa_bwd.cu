@@ -1,0 +1,1112 @@
+// Backward pass of the VSA block-sparse attention: gradients of <out, dO> with
+// respect to q, k, v and the gate, the block selection held fixed (it is a
+// piecewise-constant function of the inputs). The pages train and distil
+// checkpoints against these modes ("BSAI FastH3 Native VSA (recipe)" and
+// "ComfyUI-Ref2VA-VSA", "The Solution: Ref2VAVSAGatePatch"); they do not spell
+// the backward out, so this is the exact derivative of the forward as the
+// forward kernels compute it (mean-pooled coarse branch).
+//
+// out_i = o_fine_i + cr_i g_i o_coarse[tile(i)]   (cr_i = 0 on dense conditioning rows)
+//  * gate:   dg_i = cr_i <dO_i, o_coarse[tile(i)]> (per channel: the products).
+//  * fine:   exact attention over each query tile's key set: with the row
+//            log2-sum-exp2 and D_i = <dO_i, o_fine_i> from a forward pass in
+//            statistics mode, P = 2^(c s - lse), dS = P (dO V^T - D),
+//            dq = scale dS K, dk = scale dS^T q, dv = P^T dO.
+//  * coarse: o_coarse[t] = softmax_c(scale <Qbar_t, Kbar_c>) Vbar over the
+//            candidate tiles; dOc[t] = sum over the tile's rows of cr g dO;
+//            the tile-level softmax backward gives dQbar, dKbar, dVbar, which
+//            flow back through the pooling (1 / tile count to every valid token).
+//
+// B200 design:
+//  * dq_kernel: one CTA per (batch, head, query tile) walking its key set; per
+//    key tile S = Q K^T and dP = dO V^T are M = 64 tcgen05 MMAs with Q and dO
+//    in TMEM and K, V bulk-copied tiles (the forward's tile-major copies), the
+//    fp32 elementwise step writes dS as bf16 over S in TMEM, and
+//    dQ += dS K accumulates in TMEM (K as the MN-major B operand).
+//  * dkv_kernel: one CTA per (batch, head, key tile) walking the query tiles
+//    that attend it (all of them for conditioning keys; for a candidate tile,
+//    dense conditioning rows plus the transpose of the selection lists, built
+//    on the GPU by a counting sort); S^T = K Q^T and dP^T = V dO^T with K and
+//    V in TMEM and Q, dO bulk-copied tile-major tiles, then dV += P^T dO and
+//    dK += dS^T Q with P^T, dS^T (bf16) in TMEM.
+//  * The coarse branch runs on CUDA cores in fp32 (like its forward):
+//    dOc and dg in one pass over the tokens, a row pass per 64 query tiles
+//    (softmax statistics, P, dS, dQbar), a column pass per 64 candidate tiles
+//    (dKbar, dVbar), and a scatter through the pooling.
+//  Both fine kernels run their MMAs and the elementwise step in turn (one CTA
+//  per SM, bulk copies of the next tiles in flight meanwhile).
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+
+#include "sm100.cuh"
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBThreads = 128;
+constexpr uint32_t kBTmemCols = 512;
+constexpr uint32_t kTB = 16384;          // one tile of Q, K, V or dO: [d half][64 rows][128 B]
+constexpr uint64_t kBTimeoutNs = 4000000000ull;
+constexpr uint64_t kBDrainNs = 200000000ull;
+constexpr size_t kBHeader = 256;         // status word
+constexpr size_t kBSmem = 120 * 1024;    // requested so that one CTA holds an SM (512 TMEM columns)
+
+// TMEM columns (lanes 0-15 of every quadrant: M = 64)
+//  dq_kernel : Q 0-63, dO 64-127, S / dS 128-191, dP 192-255, dQ 256-383
+//  dkv_kernel: K 0-63, V 64-127, S^T / P^T 128-191, dP^T / dS^T 192-255, dK 256-383, dV 384-511
+constexpr uint32_t kColA0 = 0, kColA1 = 64, kColS = 128, kColP = 192, kColAcc0 = 256, kColAcc1 = 384;
+
+struct BSmem {
+  uint8_t t0[2][kTB];                    // dq: K stages; dkv: Q stages
+  uint8_t t1[2][kTB];                    // dq: V stages; dkv: dO stages
+  float rowstat[2][2][64];               // dkv: lse and D of the query tile of each stage
+  uint64_t full[2], mma_done, acc_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct BArgs {
+  DevLayout L;
+  int32_t H, sink, n_cond, cand0, n_cand, kmax, c0;     // c0 = dense conditioning rows (0 unless rows mode)
+  const uint16_t* q;                     // natural layout [B, S, H, 128]
+  const uint16_t* k;
+  const uint16_t* v;
+  const uint16_t* dout;
+  int64_t sb, ss, sh;                    // strides of q, k, v
+  int64_t d_sb, d_ss, d_sh;              // strides of dO
+  const uint8_t* kv;                     // tile-major K, V: ((b * H + h) * n_tiles + t) * 32 KB
+  const uint8_t* qtm;                    // tile-major Q, dO: ((b * H + h) * n_tiles + t) * 16 KB
+  const uint8_t* dotm;
+  const float* lse;                      // [B, H, n_tiles, 64]
+  const float* dd;                       // [B, H, n_tiles, 64]
+  const int32_t* idx;
+  const int32_t* cnt;
+  const int32_t* csr_off;                // [B, H, n_cand + 1]
+  const int32_t* csr_list;               // query tiles per candidate
+  float* dq;                             // fp32 [B, S, H, 128] at element strides o_sb, o_ss, o_sh
+  float* dk;
+  float* dv;
+  int64_t o_sb, o_ss, o_sh;
+  float scale, c_log2;
+  int* err;
+};
+
+__device__ __forceinline__ void b_abort(BSmem& sm, int* err) {
+  atomicExch(err, VSA_ERR_TIMEOUT);
+  *reinterpret_cast<volatile int*>(&sm.abort) = 1;
+}
+
+// every thread of the block waits (bounded) on a barrier phase
+__device__ __forceinline__ bool b_wait(BSmem& sm, uint64_t& bar, uint32_t parity, int* err) {
+  const bool ok = mbar_wait(smem_u32(&bar), parity, &sm.abort, kBTimeoutNs);
+  if (!ok) b_abort(sm, err);
+  return ok;
+}
+
+// 64-row tile of a natural-layout [B, S, H, 128] tensor into TMEM as an M = 64
+// A operand (bf16 pairs, 64 columns): thread (row r, half hf) its 64 dims.
+__device__ __forceinline__ void rows_to_tmem(const uint16_t* base, const int32_t* perm_tile, int64_t ss, int r, int hf,
+                                             uint32_t taddr) {
+  const int t = perm_tile[r];
+  const uint4* src = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t) * ss + 64 * hf);
+  uint32_t w[32];
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    const uint4 u = t >= 0 ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
+    w[4 * cc] = u.x;
+    w[4 * cc + 1] = u.y;
+    w[4 * cc + 2] = u.z;
+    w[4 * cc + 3] = u.w;
+  }
+  tmem_st16x2_32<32>(taddr, w);
+}
+
+// Key tile of step jj of query tile qt's key set in the forward: dense rows
+// all tiles; otherwise the conditioning tiles (unless the sink is off), then
+// the selection list.
+__device__ __forceinline__ int dq_step_tile(const BArgs& a, int qt, size_t row, int jj, bool dense, int n_fixed) {
+  if (dense || jj < n_fixed) return jj;
+  const int c = a.idx[row * a.kmax + (jj - n_fixed)];
+  return a.cand0 + min(max(c, 0), a.n_cand - 1);
+}
+
+// Query tile of step jj of key tile kt's attending set: all query tiles for a
+// conditioning key tile (sink on); otherwise dense conditioning rows, then the
+// query tiles whose lists hold the tile.
+__device__ __forceinline__ int dkv_step_tile(const BArgs& a, const int32_t* list, int jj, bool all_rows) {
+  if (all_rows || jj < a.c0) return jj;
+  return list[jj - a.c0];
+}
+
+// -------------------------------------------------------------------- dQ
+__global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant__ BArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
+    return;
+  }
+  BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hf = lane >> 4;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  const size_t row = bh * a.L.n_tiles + qt;
+  const bool dense = qt < a.c0;
+  const int n_fixed = (a.sink == VSA_SINK_OFF || dense) ? 0 : a.n_cond;
+  const int n = dense ? a.L.n_tiles : n_fixed + min(max(a.cnt[row], 1), a.kmax);
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.full[0]), 1);
+    mbar_init(smem_u32(&sm.full[1]), 1);
+    mbar_init(smem_u32(&sm.mma_done), 1);
+    mbar_init(smem_u32(&sm.acc_done), 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kBTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // lanes 32 w .. 32 w + 15
+  const int r = warp * 16 + (lane & 15);
+  const int32_t* perm_q = a.L.perm + qt * kTile;
+  rows_to_tmem(a.q + b * a.sb + h * a.sh, perm_q, a.ss, r, hf, lane_addr + kColA0);
+  rows_to_tmem(a.dout + b * a.d_sb + h * a.d_sh, perm_q, a.d_ss, r, hf, lane_addr + kColA1);
+  tmem_wait_st();
+  const float lse = a.lse[row * kTile + r];
+  const float dd = a.dd[row * kTile + r];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint8_t* head_kv = a.kv + bh * a.L.n_tiles * 32768u;
+  auto issue = [&](int jj) {           // K and V of step jj into stage jj & 1
+    const int t = dq_step_tile(a, qt, row, jj, dense, n_fixed);
+    const uint32_t bar = smem_u32(&sm.full[jj & 1]);
+    mbar_arrive_expect_tx(bar, 2 * kTB);
+    bulk_load(smem_u32(sm.t0[jj & 1]), head_kv + static_cast<size_t>(t) * 32768u, kTB, bar);
+    bulk_load(smem_u32(sm.t1[jj & 1]), head_kv + static_cast<size_t>(t) * 32768u + kTB, kTB, bar);
+  };
+  if (threadIdx.x == 0) {
+    issue(0);
+    if (n > 1) issue(1);
+  }
+  bool ok = true;
+  int issued = n > 1 ? 2 : 1;
+  for (int jj = 0; jj < n; ++jj) {
+    const int st = jj & 1;
+    if (!(ok = b_wait(sm, sm.full[st], (jj >> 1) & 1, a.err))) break;
+    const int t = dq_step_tile(a, qt, row, jj, dense, n_fixed);
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      // S = Q K^T and dP = dO V^T (V K-major like K: [keys][d])
+      const uint64_t kd = smem_desc_sw128(smem_u32(sm.t0[st]), 16, 1024);
+      const uint64_t vd = smem_desc_sw128(smem_u32(sm.t1[st]), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t off = (kk >> 2) * (8192 >> 4) + (kk & 3) * 2;
+        umma_ts(tmem + kColS, tmem + kColA0 + kk * 8, kd + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
+        umma_ts(tmem + kColP, tmem + kColA1 + kk * 8, vd + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
+      }
+      umma_commit(smem_u32(&sm.mma_done));
+    }
+    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj) & 1, a.err))) break;
+    tc_fence_after();
+    float s[32], dp[32];
+    tmem_ld16x2_32f<32>(lane_addr + kColS, s);
+    tmem_ld16x2_32f<32>(lane_addr + kColP, dp);
+    tmem_wait_ld();
+    const unsigned long long vm = a.L.valid[t];
+    const uint32_t vbits = static_cast<uint32_t>(vm >> (32 * hf));
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float ds[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = 2 * i + e;
+        const float p = ((vbits >> key) & 1u) ? ex2_approx(fmaf(s[key], a.c_log2, -lse)) : 0.f;
+        ds[e] = p * (dp[key] - dd);
+      }
+      w[i] = pack_bf16x2(ds[0], ds[1]);
+    }
+    tmem_st16x2_16<16>(lane_addr + kColS, w);    // dS (bf16 pairs) over S
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      // dQ += dS K: dS (A) in TMEM, K as the MN-major B operand ([keys][d])
+      const uint64_t kmn = smem_desc_sw128(smem_u32(sm.t0[st]), 8192, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        umma_ts(tmem + kColAcc0, tmem + kColS + kk * 8, kmn + kk * (2048 >> 4), idesc_bf16_f32(64, 128, 0, 1),
+                (jj > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(smem_u32(&sm.mma_done));
+    }
+    // the stage is free (and S may be overwritten) once dQ += dS K completed
+    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj + 1) & 1, a.err))) break;
+    if (threadIdx.x == 0 && jj + 2 < n) {
+      issue(jj + 2);
+      ++issued;
+    }
+  }
+  if (ok) {
+    tc_fence_after();
+    const int tok = perm_q[r];
+#pragma unroll 1
+    for (int ch = 0; ch < 2; ++ch) {
+      float y[32];
+      tmem_ld16x2_32f<64>(lane_addr + kColAcc0 + 32 * ch, y);
+      tmem_wait_ld();
+      if (tok >= 0) {
+        float4* dst = reinterpret_cast<float4*>(a.dq + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
+                                                h * a.o_sh + 64 * hf + 32 * ch);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          dst[i / 4] = make_float4(y[i] * a.scale, y[i + 1] * a.scale, y[i + 2] * a.scale, y[i + 3] * a.scale);
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    // let every issued copy land before the block exits
+    for (int i = max(0, issued - 2); i < issued; ++i)
+      mbar_wait(smem_u32(&sm.full[i & 1]), (i >> 1) & 1, nullptr, kBDrainNs);
+    umma_commit(smem_u32(&sm.acc_done));
+    mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBTmemCols);
+  }
+}
+
+// -------------------------------------------------------------- dK and dV
+__global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant__ BArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
+    return;
+  }
+  BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hf = lane >> 4;
+  const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  const int n_tiles = a.L.n_tiles;
+  const bool all_rows = a.sink != VSA_SINK_OFF && kt < a.n_cond;
+  const int c = kt - a.cand0;                       // candidate ordinal when not all_rows
+  const int32_t* list = nullptr;
+  int n;
+  if (all_rows) {
+    n = n_tiles;
+  } else {
+    const int32_t* off = a.csr_off + bh * (a.n_cand + 1);
+    list = a.csr_list + off[c];
+    n = a.c0 + (off[c + 1] - off[c]);
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.full[0]), 1);
+    mbar_init(smem_u32(&sm.full[1]), 1);
+    mbar_init(smem_u32(&sm.mma_done), 1);
+    mbar_init(smem_u32(&sm.acc_done), 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kBTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const int r = warp * 16 + (lane & 15);            // key slot of this thread
+  const int32_t* perm_k = a.L.perm + kt * kTile;
+  rows_to_tmem(a.k + b * a.sb + h * a.sh, perm_k, a.ss, r, hf, lane_addr + kColA0);
+  rows_to_tmem(a.v + b * a.sb + h * a.sh, perm_k, a.ss, r, hf, lane_addr + kColA1);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  auto issue = [&](int jj) {           // Q, dO and the row statistics of step jj into stage jj & 1
+    const int qt = dkv_step_tile(a, list, jj, all_rows);
+    const size_t tq = bh * n_tiles + qt;
+    const uint32_t bar = smem_u32(&sm.full[jj & 1]);
+    mbar_arrive_expect_tx(bar, 2 * kTB + 2 * 256);
+    bulk_load(smem_u32(sm.t0[jj & 1]), a.qtm + tq * kTB, kTB, bar);
+    bulk_load(smem_u32(sm.t1[jj & 1]), a.dotm + tq * kTB, kTB, bar);
+    bulk_load(smem_u32(sm.rowstat[jj & 1][0]), a.lse + tq * kTile, 256, bar);
+    bulk_load(smem_u32(sm.rowstat[jj & 1][1]), a.dd + tq * kTile, 256, bar);
+  };
+  if (threadIdx.x == 0) {
+    if (n > 0) issue(0);
+    if (n > 1) issue(1);
+  }
+  bool ok = true;
+  int issued = min(n, 2);
+  for (int jj = 0; jj < n; ++jj) {
+    const int st = jj & 1;
+    if (!(ok = b_wait(sm, sm.full[st], (jj >> 1) & 1, a.err))) break;
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      // S^T = K Q^T and dP^T = V dO^T: K, V (A) in TMEM, Q and dO K-major
+      const uint64_t qd = smem_desc_sw128(smem_u32(sm.t0[st]), 16, 1024);
+      const uint64_t od = smem_desc_sw128(smem_u32(sm.t1[st]), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t off = (kk >> 2) * (8192 >> 4) + (kk & 3) * 2;
+        umma_ts(tmem + kColS, tmem + kColA0 + kk * 8, qd + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
+        umma_ts(tmem + kColP, tmem + kColA1 + kk * 8, od + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
+      }
+      umma_commit(smem_u32(&sm.mma_done));
+    }
+    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj) & 1, a.err))) break;
+    tc_fence_after();
+    float s[32], dp[32];
+    tmem_ld16x2_32f<32>(lane_addr + kColS, s);
+    tmem_ld16x2_32f<32>(lane_addr + kColP, dp);
+    tmem_wait_ld();
+    uint32_t wp[16], wd[16];
+    const float* lse = sm.rowstat[st][0] + 32 * hf;     // queries 32 hf .. 32 hf + 31 (columns of this thread)
+    const float* dd = sm.rowstat[st][1] + 32 * hf;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float p[2], ds[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int qi = 2 * i + e;
+        p[e] = ex2_approx(fmaf(s[qi], a.c_log2, -lse[qi]));    // padding query rows: lse = +inf, P = 0
+        ds[e] = p[e] * (dp[qi] - dd[qi]);
+      }
+      wp[i] = pack_bf16x2(p[0], p[1]);
+      wd[i] = pack_bf16x2(ds[0], ds[1]);
+    }
+    tmem_st16x2_16<16>(lane_addr + kColS, wp);          // P^T over S^T
+    tmem_st16x2_16<16>(lane_addr + kColP, wd);          // dS^T over dP^T
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      // dV += P^T dO and dK += dS^T Q: dO and Q as MN-major B operands ([queries][d])
+      const uint64_t omn = smem_desc_sw128(smem_u32(sm.t1[st]), 8192, 1024);
+      const uint64_t qmn = smem_desc_sw128(smem_u32(sm.t0[st]), 8192, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        umma_ts(tmem + kColAcc1, tmem + kColS + kk * 8, omn + kk * (2048 >> 4), idesc_bf16_f32(64, 128, 0, 1),
+                (jj > 0 || kk > 0) ? 1u : 0u);
+        umma_ts(tmem + kColAcc0, tmem + kColP + kk * 8, qmn + kk * (2048 >> 4), idesc_bf16_f32(64, 128, 0, 1),
+                (jj > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(smem_u32(&sm.mma_done));
+    }
+    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj + 1) & 1, a.err))) break;
+    if (threadIdx.x == 0 && jj + 2 < n) {
+      issue(jj + 2);
+      ++issued;
+    }
+  }
+  if (ok) {
+    tc_fence_after();
+    const int tok = perm_k[r];
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {          // dK (scaled), dV
+      float* dst_base = which == 0 ? a.dk : a.dv;
+      const float f = which == 0 ? a.scale : 1.0f;
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        float y[32];
+        if (n > 0) {
+          tmem_ld16x2_32f<64>(lane_addr + (which == 0 ? kColAcc0 : kColAcc1) + 32 * ch, y);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = 0.f;
+        }
+        if (tok >= 0) {
+          float4* dst = reinterpret_cast<float4*>(dst_base + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
+                                                  h * a.o_sh + 64 * hf + 32 * ch);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            dst[i / 4] = make_float4(y[i] * f, y[i + 1] * f, y[i + 2] * f, y[i + 3] * f);
+        }
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    for (int i = max(0, issued - 2); i < issued; ++i)
+      mbar_wait(smem_u32(&sm.full[i & 1]), (i >> 1) & 1, nullptr, kBDrainNs);
+    umma_commit(smem_u32(&sm.acc_done));
+    mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBTmemCols);
+  }
+}
+
+// ------------------------------------------- transpose of the selection lists
+// grid (sparse query tiles, H, B): counts of query tiles per candidate tile
+__global__ void csr_count_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int kmax,
+                                 int n_cand, int n_tiles, int c0, int H, int32_t* __restrict__ counts) {
+  const int qt = c0 + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * H + h;
+  const size_t row = bh * n_tiles + qt;
+  const int n = min(max(cnt[row], 1), kmax);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int c = min(max(idx[row * kmax + i], 0), n_cand - 1);
+    atomicAdd(&counts[bh * (n_cand + 1) + c], 1);
+  }
+}
+
+// grid (H, B), 1024 threads: exclusive scan of the counts of one (b, h) into
+// offsets (n_cand + 1 entries, relative to the head's list base bh * n_tiles *
+// kmax); the cursors for the fill start at the offsets.
+__global__ void __launch_bounds__(1024) csr_scan_kernel(int32_t* __restrict__ counts_off, int32_t* __restrict__ cursor,
+                                                        int n_cand, int n_tiles, int kmax, int H) {
+  const size_t bh = static_cast<size_t>(blockIdx.y) * H + blockIdx.x;
+  int32_t* c = counts_off + bh * (n_cand + 1);
+  int32_t* cur = cursor + bh * (n_cand + 1);
+  __shared__ int32_t part[1024];
+  const int per = (n_cand + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * per, hi = min(n_cand, lo + per);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += c[i];
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  for (int off = 1; off < static_cast<int>(blockDim.x); off <<= 1) {
+    const int v = threadIdx.x >= static_cast<unsigned>(off) ? part[threadIdx.x - off] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int run = static_cast<int>(bh * static_cast<size_t>(n_tiles) * kmax) + part[threadIdx.x] - sum;
+  for (int i = lo; i < hi; ++i) {
+    const int ci = c[i];
+    c[i] = run;
+    cur[i] = run;
+    run += ci;
+  }
+  if (threadIdx.x == blockDim.x - 1) c[n_cand] = run;
+}
+
+__global__ void csr_fill_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int kmax,
+                                int n_cand, int n_tiles, int c0, int H, int32_t* __restrict__ cursor,
+                                int32_t* __restrict__ list) {
+  const int qt = c0 + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * H + h;
+  const size_t row = bh * n_tiles + qt;
+  const int n = min(max(cnt[row], 1), kmax);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int c = min(max(idx[row * kmax + i], 0), n_cand - 1);
+    list[atomicAdd(&cursor[bh * (n_cand + 1) + c], 1)] = qt;
+  }
+}
+
+// One tensor of [B, S, H, 128] into tile-major 16 KB blocks (as the forward's).
+__global__ void __launch_bounds__(256)
+permute_one_kernel(DevLayout L, const uint16_t* __restrict__ x, int64_t sb, int64_t ss, int64_t sh, int H,
+                   uint8_t* __restrict__ xtm) {
+  const int tile = blockIdx.x, b = blockIdx.y;
+  __shared__ int tok[kTile];
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
+  __syncthreads();
+  for (int w = threadIdx.x; w < H * 1024; w += blockDim.x) {
+    const int pc = w & 7, r = (w >> 3) & 63, j = (w >> 9) & 1, h = w >> 10;
+    const int t = tok[r];
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= 0)
+      val = __ldg(reinterpret_cast<const uint4*>(x + b * sb + static_cast<int64_t>(t) * ss + h * sh + j * 64 +
+                                                 ((pc ^ (r & 7)) << 3)));
+    *reinterpret_cast<uint4*>(xtm + ((static_cast<size_t>(b) * H + h) * L.n_tiles + tile) * 16384u + j * 8192 +
+                              r * 128 + pc * 16) = val;
+  }
+}
+
+// ---------------------------------------------------------- coarse branch
+// Pooled means of Q, K, V: [3, B, H, n_tiles, 128]; grid (n_tiles, B, 3).
+__global__ void __launch_bounds__(1024)
+pool3_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+             const uint16_t* __restrict__ v, int64_t sb, int64_t ss, int64_t sh, int H, int B,
+             float* __restrict__ pooled) {
+  const int tile = blockIdx.x, b = blockIdx.y, which = blockIdx.z;
+  const uint16_t* x = which == 0 ? q : (which == 1 ? k : v);
+  __shared__ int tok[kTile];
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
+  __syncthreads();
+  const float n = static_cast<float>(L.count[tile]);
+  for (int c = threadIdx.x; c < H * 16; c += blockDim.x) {
+    const int h = c >> 4, d0 = (c & 15) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < kTile; ++s) {
+      const int t = tok[s];
+      if (t < 0) continue;
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + b * sb + static_cast<int64_t>(t) * ss + h * sh + d0));
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += __uint_as_float(u[e] << 16);
+        acc[2 * e + 1] += __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+    }
+    float* dst = pooled + ((((static_cast<size_t>(which) * B + b) * H + h) * L.n_tiles + tile) * kHeadDim + d0);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[e] = acc[e] / n;
+  }
+}
+
+// dOc[b, h, t] = sum over the valid rows i of tile t of cr_i g_i dO_i (per
+// channel: g_{i,d} dO_{i,d}); dg_i = cr_i <dO_i, o_coarse[t]> (per channel:
+// cr_i dO_{i,d} o_coarse[t, d]). cr = 0 on dense conditioning rows.
+// grid (n_tiles, B), thread c: head c / 16, dims 8 (c % 16) .. + 7.
+__global__ void __launch_bounds__(1024)
+gate_bwd_kernel(DevLayout L, const uint16_t* __restrict__ dout, int64_t d_sb, int64_t d_ss, int64_t d_sh,
+                const uint16_t* __restrict__ g, int64_t g_sb, int64_t g_ss, int64_t g_sh, int64_t g_sd,
+                const float* __restrict__ o_coarse, int H, int c0, float* __restrict__ doc, float* __restrict__ dg,
+                int64_t dg_sb, int64_t dg_ss, int64_t dg_sh, int64_t dg_sd) {
+  const int tile = blockIdx.x, b = blockIdx.y;
+  __shared__ int tok[kTile];
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
+  __syncthreads();
+  const bool cr = tile >= c0;
+  // every lane of a warp runs the loop (the shuffle-sum below needs them all);
+  // threads past the last head compute on head 0 and write nothing
+  for (int cb = 0; cb < H * 16; cb += blockDim.x) {
+    const int c = cb + threadIdx.x;
+    const bool act = c < H * 16;
+    const int h = act ? c >> 4 : 0, d0 = (c & 15) * 8, part = c & 15;
+    const size_t th = (static_cast<size_t>(b) * H + h) * L.n_tiles + tile;
+    const float* oc = o_coarse + th * kHeadDim + d0;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < kTile; ++s) {
+      const int t = tok[s];
+      if (t < 0) continue;     // uniform over the block: every thread sees the same token list
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(dout + b * d_sb + static_cast<int64_t>(t) * d_ss +
+                                                           h * d_sh + d0));
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+      float dov[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dov[2 * e] = __uint_as_float(u[e] << 16);
+        dov[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+      const uint16_t* gp = g + b * g_sb + static_cast<int64_t>(t) * g_ss + h * g_sh;
+      float* dgp = dg + b * dg_sb + static_cast<int64_t>(t) * dg_ss + h * dg_sh;
+      if (g_sd > 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float ge = __uint_as_float(static_cast<uint32_t>(gp[(d0 + e) * g_sd]) << 16);
+          acc[e] = fmaf(cr ? ge : 0.f, dov[e], acc[e]);
+          if (act) dgp[(d0 + e) * dg_sd] = cr ? dov[e] * oc[e] : 0.f;
+        }
+      } else {
+        const float ge = cr ? __uint_as_float(static_cast<uint32_t>(gp[0]) << 16) : 0.f;
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc[e] = fmaf(ge, dov[e], acc[e]);
+          dot = fmaf(dov[e], oc[e], dot);
+        }
+        // the 16 threads of a head hold the 16 parts of <dO, o_coarse>: shuffle-sum
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (act && part == 0) dgp[0] = cr ? dot : 0.f;
+      }
+    }
+    if (act) {
+      float* dst = doc + th * kHeadDim + d0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dst[e] = acc[e];
+    }
+  }
+}
+
+// Row pass of the coarse softmax backward: per block of 64 query tiles of one
+// (b, h), two sweeps over the candidate tiles: (1) row max and sum of
+// s = scale <Qbar, Kbar>; (2) P = softmax, dP = <dOc, Vbar>, dS = P (dP - D)
+// with D = <dOc, o_coarse>, dQbar += scale dS Kbar; P and dS are stored for the
+// column pass. Thread (ty, tx) = (tid / 16, tid % 16): rows 4 ty .. 4 ty + 3,
+// candidate columns 4 tx .. 4 tx + 3 of a chunk, output dims 8 tx .. 8 tx + 7.
+constexpr int kCR = 64, kCC = 64, kCThreads = 256;
+
+struct CRSmem {
+  float qT[kHeadDim][kCR];               // Qbar rows, transposed
+  float gT[kHeadDim][kCR];               // dOc rows, transposed
+  float kT[kHeadDim][kCC];               // Kbar chunk, transposed
+  float vT[kHeadDim][kCC];               // Vbar chunk, transposed
+  float kr[kCC][kHeadDim];               // Kbar chunk, rows (for dQbar)
+  float ds[kCR][kCC + 4];
+  float dsum[kCR];                       // D per row
+};
+
+__global__ void __launch_bounds__(kCThreads)
+coarse_bwd_rows_kernel(int n_tiles, int cand0, int n_cand, int H, int B, const float* __restrict__ pooled,
+                       const float* __restrict__ doc, const float* __restrict__ o_coarse, float scale,
+                       float* __restrict__ pm, float* __restrict__ dsm, int ld, float* __restrict__ dqbar) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  CRSmem& sm = *reinterpret_cast<CRSmem*>(smem_raw);
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int qt0 = blockIdx.x * kCR, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * H + h;
+  const size_t plane = static_cast<size_t>(B) * H * n_tiles * kHeadDim;
+  const float* qbar = pooled + bh * n_tiles * kHeadDim;
+  const float* kbar = pooled + plane + (bh * n_tiles + cand0) * kHeadDim;
+  const float* vbar = pooled + 2 * plane + (bh * n_tiles + cand0) * kHeadDim;
+  for (int f = tid; f < kCR * kHeadDim; f += kCThreads) {
+    const int r = f % kCR, d = f / kCR;
+    const bool in = qt0 + r < n_tiles;
+    sm.qT[d][r] = in ? qbar[static_cast<size_t>(qt0 + r) * kHeadDim + d] : 0.f;
+    sm.gT[d][r] = in ? doc[(bh * n_tiles + qt0 + r) * kHeadDim + d] : 0.f;
+  }
+  if (tid < kCR) {
+    float s = 0.f;
+    if (qt0 + tid < n_tiles)
+      for (int d = 0; d < kHeadDim; ++d)
+        s += doc[(bh * n_tiles + qt0 + tid) * kHeadDim + d] * o_coarse[(bh * n_tiles + qt0 + tid) * kHeadDim + d];
+    sm.dsum[tid] = s;
+  }
+  float m[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+  }
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int c0 = 0; c0 < n_cand; c0 += kCC) {
+      __syncthreads();
+      for (int f = tid; f < kCC * kHeadDim; f += kCThreads) {
+        const int cc = f / kHeadDim, d = f % kHeadDim;
+        const bool in = c0 + cc < n_cand;
+        const float kv = in ? kbar[static_cast<size_t>(c0 + cc) * kHeadDim + d] : 0.f;
+        sm.kT[d][cc] = kv;
+        sm.kr[cc][d] = kv;
+        sm.vT[d][cc] = in ? vbar[static_cast<size_t>(c0 + cc) * kHeadDim + d] : 0.f;
+      }
+      __syncthreads();
+      float s[4][4], dp[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[i][j] = dp[i][j] = 0.f;
+      for (int d = 0; d < kHeadDim; ++d) {
+        float qa[4], kb[4], ga[4], vb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          qa[i] = sm.qT[d][4 * ty + i];
+          ga[i] = sm.gT[d][4 * ty + i];
+          kb[i] = sm.kT[d][4 * tx + i];
+          vb[i] = sm.vT[d][4 * tx + i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            s[i][j] = fmaf(qa[i], kb[j], s[i][j]);
+            if (pass) dp[i][j] = fmaf(ga[i], vb[j], dp[i][j]);
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[i][j] = (c0 + 4 * tx + j < n_cand) ? s[i][j] * scale : -INFINITY;
+      if (pass == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float cm = fmaxf(fmaxf(s[i][0], s[i][1]), fmaxf(s[i][2], s[i][3]));
+#pragma unroll
+          for (int off = 1; off < 16; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+          const float mn = fmaxf(m[i], cm);
+          float ps = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ps += expf(s[i][j] - mn);
+#pragma unroll
+          for (int off = 1; off < 16; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+          l[i] = l[i] * expf(m[i] - mn) + ps;
+          m[i] = mn;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = 4 * ty + i, row = qt0 + rr;
+          const float dsum = sm.dsum[rr];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int col = c0 + 4 * tx + j;
+            const float p = col < n_cand ? expf(s[i][j] - m[i]) / l[i] : 0.f;
+            const float dsv = p * (dp[i][j] - dsum);
+            sm.ds[rr][4 * tx + j] = dsv;
+            if (row < n_tiles && col < n_cand) {
+              pm[(bh * n_tiles + row) * ld + col] = p;
+              dsm[(bh * n_tiles + row) * ld + col] = dsv;
+            }
+          }
+        }
+        __syncthreads();
+        for (int cc = 0; cc < kCC; ++cc) {
+          float dsr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dsr[i] = sm.ds[4 * ty + i][cc];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float kv = sm.kr[cc][8 * tx + e];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i][e] = fmaf(dsr[i], kv, acc[i][e]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = qt0 + 4 * ty + i;
+    if (row < n_tiles)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dqbar[(bh * n_tiles + row) * kHeadDim + 8 * tx + e] = acc[i][e] * scale;
+  }
+}
+
+// Column pass: per block of 64 candidate tiles, dKbar = scale dS^T Qbar and
+// dVbar = P^T dOc over all query tiles. Thread (ty, tx): candidates 4 ty ..,
+// dims 8 tx ...
+struct CCSmem {
+  float ds[kCR][kCC + 4];
+  float p[kCR][kCC + 4];
+  float q[kCR][kHeadDim];
+  float g[kCR][kHeadDim];
+};
+
+__global__ void __launch_bounds__(kCThreads)
+coarse_bwd_cols_kernel(int n_tiles, int n_cand, int H, int B, const float* __restrict__ pooled,
+                       const float* __restrict__ doc, float scale, const float* __restrict__ pm,
+                       const float* __restrict__ dsm, int ld, float* __restrict__ dkbar, float* __restrict__ dvbar) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  CCSmem& sm = *reinterpret_cast<CCSmem*>(smem_raw);
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int c0 = blockIdx.x * kCC, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * H + h;
+  const float* qbar = pooled + bh * n_tiles * kHeadDim;
+  float ak[4][8], av[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ak[i][e] = av[i][e] = 0.f;
+  for (int r0 = 0; r0 < n_tiles; r0 += kCR) {
+    __syncthreads();
+    for (int f = tid; f < kCR * kCC; f += kCThreads) {
+      const int rr = f / kCC, cc = f % kCC;
+      const bool in = r0 + rr < n_tiles && c0 + cc < n_cand;
+      sm.ds[rr][cc] = in ? dsm[(bh * n_tiles + r0 + rr) * ld + c0 + cc] : 0.f;
+      sm.p[rr][cc] = in ? pm[(bh * n_tiles + r0 + rr) * ld + c0 + cc] : 0.f;
+    }
+    for (int f = tid; f < kCR * kHeadDim; f += kCThreads) {
+      const int rr = f / kHeadDim, d = f % kHeadDim;
+      const bool in = r0 + rr < n_tiles;
+      sm.q[rr][d] = in ? qbar[static_cast<size_t>(r0 + rr) * kHeadDim + d] : 0.f;
+      sm.g[rr][d] = in ? doc[(bh * n_tiles + r0 + rr) * kHeadDim + d] : 0.f;
+    }
+    __syncthreads();
+    for (int rr = 0; rr < kCR; ++rr) {
+      float dsr[4], pr[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dsr[i] = sm.ds[rr][4 * ty + i];
+        pr[i] = sm.p[rr][4 * ty + i];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float qv = sm.q[rr][8 * tx + e], gv = sm.g[rr][8 * tx + e];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ak[i][e] = fmaf(dsr[i], qv, ak[i][e]);
+          av[i][e] = fmaf(pr[i], gv, av[i][e]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = c0 + 4 * ty + i;
+    if (c < n_cand)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        dkbar[(bh * n_cand + c) * kHeadDim + 8 * tx + e] = ak[i][e] * scale;
+        dvbar[(bh * n_cand + c) * kHeadDim + 8 * tx + e] = av[i][e];
+      }
+  }
+}
+
+// The pooled gradients back to the tokens: dq += dQbar[t] / n_t for every
+// valid token of tile t, dk += dKbar / n_t, dv += dVbar / n_t for candidate
+// tiles. grid (n_tiles, B).
+__global__ void __launch_bounds__(1024)
+pool_scatter_kernel(DevLayout L, int H, int cand0, int n_cand, const float* __restrict__ dqbar,
+                    const float* __restrict__ dkbar, const float* __restrict__ dvbar, float* __restrict__ dq,
+                    float* __restrict__ dk, float* __restrict__ dv, int64_t o_sb, int64_t o_ss, int64_t o_sh) {
+  const int tile = blockIdx.x, b = blockIdx.y;
+  __shared__ int tok[kTile];
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
+  __syncthreads();
+  const float inv_n = 1.0f / static_cast<float>(L.count[tile]);
+  const int c = tile - cand0;
+  const bool cand = c >= 0 && c < n_cand;
+  for (int w = threadIdx.x; w < H * kHeadDim; w += blockDim.x) {
+    const int h = w / kHeadDim, d = w % kHeadDim;
+    const size_t bh = static_cast<size_t>(b) * H + h;
+    const float gq = dqbar[(bh * L.n_tiles + tile) * kHeadDim + d] * inv_n;
+    const float gk = cand ? dkbar[(bh * n_cand + c) * kHeadDim + d] * inv_n : 0.f;
+    const float gv = cand ? dvbar[(bh * n_cand + c) * kHeadDim + d] * inv_n : 0.f;
+    for (int s = 0; s < kTile; ++s) {
+      const int t = tok[s];
+      if (t < 0) continue;
+      const int64_t off = b * o_sb + static_cast<int64_t>(t) * o_ss + h * o_sh + d;
+      dq[off] += gq;
+      if (cand) {
+        dk[off] += gk;
+        dv[off] += gv;
+      }
+    }
+  }
+}
+
+// [header][attention workspace][lse][D][tile-major Q][tile-major dO][CSR offsets][CSR cursors][CSR lists]
+// [pooled Q, K, V][dOc][P][dS][dQbar][dKbar][dVbar]
+struct BWorkspace {
+  size_t attn, attn_bytes, lse, dd, qtm, dotm, off, cur, list, pooled, doc, pm, dsm, dqbar, dkbar, dvbar, total;
+  int32_t ld;
+};
+
+BWorkspace b_workspace(const vsa_layout* L, int B, int H, const vsa_params* p) {
+  BWorkspace w{};
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t tiles = bh * L->n_tiles;
+  const Candidates cand = candidates(L, p->sink);
+  int32_t kmax = 0;
+  vsa_select_kmax(L, p, &kmax);
+  size_t attn_bytes = 0;
+  vsa_sparse_attn_workspace_size(L, B, H, p, &attn_bytes);
+  w.ld = (cand.count + 3) / 4 * 4;
+  size_t o = kBHeader;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  w.attn = take(attn_bytes);
+  w.attn_bytes = attn_bytes;
+  w.lse = take(tiles * kTile * sizeof(float));
+  w.dd = take(tiles * kTile * sizeof(float));
+  w.qtm = take(tiles * kTB);
+  w.dotm = take(tiles * kTB);
+  w.off = take(bh * (cand.count + 1) * sizeof(int32_t));
+  w.cur = take(bh * (cand.count + 1) * sizeof(int32_t));
+  w.list = take(tiles * static_cast<size_t>(kmax) * sizeof(int32_t));
+  w.pooled = take(3 * tiles * kHeadDim * sizeof(float));
+  w.doc = take(tiles * kHeadDim * sizeof(float));
+  w.pm = take(tiles * static_cast<size_t>(w.ld) * sizeof(float));
+  w.dsm = take(tiles * static_cast<size_t>(w.ld) * sizeof(float));
+  w.dqbar = take(tiles * kHeadDim * sizeof(float));
+  w.dkbar = take(bh * cand.count * kHeadDim * sizeof(float));
+  w.dvbar = take(bh * cand.count * kHeadDim * sizeof(float));
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+}  // namespace vsa
+
+using namespace vsa;
+
+extern "C" {
+
+vsa_status vsa_sparse_attn_bwd_workspace_size(const vsa_layout* L, int32_t B, int32_t H, const vsa_params* p,
+                                              size_t* bytes) {
+  if (!L || !bytes || B <= 0 || H <= 0) return VSA_ERR_INVALID_ARG;
+  vsa_status st = check_params(p);
+  if (st != VSA_OK) return st;
+  *bytes = b_workspace(L, B, H, p).total;
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_bwd(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H, const void* q,
+                               const void* k, const void* v, int64_t sb, int64_t ss, int64_t sh, const void* g,
+                               int64_t g_sb, int64_t g_ss, int64_t g_sh, int64_t g_sd, const int32_t* idx,
+                               const int32_t* cnt, int32_t kmax, const float* o_coarse, const void* dout,
+                               int64_t d_sb, int64_t d_ss, int64_t d_sh, float* dq, float* dk, float* dv,
+                               int64_t o_sb, int64_t o_ss, int64_t o_sh, float* dg, int64_t dg_sb, int64_t dg_ss,
+                               int64_t dg_sh, int64_t dg_sd, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  if (!L) return VSA_ERR_INVALID_ARG;
+  vsa_status st = check_params(p);
+  if (st != VSA_OK) return st;
+  if (p->coarse != VSA_COARSE_MEAN || p->extra_tokens != 0) return VSA_ERR_UNSUPPORTED;
+  st = check_qkv(q, k, v, sb, ss, sh, B, H);
+  if (st != VSA_OK) return st;
+  st = check_qkv(dout, dout, dout, d_sb, d_ss, d_sh, B, H);
+  if (st != VSA_OK) return st;
+  if (!g || !idx || !cnt || !o_coarse || !dq || !dk || !dv || !dg || !workspace) return VSA_ERR_INVALID_ARG;
+  if (g_sb < 0 || g_ss <= 0 || g_sh <= 0 || g_sd < 0 || dg_sb < 0 || dg_ss <= 0 || dg_sh <= 0 || dg_sd < 0 ||
+      (g_sd > 0) != (dg_sd > 0))
+    return VSA_ERR_INVALID_ARG;
+  if (o_sb < 0 || o_ss <= 0 || o_sh <= 0 || (o_sb * 4) % 16 || (o_ss * 4) % 16 || (o_sh * 4) % 16 ||
+      reinterpret_cast<uintptr_t>(dq) % 16 || reinterpret_cast<uintptr_t>(dk) % 16 ||
+      reinterpret_cast<uintptr_t>(dv) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256 ||
+      reinterpret_cast<uintptr_t>(o_coarse) % 16)
+    return VSA_ERR_INVALID_ARG;
+  const BWorkspace ws = b_workspace(L, B, H, p);
+  if (workspace_bytes < ws.total) return VSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!L->dev_buf) return VSA_ERR_NOT_UPLOADED;
+  int32_t want_kmax = 0;
+  vsa_select_kmax(L, p, &want_kmax);
+  if (kmax != want_kmax) return VSA_ERR_INVALID_ARG;
+
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  const DevLayout D = L->dev();
+  const Candidates cand = candidates(L, p->sink);
+  const int c0 = p->sink == VSA_SINK_EXACT_KV_AND_ROWS ? L->n_cond : 0;
+  const float scale = effective_scale(p);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaMemsetAsync", e);
+
+  // 1. the forward's row statistics (log2-sum-exp2, D = <dO, o_fine>)
+  AttnStats stats{};
+  stats.lse = reinterpret_cast<float*>(w + ws.lse);
+  stats.d = reinterpret_cast<float*>(w + ws.dd);
+  stats.dout = dout;
+  stats.d_sb = d_sb;
+  stats.d_ss = d_ss;
+  stats.d_sh = d_sh;
+  st = attn_forward(L, p, B, H, q, k, v, sb, ss, sh, nullptr, 0, 0, 0, 0, idx, cnt, kmax, nullptr, nullptr,
+                    nullptr, nullptr, VSA_OUT_F32, 0, 0, 0, &stats, w + ws.attn, ws.attn_bytes, stream);
+  if (st != VSA_OK) return st;
+  // the attention workspace now holds the tile-major K and V right after its 256-byte header
+  const uint8_t* kv = w + ws.attn + 256;
+
+  // 2. tile-major Q and dO; the transpose of the selection lists
+  permute_one_kernel<<<dim3(L->n_tiles, B), 256, 0, stream>>>(D, static_cast<const uint16_t*>(q), sb, ss, sh, H,
+                                                             w + ws.qtm);
+  permute_one_kernel<<<dim3(L->n_tiles, B), 256, 0, stream>>>(D, static_cast<const uint16_t*>(dout), d_sb, d_ss,
+                                                             d_sh, H, w + ws.dotm);
+  int32_t* off = reinterpret_cast<int32_t*>(w + ws.off);
+  int32_t* cur = reinterpret_cast<int32_t*>(w + ws.cur);
+  int32_t* list = reinterpret_cast<int32_t*>(w + ws.list);
+  e = cudaMemsetAsync(off, 0, static_cast<size_t>(B) * H * (cand.count + 1) * sizeof(int32_t), stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaMemsetAsync(csr)", e);
+  const int nq = L->n_tiles - c0;
+  if (nq > 0) csr_count_kernel<<<dim3(nq, H, B), 128, 0, stream>>>(idx, cnt, kmax, cand.count, L->n_tiles, c0, H, off);
+  csr_scan_kernel<<<dim3(H, B), 1024, 0, stream>>>(off, cur, cand.count, L->n_tiles, kmax, H);
+  if (nq > 0)
+    csr_fill_kernel<<<dim3(nq, H, B), 128, 0, stream>>>(idx, cnt, kmax, cand.count, L->n_tiles, c0, H, cur, list);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: permute/transpose launch", e);
+
+  // 3. the fine branch: dq, then dk and dv (each written once per token)
+  BArgs a{};
+  a.L = D;
+  a.H = H;
+  a.sink = p->sink;
+  a.n_cond = L->n_cond;
+  a.cand0 = cand.first;
+  a.n_cand = cand.count;
+  a.kmax = kmax;
+  a.c0 = c0;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.dout = static_cast<const uint16_t*>(dout);
+  a.sb = sb;
+  a.ss = ss;
+  a.sh = sh;
+  a.d_sb = d_sb;
+  a.d_ss = d_ss;
+  a.d_sh = d_sh;
+  a.kv = kv;
+  a.qtm = w + ws.qtm;
+  a.dotm = w + ws.dotm;
+  a.lse = stats.lse;
+  a.dd = stats.d;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.csr_off = off;
+  a.csr_list = list;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.o_sb = o_sb;
+  a.o_ss = o_ss;
+  a.o_sh = o_sh;
+  a.scale = scale;
+  a.c_log2 = scale * 1.4426950408889634f;
+  a.err = static_cast<int*>(workspace);
+  for (auto kern : {dq_kernel, dkv_kernel}) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kBSmem));
+    if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute", e);
+  }
+  dq_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kBSmem, stream>>>(a);
+  dkv_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kBSmem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: fine-branch launch", e);
+
+  // 4. gate and coarse branch, then the pooled gradients back to the tokens
+  float* pooled = reinterpret_cast<float*>(w + ws.pooled);
+  float* doc = reinterpret_cast<float*>(w + ws.doc);
+  const int pool_threads = std::min(1024, (16 * H + 31) / 32 * 32);
+  pool3_kernel<<<dim3(L->n_tiles, B, 3), pool_threads, 0, stream>>>(
+      D, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), sb, ss,
+      sh, H, B, pooled);
+  gate_bwd_kernel<<<dim3(L->n_tiles, B), pool_threads, 0, stream>>>(
+      D, static_cast<const uint16_t*>(dout), d_sb, d_ss, d_sh, static_cast<const uint16_t*>(g), g_sb, g_ss, g_sh,
+      g_sd, o_coarse, H, c0, doc, dg, dg_sb, dg_ss, dg_sh, dg_sd);
+  float* pm = reinterpret_cast<float*>(w + ws.pm);
+  float* dsm = reinterpret_cast<float*>(w + ws.dsm);
+  float* dqbar = reinterpret_cast<float*>(w + ws.dqbar);
+  float* dkbar = reinterpret_cast<float*>(w + ws.dkbar);
+  float* dvbar = reinterpret_cast<float*>(w + ws.dvbar);
+  e = cudaFuncSetAttribute(coarse_bwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sizeof(CRSmem)));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(rows)", e);
+  e = cudaFuncSetAttribute(coarse_bwd_cols_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sizeof(CCSmem)));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(cols)", e);
+  coarse_bwd_rows_kernel<<<dim3((L->n_tiles + kCR - 1) / kCR, H, B), kCThreads, sizeof(CRSmem), stream>>>(
+      L->n_tiles, cand.first, cand.count, H, B, pooled, doc, o_coarse, scale, pm, dsm, ws.ld, dqbar);
+  coarse_bwd_cols_kernel<<<dim3((cand.count + kCC - 1) / kCC, H, B), kCThreads, sizeof(CCSmem), stream>>>(
+      L->n_tiles, cand.count, H, B, pooled, doc, scale, pm, dsm, ws.ld, dkbar, dvbar);
+  pool_scatter_kernel<<<dim3(L->n_tiles, B), 1024, 0, stream>>>(D, H, cand.first, cand.count, dqbar, dkbar, dvbar,
+                                                               dq, dk, dv, o_sb, o_ss, o_sh);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: coarse-branch launch", e);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_bwd_status(const void* workspace, cudaStream_t stream) {
+  if (!workspace) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd_status: cudaStreamSynchronize", e);
+  // word 0: the backward kernels; the attention workspace (right after the
+  // 256-byte header) holds the status of the forward pass in statistics mode
+  int err[2] = {0, 0};
+  e = cudaMemcpy(&err[0], workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd_status: cudaMemcpy", e);
+  e = cudaMemcpy(&err[1], static_cast<const uint8_t*>(workspace) + kBHeader, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd_status: cudaMemcpy", e);
+  const int st = err[0] != 0 ? err[0] : err[1];
+  return st == 0 ? VSA_OK : static_cast<vsa_status>(st);
+}
+
+}  // extern "C"

@@ -109,4 +109,23 @@ struct SelectWorkspace {
 };
 SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H, const vsa_params* p);
 
+// Statistics the backward pass needs from a forward call: per query row
+// ([B, H, n_tiles, 64], +inf for padding rows) the log2-sum-exp2 of the fine
+// branch's scaled logits and D = <dO, o_fine>.
+struct AttnStats {
+  float* lse;
+  float* d;
+  const void* dout;          // dO bf16 [B, S, H, 128] at element strides
+  int64_t d_sb, d_ss, d_sh;
+};
+
+// vsa_sparse_attn_fwd, or with `stats` its statistics instead of the output.
+vsa_status attn_forward(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H, const void* q,
+                        const void* k, const void* v, int64_t sb, int64_t ss, int64_t sh, const void* g,
+                        int64_t g_sb, int64_t g_ss, int64_t g_sh, int64_t g_sd, const int32_t* idx,
+                        const int32_t* cnt, int32_t kmax, const float* o_coarse, const int32_t* extra_idx,
+                        const int32_t* extra_cnt, void* out, int32_t out_dtype, int64_t o_sb, int64_t o_ss,
+                        int64_t o_sh, const AttnStats* stats, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
 }  // namespace vsa

@@ -77,6 +77,11 @@ _SIGNATURES = {
     "vsa_extra_tokens_select": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _I64, _I64, _I64,
                                        _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "vsa_extra_tokens_status": (_I32, [_P, _P]),
+    "vsa_sparse_attn_bwd_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
+    "vsa_sparse_attn_bwd": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
+                                   _P, _I64, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I64, _I64, _I64,
+                                   _P, _P, _P, _I64, _I64, _I64, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "vsa_sparse_attn_bwd_status": (_I32, [_P, _P]),
     "vsa_sparse_attn_status": (_I32, [_P, _P]),
     "vsa_sparse_attn_workspace_init": (_I32, [_P, _P]),
     "vsa_sparse_attn_failed_calls": (_I32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -191,6 +196,12 @@ class Layout:
                "vsa_extra_tokens_workspace_size")
         return n.value
 
+    def sparse_attn_bwd_workspace_size(self, B: int, H: int, params: Params) -> int:
+        n = _SZ()
+        _check(lib().vsa_sparse_attn_bwd_workspace_size(self._h, B, H, ctypes.byref(params), ctypes.byref(n)),
+               "vsa_sparse_attn_bwd_workspace_size")
+        return n.value
+
     def sparse_attn_workspace_size(self, B: int, H: int, params: Params) -> int:
         n = _SZ()
         _check(lib().vsa_sparse_attn_workspace_size(self._h, B, H, ctypes.byref(params), ctypes.byref(n)),
@@ -273,6 +284,33 @@ def sparse_attn_fwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: 
                                      out.data_ptr(), od, out.stride(0), out.stride(1), out.stride(2),
                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                      _stream_handle(stream)), "vsa_sparse_attn_fwd")
+
+
+def sparse_attn_bwd(layout: Layout, params: Params, q, k, v, g, idx, cnt, kmax: int, o_coarse, dout,
+                    dq, dk, dv, dg, workspace, stream=None) -> None:
+    """vsa_sparse_attn_bwd on torch tensors: dout bf16 [B, S, H, 128]; dq, dk, dv
+    float32 [B, S, H, 128] and dg float32 shaped like g (outputs)."""
+    B, S, H, _ = q.shape
+    sb, ss, sh = _qkv_strides(q, k, v)
+    if dout.dim() != 4 or dout.stride(-1) != 1:
+        raise ValueError("dout must be [B, S, H, 128] with a contiguous head dim")
+    if not (dq.stride() == dk.stride() == dv.stride()):
+        raise ValueError("dq, dk and dv must share strides")
+    g_sd = g.stride(3) if g.dim() == 4 else 0
+    dg_sd = dg.stride(3) if dg.dim() == 4 else 0
+    _check(lib().vsa_sparse_attn_bwd(layout.handle, ctypes.byref(params), B, H, q.data_ptr(), k.data_ptr(),
+                                     v.data_ptr(), sb, ss, sh, g.data_ptr(), g.stride(0), g.stride(1), g.stride(2),
+                                     g_sd, idx.data_ptr(), cnt.data_ptr(), kmax, o_coarse.data_ptr(),
+                                     dout.data_ptr(), dout.stride(0), dout.stride(1), dout.stride(2),
+                                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dq.stride(0), dq.stride(1),
+                                     dq.stride(2), dg.data_ptr(), dg.stride(0), dg.stride(1), dg.stride(2), dg_sd,
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream)), "vsa_sparse_attn_bwd")
+
+
+def sparse_attn_bwd_status(workspace, stream=None) -> int:
+    """Synchronises the stream; the backward pass's status (OK or ERR_TIMEOUT)."""
+    return lib().vsa_sparse_attn_bwd_status(workspace.data_ptr(), _stream_handle(stream))
 
 
 def sparse_attn_status(workspace, stream=None) -> int:

@@ -373,6 +373,55 @@ vsa_status vsa_sparse_attn_workspace_init(void* workspace, cudaStream_t stream);
  * a failure of any earlier call, not only the latest one. */
 vsa_status vsa_sparse_attn_failed_calls(const void* workspace, cudaStream_t stream, uint32_t* count);
 
+/* ------------------------------------------------------------------------ */
+/* Backward pass                                                             */
+/* ------------------------------------------------------------------------ */
+
+vsa_status vsa_sparse_attn_bwd_workspace_size(const vsa_layout* layout, int32_t B, int32_t H,
+                                              const vsa_params* params, size_t* bytes);
+
+/* vsa_sparse_attn_bwd: gradients of sum(out * dout) with respect to q, k, v
+ * and g, for the forward of vsa_coarse_select + vsa_sparse_attn_fwd with the
+ * same params, the block selection held fixed (piecewise constant in the
+ * inputs). The pages train and distil checkpoints against these modes ("BSAI
+ * FastH3 Native VSA (recipe)"; "ComfyUI-Ref2VA-VSA", "The Solution:
+ * Ref2VAVSAGatePatch") without spelling the backward out; this is the exact
+ * derivative of the forward: the fine branch's attention backward over each
+ * query tile's key set, the gate's product rule, and the coarse branch's
+ * tile-level softmax backward flowing back through the mean pooling.
+ *
+ *  q, k, v, strides : as vsa_coarse_select; g and its strides as
+ *                     vsa_sparse_attn_fwd.
+ *  idx, cnt, kmax   : the lists of vsa_coarse_select (same params).
+ *  o_coarse         : the o_coarse of vsa_coarse_select.
+ *  dout             : bf16 [B, S, H, 128] at element strides dout_stride_*.
+ *  dq, dk, dv       : fp32 [B, S, H, 128] out at element strides
+ *                     grad_stride_* (16-byte multiples), every token written.
+ *  dg               : fp32 out shaped like g ([B, S, H] with dg_stride_d = 0,
+ *                     or [B, S, H, 128] with dg_stride_d > 0, as g).
+ *  workspace        : vsa_sparse_attn_bwd_workspace_size bytes, 256-byte aligned.
+ * Errors: UNSUPPORTED for the Spark-Reweight coarse branch and for
+ * extra_tokens > 0 (not differentiated on the GPU). A kernel wait that runs
+ * out is reported by vsa_sparse_attn_bwd_status. */
+vsa_status vsa_sparse_attn_bwd(const vsa_layout* layout, const vsa_params* params,
+                               int32_t B, int32_t H, const void* q, const void* k, const void* v,
+                               int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                               const void* g, int64_t g_stride_b, int64_t g_stride_s,
+                               int64_t g_stride_h, int64_t g_stride_d,
+                               const int32_t* idx, const int32_t* cnt, int32_t kmax,
+                               const float* o_coarse, const void* dout, int64_t dout_stride_b,
+                               int64_t dout_stride_s, int64_t dout_stride_h,
+                               float* dq, float* dk, float* dv, int64_t grad_stride_b,
+                               int64_t grad_stride_s, int64_t grad_stride_h,
+                               float* dg, int64_t dg_stride_b, int64_t dg_stride_s,
+                               int64_t dg_stride_h, int64_t dg_stride_d,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream` and reads the status a previous vsa_sparse_attn_bwd
+ * left in `workspace`: VSA_OK or VSA_ERR_TIMEOUT. No counterpart on the pages
+ * (error reporting of this library). */
+vsa_status vsa_sparse_attn_bwd_status(const void* workspace, cudaStream_t stream);
+
 /* Synchronises `stream` and reads the error word a previous
  * vsa_sparse_attn_fwd left in `workspace`: VSA_OK, VSA_ERR_TIMEOUT (a bounded
  * wait in the kernel ran out; the output is incomplete) or VSA_ERR_CUDA. */
