@@ -41,10 +41,10 @@ COARSES = {"mean": 0, "reweight": 1}
 
 
 def captured_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed counter capture of
-    this workload (profiles/vsa_attn_kernel_<workload>_dram.json), or None when
-    there is none or the kernel code changed since the counters were taken
-    (the capture records the code hash of kernel_code_hash())."""
+    """DRAM bytes per attention call (the sum over the kernels the committed
+    counter capture of this workload lists, profiles/vsa_attn_kernel_<workload>_dram.json),
+    or None when there is none or the kernel code changed since the counters
+    were taken (the capture records the code hash of kernel_code_hash())."""
     path = os.path.join(ROOT, "profiles", "vsa_attn_kernel_%s_dram.json" % workload)
     try:
         with open(path) as f:
@@ -53,7 +53,7 @@ def captured_traffic(workload: str):
         return None
     if cap.get("kernel_code_sha256_16") != kernel_code_hash():
         return None
-    return int(cap["dram_bytes_read"]) + int(cap["dram_bytes_write"])
+    return sum(int(k["dram_bytes_read"]) + int(k["dram_bytes_write"]) for k in cap["kernels"].values())
 
 
 def kernel_code_hash() -> str:
@@ -352,6 +352,47 @@ def valid_flop_extra(counts, extra_cnt, rows_dense, n_cond):
     return 4.0 * 128.0 * float((e * counts[None, None, :].astype(np.float64)).sum())
 
 
+def measure_backward(wl, params, q, k, v, g, dev, stream, n_calls, fwd_flop):
+    """vsa_sparse_attn_bwd on the inputs of this run (a seeded dO): ms per call.
+    Its tensor work is 7 products of 64 x 64 x 128 per (query tile, key tile)
+    pair (S, dP and dQ per query tile; S^T, dP^T, dK and dV per key tile)
+    against the forward's 2, so the executed-work rate counts 3.5 x the
+    forward's valid FLOP."""
+    import torch
+    from block_sparse_video_geometry_b200 import vsa
+    lay = vsa.Layout(wl.segments(), wl.seq_len)
+    with torch.cuda.stream(stream):
+        fwd = vsa.Forward(lay, params, wl.B, wl.H, device=dev, stream=stream)
+        gen = torch.Generator(device=dev).manual_seed(77)
+        dout = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+        grads = [torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3)]
+        dg = torch.empty(g.shape, dtype=torch.float32, device=dev)
+        ws = torch.empty(lay.sparse_attn_bwd_workspace_size(wl.B, wl.H, params), dtype=torch.uint8, device=dev)
+    vsa.coarse_select(lay, params, q, k, v, fwd.idx, fwd.cnt, fwd.o_coarse, fwd.ws_select, stream)
+    bwd = lambda: vsa.sparse_attn_bwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse, dout,
+                                      *grads, dg, ws, stream)
+    for _ in range(2):
+        bwd()
+    ms = []
+    for _ in range(n_calls):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        bwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    if vsa.sparse_attn_bwd_status(ws, stream) != vsa.OK:
+        raise RuntimeError("backward: a kernel wait ran out")
+    t = statistics.median(ms)
+    res = {"workload": describe(wl) + ", backward", "ms_per_call": t,
+           "tflops_executed": 3.5 * fwd_flop / (t * 1e-3) / 1e12, "calls": n_calls,
+           "flop_accounting": "3.5 x the forward's valid FLOP (7 tile products per attended pair vs 2)",
+           "dout": "seeded N(0, 1) in bf16"}
+    del fwd, dout, grads, dg, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     from block_sparse_video_geometry_b200 import vsa, workloads as W
@@ -489,6 +530,7 @@ def run_ours(args):
         configs["5s_extra_tokens16"] = measure_config(
             "extra tokens 16", wl, mk(extra_tokens=16), q, k, v, g, dev, stream, out_dtype, peak, max(3, n // 2),
             inputs_note=note)
+        configs["5s_backward"] = measure_backward(wl, mk(), q, k, v, g, dev, stream, max(3, n // 2), flop)
         configs["5s_keep100"] = measure_config("keep 100%", wl.with_(keep=1.0), mk(keep=1.0), q, k, v, g, dev,
                                                stream, out_dtype, peak, max(3, n // 2), dense=dense_ms,
                                                inputs_note=note)
@@ -526,11 +568,12 @@ def run_ours(args):
                 ", %d extra tokens" % args.extra_tokens if args.extra_tokens else ""),
                        "B": wl.B, "seq_len": wl.seq_len, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
                        "l2": "inputs (2.5 GB) larger than L2; no flush"},
-            "roofline": {"bound": "tensor", "kernel": "vsa_attn_kernel", "achieved": achieved, "peak": peak,
+            "roofline": {"bound": "tensor", "kernel": "vsa_sparse_attn_fwd (pair_attn_kernel + vsa_attn_kernel)",
+                         "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
                          "traffic": (captured_traffic(args.workload) if args.sink is None and args.coarse == "mean"
                                      and args.gate == "token" and args.out_dtype == "f32" else None),
-                         "traffic_unit": "bytes per launch (ncu dram read + write)",
+                         "traffic_unit": "bytes per call (ncu dram read + write of the two attention kernels)",
                          "peak_source": "%s bf16_tflops (burst: the kernel is timed alone, once per call)" % src,
                          "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
                          "flop_per_launch": flop, "ms_per_launch": att_ms},
