@@ -18,7 +18,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3",
                      "-I" + INCLUDE, "-I" + CSRC]
 
-LIBVSA_SOURCES = ["vsa_layout.cpp", "vsa_select.cu", "vsa_attn.cu", "vsa_extra.cu", "vsa_bwd.cu"]
+LIBVSA_SOURCES = ["vsa_layout.cpp", "vsa_select.cu", "vsa_select_tc.cu", "vsa_attn.cu", "vsa_extra.cu", "vsa_bwd.cu"]
 LIBVSA = os.path.join(PKG, "libvsa.so")
 CHECK_SOURCE = os.path.join(ROOT, "tests", "native", "mma_check.cu")
 CHECK_LIB = os.path.join(ROOT, "tests", "native", "libmma_check.so")

@@ -100,14 +100,31 @@ float effective_scale(const vsa_params* p);
 vsa_status check_qkv(const void* q, const void* k, const void* v, int64_t sb, int64_t ss,
                      int64_t sh, int32_t B, int32_t H);
 
-// Workspace layout of vsa_coarse_select.
+// Workspace layout of vsa_coarse_select. Bytes [0, 256): status word and
+// count of failed calls; the pooled means [3, B, H, n_tiles, 128] fp32 follow.
+// VSA_COARSE_MEAN runs the tensor-core kernels (vsa_select_tc.cu): Kbar and
+// Vbar split into hi/lo bf16 chunks of 64 candidates (32 KB per chunk:
+// [term][d half][64][128 B], 128-byte swizzled), per-query-tile max score and
+// its candidate, per-block adaptive sums, and per-query-tile selection marks.
+// VSA_COARSE_REWEIGHT runs the fp32 kernels of vsa_select.cu over a score
+// matrix in the workspace.
+constexpr size_t kSelectHeader = 256;
 struct SelectWorkspace {
   size_t pooled, scores, stats, total;
   size_t anchor, summaries, bias;   // VSA_COARSE_REWEIGHT only: [B,H,128], [2,B,H,Nc,128], [B,H,Nc]
-  int32_t n_row_blocks;   // 64-query-tile blocks of the coarse kernel
+  size_t ksplit, vsplit, rowmax, rowarg, bits;   // VSA_COARSE_MEAN only
+  int32_t n_row_blocks;   // query-tile blocks: 64 per block (fp32 kernels), 128 (tensor-core kernels)
   int32_t ld_scores;      // score row stride: Nc rounded up to 64
+  int32_t n_chunks;       // 64-candidate chunks
 };
 SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H, const vsa_params* p);
+
+// The tensor-core coarse branch + selection (VSA_COARSE_MEAN), after the
+// pooling kernel filled the pooled means and the split chunks of `ws`.
+vsa_status select_tc(const vsa_layout* L, const vsa_params* p, int32_t B, int32_t H, const SelectWorkspace& ws,
+                     void* workspace, int32_t* idx, int32_t* cnt, float* o_coarse, uint64_t stall_ns,
+                     cudaStream_t stream);
+size_t select_tc_smem_bytes();
 
 // Statistics the backward pass needs from a forward call: per query row
 // ([B, H, n_tiles, 64], +inf for padding rows) the log2-sum-exp2 of the fine

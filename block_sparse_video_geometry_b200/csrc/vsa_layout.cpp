@@ -79,24 +79,40 @@ vsa_status check_qkv(const void* q, const void* k, const void* v, int64_t sb, in
 SelectWorkspace select_workspace(const vsa_layout* L, int32_t B, int32_t H, const vsa_params* p) {
   SelectWorkspace w{};
   const size_t bh = static_cast<size_t>(B) * H;
-  w.n_row_blocks = (L->n_tiles + 63) / 64;
-  w.ld_scores = (candidates(L, p->sink).count + 63) / 64 * 64;
-  size_t off = 0;
+  const size_t nt = static_cast<size_t>(L->n_tiles);
+  const int32_t nc = candidates(L, p->sink).count;
+  const bool tc = p->coarse == VSA_COARSE_MEAN;
+  w.n_row_blocks = tc ? (L->n_tiles + 127) / 128 : (L->n_tiles + 63) / 64;
+  w.ld_scores = (nc + 63) / 64 * 64;
+  w.n_chunks = (nc + 63) / 64;
+  size_t off = kSelectHeader;
   w.pooled = off;
-  off = align_up(off + 3 * bh * L->n_tiles * kHeadDim * sizeof(float), 256);
-  w.scores = off;
-  off = align_up(off + bh * L->n_tiles * static_cast<size_t>(w.ld_scores) * sizeof(float), 256);
+  off = align_up(off + 3 * bh * nt * kHeadDim * sizeof(float), 256);
   w.stats = off;
   off = align_up(off + bh * w.n_row_blocks * 2 * sizeof(double), 256);
-  w.anchor = w.summaries = w.bias = off;
-  if (p->coarse == VSA_COARSE_REWEIGHT) {
-    const size_t nc = static_cast<size_t>(candidates(L, p->sink).count);
+  w.scores = w.anchor = w.summaries = w.bias = off;
+  w.ksplit = w.vsplit = w.rowmax = w.rowarg = w.bits = off;
+  if (tc) {
+    const size_t chunks = bh * static_cast<size_t>(w.n_chunks) * 32768u;
+    w.ksplit = off;
+    off = align_up(off + chunks, 256);
+    w.vsplit = off;
+    off = align_up(off + chunks, 256);
+    w.rowmax = off;
+    off = align_up(off + bh * nt * sizeof(float), 256);
+    w.rowarg = off;
+    off = align_up(off + bh * nt * sizeof(int32_t), 256);
+    w.bits = off;
+    off = align_up(off + bh * nt * 2 * static_cast<size_t>(w.n_chunks) * sizeof(uint32_t), 256);
+  } else {
+    w.scores = off;
+    off = align_up(off + bh * nt * static_cast<size_t>(w.ld_scores) * sizeof(float), 256);
     w.anchor = off;
     off = align_up(off + bh * kHeadDim * sizeof(float), 256);
     w.summaries = off;
-    off = align_up(off + 2 * bh * nc * kHeadDim * sizeof(float), 256);
+    off = align_up(off + 2 * bh * static_cast<size_t>(nc) * kHeadDim * sizeof(float), 256);
     w.bias = off;
-    off = align_up(off + bh * nc * sizeof(float), 256);
+    off = align_up(off + bh * static_cast<size_t>(nc) * sizeof(float), 256);
   }
   w.total = off;
   return w;
@@ -294,7 +310,7 @@ const char* vsa_status_string(vsa_status s) {
   return "unknown status";
 }
 
-int32_t vsa_version(void) { return (1 << 16) | 3; }
+int32_t vsa_version(void) { return (1 << 16) | 4; }
 
 const char* vsa_last_error_detail(void) { return g_detail; }
 

@@ -1,16 +1,24 @@
-// Coarse branch and block selection.
+// Coarse branch and block selection: the entry points, the pooling kernel,
+// and the fp32 kernels of the Spark-Reweight coarse branch.
 //
 // 1. pool_kernel      : mean of Q, K, V over the valid tokens of every tile
 //                       (fp32), read straight from the natural [B, S, H, 128]
-//                       layout through the tile's token list.
-// 2. coarse_kernel    : for a block of 64 query tiles of one (batch, head):
+//                       layout through the tile's token list. For
+//                       VSA_COARSE_MEAN it also writes Kbar and Vbar of the
+//                       candidate tiles as hi/lo bf16 chunks for the tensor-core
+//                       kernels of vsa_select_tc.cu, which then do the scores,
+//                       the selection and the coarse softmax on chip.
+// VSA_COARSE_REWEIGHT runs:
+// 2. anchor_kernel, reweight_kernel: the Spark-Reweight summaries.
+// 3. coarse_kernel    : for a block of 64 query tiles of one (batch, head):
 //                       s = scale * Qbar Kbar^T against every candidate
 //                       key tile (the video tiles, or every tile with
-//                       VSA_SINK_OFF), in fp32 FMA; the scores go to the workspace for selection
-//                       and feed an online softmax against Vbar that yields
-//                       o_coarse. With the adaptive threshold it also sums s
-//                       and s^2 in fp64 per block.
-// 3. select_kernel    : one warp per query tile: radix select of the k-th
+//                       VSA_SINK_OFF), in fp32 FMA; the scores go to the
+//                       workspace for selection, and the reweighted logits feed
+//                       an online softmax against V~ that yields o_coarse. With
+//                       the adaptive threshold it also sums s and s^2 in fp64
+//                       per block.
+// 4. select_kernel    : one warp per query tile: radix select of the k-th
 //                       largest score (ties -> lower tile) or the adaptive
 //                       threshold mean + tau * std, emitted as an ascending
 //                       list of candidate ordinals.
@@ -19,16 +27,17 @@
 // Central de Atencion Dispersa y Compilador Comfy", "Atencion dispersa por
 // bloques" (top-k keep percent; Sol-Attn per-head threshold in sigmas; VSA
 // coarse compression branch); "Spark-H3 ...", "Que cambia Spark-Attn" (the
-// compressed branch summarises K/V by mean pooling).
+// compressed branch summarises K/V by mean pooling, Spark-Reweight by anchor
+// weights).
 //
-// These kernels are bound by HBM (pooling reads Q, K, V once) and by fp32
-// FMA throughput (scores and the coarse softmax, ~2 * Nt * Nc * 128 FMA per
-// head). Scores stay fp32 end to end so that the selected sets match an fp64
-// evaluation except on near-ties.
+// Pooling is bound by HBM (it reads Q, K, V once). Scores stay fp32-accurate
+// end to end so that the selected sets match an fp64 evaluation except on
+// near-ties.
 
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
 #include <cmath>
 
@@ -39,6 +48,7 @@ namespace vsa {
 namespace {
 
 constexpr int kPoolMaxThreads = 1024;
+std::atomic<uint64_t> g_select_stall_ns{0};   // vsa_debug_inject_select_wait_timeout
 constexpr int kCoarseRows = 64;       // query tiles per coarse block
 constexpr int kCoarseCols = 64;       // candidate key tiles per streamed chunk
 constexpr int kCoarseThreads = 256;
@@ -48,19 +58,51 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ------------------------------------------------------------------ pooling
-// grid (n_tiles, B, 3), block = min(1024, 16 * H) rounded up to a warp.
-// Thread c handles head c / 16, dims 8 * (c % 16) .. + 7.
+// The split Kbar / Vbar chunks of the tensor-core kernels (VSA_COARSE_MEAN):
+// candidate c of (b, h) is row c % 64 of chunk c / 64; a chunk is
+// [term: hi, lo][d half][64 rows][128 B] with 16-byte unit u of a row at
+// 16 (u ^ (row & 7)) (the 128-byte swizzle the MMA descriptors expect).
+struct SplitOut {
+  uint8_t* kv[2];           // K, V chunks, or null (fp32 kernels)
+  int32_t cand0, n_cand, n_chunks;
+};
+
+__device__ __forceinline__ uint32_t bf16_pair_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// grid (n_tiles + pad, B, 3), block = min(1024, 16 * H) rounded up to a warp.
+// Thread c handles head c / 16, dims 8 * (c % 16) .. + 7. Blocks past n_tiles
+// (split output only) zero the pad rows of the last chunk. Block (0, 0, 0)
+// also clears the call's status word.
 __global__ void __launch_bounds__(kPoolMaxThreads)
 pool_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
             const uint16_t* __restrict__ v, int64_t sb, int64_t ss, int64_t sh, int H, int B,
-            float* __restrict__ pooled) {
+            float* __restrict__ pooled, SplitOut so, int* __restrict__ status) {
   const int tile = blockIdx.x, b = blockIdx.y, which = blockIdx.z;
+  if (tile == 0 && b == 0 && which == 0 && threadIdx.x == 0) status[0] = 0;
+  const int nchunks = H * 16;
+  if (tile >= L.n_tiles) {
+    if (which == 0) return;
+    const int c = so.n_cand + (tile - L.n_tiles);
+    for (int t = threadIdx.x; t < nchunks; t += blockDim.x) {
+      const int h = t >> 4, d0 = (t & 15) * 8, r = c & 63, u = (d0 & 63) >> 3;
+      uint8_t* dst = so.kv[which - 1] + ((static_cast<size_t>(b) * H + h) * so.n_chunks + (c >> 6)) * 32768u +
+                     (d0 >> 6) * 8192 + r * 128 + ((u ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(dst + 16384) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    return;
+  }
   const uint16_t* x = which == 0 ? q : (which == 1 ? k : v);
   __shared__ int tok[kTile];
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) tok[i] = L.perm[tile * kTile + i];
   __syncthreads();
   const float n = static_cast<float>(L.count[tile]);
-  const int nchunks = H * 16;
+  const int cand = tile - so.cand0;
+  const bool split = which > 0 && so.kv[0] != nullptr && cand >= 0 && cand < so.n_cand;
   for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
     const int h = c >> 4, d0 = (c & 15) * 8;
     const uint16_t* base = x + b * sb + h * sh + d0;
@@ -78,9 +120,25 @@ pool_kernel(DevLayout L, const uint16_t* __restrict__ q, const uint16_t* __restr
         acc[6] += bf16lo(w.w); acc[7] += bf16hi(w.w);
       }
     }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] /= n;
     float* dst = pooled + ((((static_cast<size_t>(which) * B + b) * H + h) * L.n_tiles + tile) * kHeadDim + d0);
-    reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0] / n, acc[1] / n, acc[2] / n, acc[3] / n);
-    reinterpret_cast<float4*>(dst)[1] = make_float4(acc[4] / n, acc[5] / n, acc[6] / n, acc[7] / n);
+    reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    reinterpret_cast<float4*>(dst)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    if (split) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hi[e] = bf16_pair_rn(acc[2 * e], acc[2 * e + 1]);
+        lo[e] = bf16_pair_rn(acc[2 * e] - __uint_as_float(hi[e] << 16),
+                             acc[2 * e + 1] - __uint_as_float(hi[e] & 0xFFFF0000u));
+      }
+      const int r = cand & 63, u = (d0 & 63) >> 3;
+      uint8_t* o = so.kv[which - 1] + ((static_cast<size_t>(b) * H + h) * so.n_chunks + (cand >> 6)) * 32768u +
+                   (d0 >> 6) * 8192 + r * 128 + ((u ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(o + 16384) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
   }
 }
 
@@ -547,11 +605,16 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
   const SelectWorkspace ws = select_workspace(L, B, H, p);
   const Candidates cand = candidates(L, p->sink);
   if (workspace_bytes < ws.total) return VSA_ERR_WORKSPACE_TOO_SMALL;
+  const bool reweight = p->coarse == VSA_COARSE_REWEIGHT;
+  if (!reweight && cand.count > 65535) {   // 16-bit histogram counters of the tensor-core kernel
+    set_detail("vsa_coarse_select: more than 65535 candidate key tiles");
+    return VSA_ERR_UNSUPPORTED;
+  }
 
   const int ld = ws.ld_scores;
   const size_t row_bytes = static_cast<size_t>(ld) * sizeof(float);
   const int rows_per_block = static_cast<int>(std::min<size_t>(kSelectWarps, (200u << 10) / row_bytes));
-  if (rows_per_block < 1) return VSA_ERR_UNSUPPORTED;   // more than 51200 candidate tiles
+  if (reweight && rows_per_block < 1) return VSA_ERR_UNSUPPORTED;   // more than 51200 candidate tiles
 
   char* w = static_cast<char*>(workspace);
   float* pooled = reinterpret_cast<float*>(w + ws.pooled);
@@ -563,27 +626,34 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
   int32_t kmax = 0;
   vsa_select_kmax(L, p, &kmax);
 
+  SplitOut so{};
+  so.kv[0] = reweight ? nullptr : reinterpret_cast<uint8_t*>(w + ws.ksplit);
+  so.kv[1] = reweight ? nullptr : reinterpret_cast<uint8_t*>(w + ws.vsplit);
+  so.cand0 = cand.first;
+  so.n_cand = cand.count;
+  so.n_chunks = ws.n_chunks;
+  const int pad = reweight ? 0 : ws.n_chunks * 64 - cand.count;
   const int pool_threads = std::min(kPoolMaxThreads, (16 * H + 31) / 32 * 32);
-  pool_kernel<<<dim3(L->n_tiles, B, 3), pool_threads, 0, stream>>>(
+  pool_kernel<<<dim3(L->n_tiles + pad, B, 3), pool_threads, 0, stream>>>(
       D, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-      static_cast<const uint16_t*>(v), sb, ss, sh, H, B, pooled);
+      static_cast<const uint16_t*>(v), sb, ss, sh, H, B, pooled, so, static_cast<int*>(workspace));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: pool launch", e);
+  if (!reweight)
+    return select_tc(L, p, B, H, ws, workspace, idx, cnt, o_coarse, g_select_stall_ns.load(std::memory_order_relaxed),
+                     stream);
 
-  const bool reweight = p->coarse == VSA_COARSE_REWEIGHT;
   float* anchor = reinterpret_cast<float*>(w + ws.anchor);
   float* summaries = reinterpret_cast<float*>(w + ws.summaries);
   float* rbias = reinterpret_cast<float*>(w + ws.bias);
-  if (reweight) {
-    anchor_kernel<<<dim3(H, B), kHeadDim, 0, stream>>>(D, H, pooled, anchor);
-    reweight_kernel<<<dim3(cand.count, B), kReweightThreads, 0, stream>>>(
-        D, cand.first, cand.count, static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), sb, ss, sh, H,
-        B, scale, anchor, summaries, rbias);
-  }
+  anchor_kernel<<<dim3(H, B), kHeadDim, 0, stream>>>(D, H, pooled, anchor);
+  reweight_kernel<<<dim3(cand.count, B), kReweightThreads, 0, stream>>>(
+      D, cand.first, cand.count, static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), sb, ss, sh, H,
+      B, scale, anchor, summaries, rbias);
 
   const size_t coarse_smem = sizeof(CoarseSmem);
-  auto ck = adaptive ? (reweight ? coarse_kernel<true, true> : coarse_kernel<true, false>)
-                     : (reweight ? coarse_kernel<false, true> : coarse_kernel<false, false>);
-  cudaError_t e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(coarse_smem));
+  auto ck = adaptive ? coarse_kernel<true, true> : coarse_kernel<false, true>;
+  e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(coarse_smem));
   if (e != cudaSuccess) return cuda_fail("vsa_coarse_select: cudaFuncSetAttribute(coarse)", e);
   ck<<<dim3(ws.n_row_blocks, H, B), kCoarseThreads, coarse_smem, stream>>>(
       L->n_tiles, cand.first, cand.count, H, B, pooled, scale, scores, ld, o_coarse, stats, summaries, rbias);
@@ -600,6 +670,37 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
   return VSA_OK;
 }
 
+vsa_status vsa_coarse_select_workspace_init(void* workspace, cudaStream_t stream) {
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kSelectHeader, stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_workspace_init: cudaMemsetAsync", e);
+  return VSA_OK;
+}
+
+vsa_status vsa_coarse_select_status(const void* workspace, cudaStream_t stream) {
+  if (!workspace) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_status: cudaStreamSynchronize", e);
+  int err = 0;
+  e = cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_status: cudaMemcpy", e);
+  return err == 0 ? VSA_OK : static_cast<vsa_status>(err);
+}
+
+vsa_status vsa_coarse_select_failed_calls(const void* workspace, cudaStream_t stream, uint32_t* count) {
+  if (!workspace || !count) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_failed_calls: cudaStreamSynchronize", e);
+  e = cudaMemcpy(count, static_cast<const int*>(workspace) + 1, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_failed_calls: cudaMemcpy", e);
+  return VSA_OK;
+}
+
+vsa_status vsa_debug_inject_select_wait_timeout(uint64_t timeout_ns) {
+  g_select_stall_ns.store(timeout_ns, std::memory_order_relaxed);
+  return VSA_OK;
+}
+
 }  // extern "C"
 
 // -------------------------------------------------------------------------
@@ -609,7 +710,7 @@ vsa_status vsa_coarse_select(const vsa_layout* L, const vsa_params* p, int32_t B
 // host framework that plans every device allocation ahead of time and forbids
 // allocations outside its plan, or callers that must not pay the device-wide
 // synchronisation and latency of cudaMalloc in the middle of a step. For them
-// the selection scratch (pooled means, score matrix, adaptive partial sums)
+// the selection scratch (status words, pooled means, split chunks, marks)
 // lives in the fixed buffer below, which is part of the library's device
 // image: every GPU that loads libvsa holds these 32 MiB until the process
 // exits. Workloads whose scratch does not fit are refused, not truncated.
@@ -627,6 +728,31 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// The built-in buffer's device address on the current device, looked up once
+// per device with that device current (host code must not use the array's
+// name as a device address). A process that resets a device with
+// cudaDeviceReset must not call the allocation-free entry points afterwards:
+// the cached address belongs to the destroyed context.
+vsa_status noalloc_scratch(void** scratch) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_noalloc: cudaGetDevice", e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) {
+    set_detail("vsa_coarse_select_noalloc: device ordinal beyond 63");
+    return VSA_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      g_noalloc_ptr[dev] = nullptr;
+      return cuda_fail("vsa_coarse_select_noalloc: cudaGetSymbolAddress", e);
+    }
+  }
+  *scratch = g_noalloc_ptr[dev];
+  return VSA_OK;
+}
 
 }  // namespace
 }  // namespace vsa
@@ -648,27 +774,16 @@ extern "C" vsa_status vsa_coarse_select_noalloc(const vsa_layout* L, const vsa_p
     set_detail(msg);
     return VSA_ERR_UNSUPPORTED;
   }
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail("vsa_coarse_select_noalloc: cudaGetDevice", e);
-  if (dev < 0 || dev >= kNoAllocMaxDevices) {
-    set_detail("vsa_coarse_select_noalloc: device ordinal beyond 63");
-    return VSA_ERR_UNSUPPORTED;
-  }
   void* scratch = nullptr;
-  {
-    // Host code must not use the array's name as a device address: the
-    // address is looked up once per device, with that device current.
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-      e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
-      if (e != cudaSuccess) {
-        g_noalloc_ptr[dev] = nullptr;
-        return cuda_fail("vsa_coarse_select_noalloc: cudaGetSymbolAddress", e);
-      }
-    }
-    scratch = g_noalloc_ptr[dev];
-  }
+  st = noalloc_scratch(&scratch);
+  if (st != VSA_OK) return st;
   return vsa_coarse_select(L, p, B, H, q, k, v, sb, ss, sh, idx, cnt, o_coarse, scratch,
                            kNoAllocScratchBytes, stream);
+}
+
+extern "C" vsa_status vsa_coarse_select_noalloc_status(cudaStream_t stream) {
+  void* scratch = nullptr;
+  vsa_status st = noalloc_scratch(&scratch);
+  if (st != VSA_OK) return st;
+  return vsa_coarse_select_status(scratch, stream);
 }

@@ -69,6 +69,11 @@ _SIGNATURES = {
                                  _P, _P, _P, _P, _SZ, _P]),
     "vsa_coarse_select_noalloc": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
                                          _P, _P, _P, _P]),
+    "vsa_coarse_select_workspace_init": (_I32, [_P, _P]),
+    "vsa_coarse_select_status": (_I32, [_P, _P]),
+    "vsa_coarse_select_failed_calls": (_I32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "vsa_coarse_select_noalloc_status": (_I32, [_P]),
+    "vsa_debug_inject_select_wait_timeout": (_I32, [ctypes.c_uint64]),
     "vsa_sparse_attn_workspace_size": (_I32, [_P, _I32, _I32, ctypes.POINTER(Params), ctypes.POINTER(_SZ)]),
     "vsa_sparse_attn_fwd": (_I32, [_P, ctypes.POINTER(Params), _I32, _I32, _P, _P, _P, _I64, _I64, _I64,
                                    _P, _I64, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _P, _P, _I32, _I64, _I64,
@@ -239,6 +244,30 @@ def coarse_select_noalloc(layout: Layout, params: Params, q, k, v, idx, cnt, o_c
            "vsa_coarse_select_noalloc")
 
 
+def coarse_select_workspace_init(workspace, stream=None) -> None:
+    """Zeroes the selection workspace header (and its count of failed calls)."""
+    _check(lib().vsa_coarse_select_workspace_init(workspace.data_ptr(), _stream_handle(stream)),
+           "vsa_coarse_select_workspace_init")
+
+
+def coarse_select_status(workspace, stream=None) -> int:
+    """Synchronises the stream and returns the selection call's status word (OK or ERR_TIMEOUT)."""
+    return lib().vsa_coarse_select_status(workspace.data_ptr(), _stream_handle(stream))
+
+
+def coarse_select_failed_calls(workspace, stream=None) -> int:
+    """Synchronises the stream; selection calls that recorded an error since the header was zeroed."""
+    n = ctypes.c_uint32()
+    _check(lib().vsa_coarse_select_failed_calls(workspace.data_ptr(), _stream_handle(stream), ctypes.byref(n)),
+           "vsa_coarse_select_failed_calls")
+    return n.value
+
+
+def coarse_select_noalloc_status(stream=None) -> int:
+    """coarse_select_status of the built-in buffer of coarse_select_noalloc (current device)."""
+    return lib().vsa_coarse_select_noalloc_status(_stream_handle(stream))
+
+
 def extra_tokens_select(layout: Layout, params: Params, q, k, idx, cnt, kmax: int, extra_idx, extra_cnt,
                         workspace, stream=None) -> None:
     """vsa_extra_tokens_select: extra_idx int32 [B, H, n_tiles, E], extra_cnt int32 [B, H, n_tiles] out."""
@@ -338,6 +367,13 @@ def debug_inject_wait_timeout(timeout_ns):
     lib().vsa_debug_inject_wait_timeout(int(timeout_ns))
 
 
+def debug_inject_select_wait_timeout(timeout_ns):
+    """Test hook: while timeout_ns > 0, each coarse_select (mean coarse branch)
+    runs into a bounded wait that nothing completes and reports ERR_TIMEOUT
+    through coarse_select_status; 0 disarms."""
+    lib().vsa_debug_inject_select_wait_timeout(int(timeout_ns))
+
+
 class Forward:
     """Holds the buffers of one shape and runs the two calls of the forward
     pass (caller-owned torch buffers; no allocation inside the calls)."""
@@ -359,6 +395,7 @@ class Forward:
         self.ws_attn = torch.empty(layout.sparse_attn_workspace_size(B, H, params), dtype=torch.uint8,
                                    device=device)
         sparse_attn_workspace_init(self.ws_attn, stream)
+        coarse_select_workspace_init(self.ws_select, stream)
         self.out_dtype = out_dtype or torch.float32
         self.stream = stream
         self.extra_idx = self.extra_cnt = self.ws_extra = None
@@ -382,8 +419,8 @@ class Forward:
         return out
 
     def pooled(self):
-        """Pooled means [3, B, H, n_tiles, 128] left in the selection workspace."""
+        """Pooled means [3, B, H, n_tiles, 128] left in the selection workspace (from byte 256)."""
         import torch
         n = 3 * self.B * self.H * self.layout.info.n_tiles * HEAD_DIM
-        return self.ws_select[: 4 * n].view(torch.float32).view(3, self.B, self.H, self.layout.info.n_tiles,
+        return self.ws_select[256: 256 + 4 * n].view(torch.float32).view(3, self.B, self.H, self.layout.info.n_tiles,
                                                                 HEAD_DIM)

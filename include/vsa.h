@@ -223,13 +223,22 @@ vsa_status vsa_coarse_select_workspace_size(const vsa_layout* layout, int32_t B,
  *                   (the scores the selection uses); with COARSE_REWEIGHT the
  *                   Spark-Reweight form of vsa_coarse_mode.
  *  workspace      : device scratch of vsa_coarse_select_workspace_size bytes,
- *                   256-byte aligned. Its first 3*B*H*n_tiles*128 floats hold
- *                   the pooled means [3 (q,k,v), B, H, n_tiles, 128] after
- *                   the call.
+ *                   256-byte aligned. Bytes [0, 256) hold the call's status
+ *                   word and the count of failed calls (see
+ *                   vsa_coarse_select_workspace_init); from byte 256,
+ *                   3*B*H*n_tiles*128 floats hold the pooled means
+ *                   [3 (q,k,v), B, H, n_tiles, 128] after the call.
  * All query tiles are processed, conditioning tiles included (under
  * EXACT_KV_AND_ROWS their lists are ignored by vsa_sparse_attn_fwd).
- * Pooling, scores, thresholds and the coarse softmax are fp32 (adaptive
- * mean/std accumulate in fp64). */
+ * Pooling is fp32. With COARSE_MEAN the scores and the coarse softmax run on
+ * the tensor cores with each fp32 mean split into two bf16 terms (three
+ * products, fp32 accumulation: fp32-class error), the score matrix stays on
+ * chip, and the kernels wait on their own copies and MMAs with bounded waits
+ * (VSA_ERR_TIMEOUT in vsa_coarse_select_status when one runs out; the lists
+ * are then incomplete, but every consumer in this library clamps list
+ * lengths and entries, so nothing reads out of bounds). With COARSE_REWEIGHT
+ * they are fp32 FMA. Adaptive mean/std accumulate in fp64. At most 65535
+ * candidate tiles with COARSE_MEAN (VSA_ERR_UNSUPPORTED beyond). */
 vsa_status vsa_coarse_select(const vsa_layout* layout, const vsa_params* params,
                              int32_t B, int32_t H,
                              const void* q, const void* k, const void* v,
@@ -244,15 +253,17 @@ vsa_status vsa_coarse_select(const vsa_layout* layout, const vsa_params* params,
  * cannot afford the synchronisation and latency of cudaMalloc inside a step.
  *
  * Same arguments, outputs and results as vsa_coarse_select, minus workspace.
- * The scratch (pooled means, score matrix, adaptive sums) is a fixed 32 MiB
- * buffer inside the library's device image, held by every GPU that loads the
- * library until the process exits. Shapes whose scratch exceeds 32 MiB
- * (roughly: B * H * n_tiles * (1536 + 4 * round_up(n_video_tiles, 64)) bytes;
- * the 17k-token, 24-head workload fits, the 1344x768 shapes do not) are
- * refused with VSA_ERR_UNSUPPORTED and a message in vsa_last_error_detail.
- * The first call on a device looks up the buffer's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. Every call on a device shares the one buffer and leaves its
+ * The scratch (status words, pooled means, split chunks, marks; the score
+ * matrix with COARSE_REWEIGHT) is a fixed 32 MiB buffer inside the library's
+ * device image, held by every GPU that loads the library until the process
+ * exits. Shapes whose scratch exceeds 32 MiB (vsa_coarse_select_workspace_size
+ * of the same shape; the 17k-token, 24-head workload fits, the 1344x768
+ * shapes do not) are refused with VSA_ERR_UNSUPPORTED and a message in
+ * vsa_last_error_detail. The first call on a device looks up the buffer's
+ * device address (once per device, with that device current); make that
+ * first call before any stream capture, and do not call it after a
+ * cudaDeviceReset of that device (the cached address belongs to the old
+ * context). Every call on a device shares the one buffer and leaves its
  * contents behind; each call writes every scratch byte it later reads, so
  * nothing needs clearing, but calls that overlap on the GPU (different
  * streams, or concurrent host threads) race on the buffer. Allocates no
@@ -263,6 +274,25 @@ vsa_status vsa_coarse_select_noalloc(const vsa_layout* layout, const vsa_params*
                                      int64_t stride_b, int64_t stride_s, int64_t stride_h,
                                      int32_t* idx, int32_t* cnt, float* o_coarse,
                                      cudaStream_t stream);
+
+/* Zeroes the selection workspace's header, including the count of failed
+ * calls that vsa_coarse_select_failed_calls reports. Call once after
+ * allocating a workspace. No counterpart on the pages. */
+vsa_status vsa_coarse_select_workspace_init(void* workspace, cudaStream_t stream);
+
+/* Synchronises `stream` and reads the status word the most recent
+ * vsa_coarse_select on `workspace` left: VSA_OK or VSA_ERR_TIMEOUT (a bounded
+ * wait ran out; the lists and o_coarse are incomplete). No counterpart on
+ * the pages. */
+vsa_status vsa_coarse_select_status(const void* workspace, cudaStream_t stream);
+
+/* Synchronises `stream` and reads how many vsa_coarse_select calls on
+ * `workspace` recorded an error since vsa_coarse_select_workspace_init. */
+vsa_status vsa_coarse_select_failed_calls(const void* workspace, cudaStream_t stream, uint32_t* count);
+
+/* vsa_coarse_select_status for the built-in buffer of
+ * vsa_coarse_select_noalloc on the current device. */
+vsa_status vsa_coarse_select_noalloc_status(cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* extra_tokens                                                              */
@@ -436,6 +466,13 @@ vsa_status vsa_sparse_attn_status(const void* workspace, cudaStream_t stream);
  * written. Nothing faults, traps or hangs, and the CUDA context stays usable.
  * timeout_ns = 0 disarms it. Always returns VSA_OK. */
 vsa_status vsa_debug_inject_wait_timeout(uint64_t timeout_ns);
+
+/* vsa_debug_inject_select_wait_timeout: the same hook for the tensor-core
+ * kernels of vsa_coarse_select (COARSE_MEAN): while timeout_ns > 0 their
+ * MMA-issue warp first waits on a barrier nothing arrives on, bounded by
+ * timeout_ns, and vsa_coarse_select_status reports VSA_ERR_TIMEOUT.
+ * timeout_ns = 0 disarms it. Always returns VSA_OK. */
+vsa_status vsa_debug_inject_select_wait_timeout(uint64_t timeout_ns);
 
 const char* vsa_status_string(vsa_status status);
 

@@ -86,10 +86,14 @@ def test_sink_off_candidates_are_all_tiles():
         assert lay.kmax(vsa.make_params(keep=keep, sink=vsa.SINK_OFF)) == \
             O.topk_count(keep, O.candidate_tiles(ref, O.SINK_OFF)[1])
     assert lay.kmax(vsa.make_params(mode=vsa.SELECT_ADAPTIVE, sink=vsa.SINK_OFF)) == nt
-    # Spark-Reweight adds its anchor, summaries and biases to the selection workspace
+    # both workspaces: a 256-byte header, then the pooled means [3, B, H, n_tiles, 128];
+    # Spark-Reweight adds its score matrix and summaries, the mean branch its
+    # split Kbar / Vbar chunks (32 KB per 64 candidates and head) and marks
+    nv, pooled = lay.info.n_video_tiles, 256 + 3 * 2 * nt * 128 * 4
     rw = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5, coarse=vsa.COARSE_REWEIGHT))
     on = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5))
-    assert rw >= on + 2 * 2 * lay.info.n_video_tiles * 128 * 4
+    assert rw >= pooled + 2 * nt * 64 * 4 + 2 * 2 * nv * 128 * 4
+    assert on >= pooled + 2 * 2 * ((nv + 63) // 64) * 32768 + 2 * nt * 2 * ((nv + 63) // 64) * 4
     # the score matrix spans every tile: the selection workspace grows accordingly
     on = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5))
     off = lay.coarse_select_workspace_size(1, 2, vsa.make_params(keep=0.5, sink=vsa.SINK_OFF))

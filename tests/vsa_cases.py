@@ -66,6 +66,7 @@ def gpu_forward(wl, bits, prm: dict, out_dtype="f32", layout=None):
     fwd = vsa.Forward(lay, p, wl.B, wl.H, device=dev,
                       out_dtype=torch.float32 if out_dtype == "f32" else torch.bfloat16)
     out = fwd(tq, tk, tv, tg)
+    assert vsa.coarse_select_status(fwd.ws_select) == vsa.OK
     st = vsa.sparse_attn_status(fwd.ws_attn)
     torch.cuda.synchronize()
     res = dict(status=st, idx=fwd.idx.cpu().numpy(), cnt=fwd.cnt.cpu().numpy(),
