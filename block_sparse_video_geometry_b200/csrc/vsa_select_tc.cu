@@ -79,8 +79,10 @@ constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kSBufs = 4;                // score buffers in TMEM
 constexpr int kBins = 256;
-constexpr int kHistWords = kBins / 2 + 4;   // two u16 counters per word; 528-byte rows (16-byte aligned)
-constexpr int kCap = 64;                 // boundary-bin members kept per row
+constexpr int kHistPairs = kBins / 2;    // histogram words per row, two 16-bit counters each
+constexpr int kCap = 64;                 // boundary-bin members ranked directly per row
+constexpr int kHalfCap = kCap / 2;       // of which each of the row's two threads keeps up to 32
+constexpr int kQStride = 528;            // staged Qbar rows: 512 bytes + 16 (conflict-free column reads)
 constexpr int kRowWarps = 8;             // two threads per query tile
 constexpr int kThreads = 64 + 32 * kRowWarps;
 constexpr uint32_t kTmemCols = 512;
@@ -127,20 +129,25 @@ struct SelArgs {
 
 struct SelSmem {
   uint8_t k[kKStages][kChunkBytes];
-  uint8_t v[kVStages][kChunkBytes];      // collect pass: boundary members, entry e of row r at e * 128 + r
-  uint32_t hist[kRows * kHistWords];
+  uint8_t v[kVStages][kChunkBytes];
+  // One region, three uses in turn: the staged Qbar rows of the block (start),
+  // the row histograms [bin pair][row] (softmax and radix passes: lane r always
+  // hits bank r), the boundary members [slot][row] (collect pass).
+  union {
+    uint8_t q[kRows * kQStride];
+    uint32_t hist[kHistPairs * kRows];
+    float2 member[kCap * kRows];
+  } u;
   float xmx[2][kRows], xmn[2][kRows], xl[2][kRows];   // the two threads of a row exchange their partial results
-  int xarg[2][kRows];
-  int n_got[kRows];                      // boundary members collected per row
+  int xarg[2][kRows], xcnt[2][kRows];
   uint64_t k_full[kKStages], k_free[kKStages], v_full[kVStages], v_free[kVStages];
   uint64_t s_full[kSBufs], s_free[kSBufs], p_full[kSBufs], pv_done[kSBufs];
-  uint64_t o_full, q_ready, decide, drain, never;
+  uint64_t o_full, q_full, q_ready, decide, drain, never;
   uint32_t tmem_base;
   int abort;
   int more;                              // top-k: the fallback passes run
   double red[2][kRowWarps];
 };
-static_assert(kVStages * kChunkBytes >= kRows * kCap * 8, "boundary members must fit the V stages");
 
 __device__ __forceinline__ void record_error(int* err, int status) {
   if (atomicExch(err, status) == 0) atomicAdd(err + 1, 1);
@@ -195,9 +202,12 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
 // Row histograms: two 16-bit counters per word (bin 2i in the low half), so
 // that the two threads of a row add with shared-memory atomics (no return
 // value: nothing waits on them); counts stay below 65536.
-__device__ __forceinline__ void hist_add(uint32_t* h, uint32_t bin) { atomicAdd(h + (bin >> 1), 1u << ((bin & 1u) << 4)); }
+// h points at the row's first word; its words are kRows apart.
+__device__ __forceinline__ void hist_add(uint32_t* h, uint32_t bin) {
+  atomicAdd(h + (bin >> 1) * kRows, 1u << ((bin & 1u) << 4));
+}
 __device__ __forceinline__ int hist_count(const uint32_t* h, int bin) {
-  return static_cast<int>((h[bin >> 1] >> ((bin & 1) << 4)) & 0xFFFFu);
+  return static_cast<int>((h[(bin >> 1) * kRows] >> ((bin & 1) << 4)) & 0xFFFFu);
 }
 
 __device__ __forceinline__ void tmem_st32x16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -225,6 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t bh = static_cast<size_t>(blockIdx.z) * a.H + blockIdx.y;
   const int n_chunks = a.n_chunks;
+  // The CTAs of a head start their passes at different chunks (the fallback
+  // passes, which count equal keys in candidate order, do not rotate).
+  const int rot = static_cast<int>((static_cast<long long>(blockIdx.x) * n_chunks) / gridDim.x);
+  auto chunk_at = [&](int kind, int i) { return kind >= kPassRadix ? i : (i + rot) % n_chunks; };
   constexpr int kBasePasses = kMode == kModeTopk ? 3 : 1;
   constexpr int kSoftPass = kMode == kModeTopk ? 1 : (kMode == kModeThresh ? 0 : -1);
 
@@ -244,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
       mbar_init(smem_u32(&sm.pv_done[b]), 1);
     }
     mbar_init(smem_u32(&sm.o_full), 1);
+    mbar_init(smem_u32(&sm.q_full), 1);
     mbar_init(smem_u32(&sm.q_ready), kRowWarps);
     mbar_init(smem_u32(&sm.decide), 1);
     mbar_init(smem_u32(&sm.drain), 1);
@@ -252,7 +267,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
     sm.more = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < kRows; i += kThreads) sm.n_got[i] = 0;
   if (warp == 1) {
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
@@ -264,6 +278,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
 
   if (warp == 0) {
     // ----------------------------------------------------------- copies
+    // Qbar rows of the block (512 bytes each) at a padded stride
+    const int n_rows = min(kRows, a.n_tiles - static_cast<int>(blockIdx.x) * kRows);
+    if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sm.q_full), static_cast<uint32_t>(n_rows) * 512u);
+    __syncwarp();
+    for (int i = lane; i < n_rows; i += 32)
+      bulk_load(smem_u32(sm.u.q + i * kQStride), a.qbar + (bh * a.n_tiles + blockIdx.x * kRows + i) * kHeadDim, 512,
+                smem_u32(&sm.q_full));
+    __syncwarp();
     if (lane == 0) {
       const uint8_t* kb = a.ksplit + bh * n_chunks * kChunkBytes;
       const uint8_t* vb = a.vsplit + bh * n_chunks * kChunkBytes;
@@ -271,8 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
       bool ok = true;
       int n_passes = kBasePasses;
       for (int p = 0; ok && p < n_passes; ++p) {
-        const bool soft = pass_kind<kMode>(p) == kPassSoftmax;
-        for (int c = 0; c < n_chunks; ++c) {
+        const int kind = pass_kind<kMode>(p);
+        const bool soft = kind == kPassSoftmax;
+        for (int i = 0; i < n_chunks; ++i) {
+          const int c = chunk_at(kind, i);
           const uint32_t st = gk % kKStages;
           if (gk >= kKStages &&
               !(ok = mbar_wait(smem_u32(&sm.k_free[st]), ((gk / kKStages) - 1) & 1, &sm.abort, kTimeoutNs)))
@@ -299,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
       }
       if (!ok) {
         raise_abort(sm, a.err);
+        mbar_wait(smem_u32(&sm.q_full), 0, nullptr, kDrainNs);
         for (uint32_t i = (gk > kKStages ? gk - kKStages : 0u); i < gk; ++i)
           mbar_wait(smem_u32(&sm.k_full[i % kKStages]), (i / kKStages) & 1, nullptr, kDrainNs);
         for (uint32_t i = (gv > kVStages ? gv - kVStages : 0u); i < gv; ++i)
@@ -403,7 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
         if (progress) {
           spins = 0;
           t0 = 0;
-        } else if ((++spins & 255u) == 0) {
+        } else if (++spins > 4) {
+          __nanosleep(32);   // nothing ready: leave the issue slots to the row warps sharing this sub-partition
+        }
+        if (!progress && (spins & 255u) == 0) {
           if (aborted(sm)) {
             ok = false;
           } else {
@@ -431,19 +459,23 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const int n_words = 2 * n_chunks;
     uint32_t* bits_row = a.bits + row * n_words;
-    uint32_t* hist = sm.hist + r * kHistWords;
-    float2* member = reinterpret_cast<float2*>(sm.v[0]);   // collect pass: (score, ordinal) at e * 128 + r
+    uint32_t* hist = sm.u.hist + r;
+    float2* member = sm.u.member;   // collect pass: (score, ordinal) of slot e of row r at e * 128 + r
+    const int et = threadIdx.x - 64;   // 0 .. 255 over the row warps
 
+    bool ok = true;
     // Qbar dims 64 half .. + 63 of this query tile, split hi / lo, as the A
     // operand (rows past the end are zero: their scores are 0 and nothing of
     // theirs is written)
     {
-      const float2* src = reinterpret_cast<const float2*>(a.qbar + row * kHeadDim) + 32 * half;
+      ok = warp_wait(sm, sm.q_full, 0, lane, a.err);
+      const float4* src = reinterpret_cast<const float4*>(sm.u.q + r * kQStride + 256 * half);
       uint32_t wh[32], wl[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float2 x = row_ok ? src[i] : make_float2(0.f, 0.f);
-        split_pair(x.x, x.y, wh[i], wl[i]);
+      for (int i = 0; i < 16; ++i) {
+        const float4 x = row_ok ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        split_pair(x.x, x.y, wh[2 * i], wl[2 * i]);
+        split_pair(x.z, x.w, wh[2 * i + 1], wl[2 * i + 1]);
       }
       tmem_st32x32(lane_addr + kColQ + 32 * half, wh);
       tmem_st32x32(lane_addr + kColQ + 64 + 32 * half, wl);
@@ -453,13 +485,12 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
       if (lane == 0) mbar_arrive(smem_u32(&sm.q_ready));
     }
 
-    bool ok = true;
     uint32_t gs = 0;
     float mx = -INFINITY, mn = INFINITY, l0 = 0.f, l1 = 0.f;
     int arg = 0;
     double s1 = 0.0, s2 = 0.0, thr = 0.0;
     float inv_w = 0.f, off = 0.f;
-    int bstar = 0, krem = 0, nmem = 0, eq_seen = 0;
+    int bstar = 0, krem = 0, nmem = 0, eq_seen = 0, n_loc = 0;
     bool fb = false;
     uint32_t prefix = 0, pmask = 0;
 
@@ -484,13 +515,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
       // the fallback passes are rare: the first thread of a row takes all 64 candidates of each chunk
       const bool solo = kind == kPassRadix || kind == kPassEmit;
       if ((kMode == kModeTopk && kind == kPassSoftmax) || kind == kPassRadix) {
-        if (half == 0) {
-          uint4* h4 = reinterpret_cast<uint4*>(hist);
-          for (int i = 0; i < kHistWords / 4; ++i) h4[i] = make_uint4(0u, 0u, 0u, 0u);
-        }
+        // every thread is done with the region (the previous pass's counts and scans, the staged Qbar)
+        rows_sync();
+        uint4* h4 = reinterpret_cast<uint4*>(sm.u.hist);
+        for (int i = et; i < kHistPairs * kRows / 4; i += 32 * kRowWarps) h4[i] = make_uint4(0u, 0u, 0u, 0u);
         rows_sync();
       }
-      for (int c = 0; c < n_chunks; ++c, ++gs) {
+      for (int ci = 0; ci < n_chunks; ++ci, ++gs) {
+        const int c = chunk_at(kind, ci);
         const uint32_t b = gs % kSBufs;
         if (ok) ok = warp_wait(sm, sm.s_full[b], (gs / kSBufs) & 1, lane, a.err);
         if (!ok) continue;
@@ -553,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
           for (int j = 0; j < 32; ++j) {
             const float s = x[j] * a.scale;
             if (j < n_valid) {
-              if (s > mx) {
+              if (s > mx || (s == mx && o0 + j < arg)) {   // the first maximal candidate in any visiting order
                 mx = s;
                 arg = o0 + j;
               }
@@ -602,8 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
               if (bn > bstar) {
                 word |= 1u << j;
               } else if (bn == bstar && !fb) {
-                const int slot = atomicAdd(&sm.n_got[r], 1);
-                if (slot < kCap) member[slot * kRows + r] = make_float2(s, __int_as_float(o0 + j));
+                if (n_loc < kHalfCap) member[(kHalfCap * half + n_loc) * kRows + r] = make_float2(s, __int_as_float(o0 + j));
+                ++n_loc;
               }
             }
           }
@@ -697,17 +729,22 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
           }
           fb = nmem > kCap;
         }
+        if (kMode == kModeTopk) rows_sync();   // every row's scan is done: the members overlay the histograms
       } else if (kind == kPassCollect) {
+        sm.xcnt[half][r] = n_loc;
         rows_sync();                              // members and marks of both threads of every row are in
+        const int n0 = sm.xcnt[0][r], n1 = sm.xcnt[1][r];
+        if (n0 > kHalfCap || n1 > kHalfCap) fb = true;   // a thread's share overflowed: the exact passes rank the row
         // rank the boundary members (score descending, lower ordinal first); take krem
         if (ok && row_ok && !fb && half == 0) {
-          const int n_got = min(sm.n_got[r], kCap);
+          const int n_got = n0 + n1;
+          auto slot = [&](int e) { return e < n0 ? e : kHalfCap + (e - n0); };
           for (int e = 0; e < n_got; ++e) {
-            const float2 me = member[e * kRows + r];
+            const float2 me = member[slot(e) * kRows + r];
             const int oe = __float_as_int(me.y);
             int rank = 0;
             for (int f = 0; f < n_got; ++f) {
-              const float2 mf = member[f * kRows + r];
+              const float2 mf = member[slot(f) * kRows + r];
               const int of = __float_as_int(mf.y);
               rank += (mf.x > me.x || (mf.x == me.x && of < oe)) ? 1 : 0;
             }
