@@ -279,12 +279,28 @@ __global__ void __launch_bounds__(kXThreads, 1) extra_select_kernel(const __grid
       const int tile = a.cand0 + t;
       const unsigned long long vm = a.L.valid[tile];
       const int32_t* perm_tile = a.L.perm + tile * kTile;
+      // slots that may enter the top-E: a branch-free mask first (after the
+      // first tiles almost none qualify, and a branch per slot costs far more
+      // than the compare), then one offer per set bit in slot order
+      const float lim = count < a.E ? -INFINITY : wv;
+      uint32_t m0 = 0, m1 = 0;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        if (((vm >> i) & 1ull) && (count < a.E || x0[i] >= wv))
-          x_offer(sm, perm_tile, r, a.E, x0[i], i, count, worst, wv, wt);
-        if (((vm >> (32 + i)) & 1ull) && (count < a.E || x1[i] >= wv))
-          x_offer(sm, perm_tile, r, a.E, x1[i], 32 + i, count, worst, wv, wt);
+        m0 |= (x0[i] >= lim ? 1u : 0u) << i;
+        m1 |= (x1[i] >= lim ? 1u : 0u) << i;
+      }
+      unsigned long long cand = (static_cast<unsigned long long>(m1) << 32 | m0) & vm;
+      while (cand) {
+        const int i = __ffsll(static_cast<long long>(cand)) - 1;
+        cand &= cand - 1;
+        // the scores stay in registers: pick slot i's without dynamic indexing
+        float xi = 0.f;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          xi = (i == u) ? x0[u] : xi;
+          xi = (i == 32 + u) ? x1[u] : xi;
+        }
+        if (count < a.E || xi >= wv) x_offer(sm, perm_tile, r, a.E, xi, i, count, worst, wv, wt);
       }
     }
     if (ok && row_ok) {

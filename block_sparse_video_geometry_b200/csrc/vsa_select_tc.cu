@@ -79,7 +79,8 @@ constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kSBufs = 4;                // score buffers in TMEM
 constexpr int kBins = 256;
-constexpr int kHistPairs = kBins / 2;    // histogram words per row, two 16-bit counters each
+constexpr int kHistPairs = kBins / 2 + 1;   // histogram words per row (two 16-bit counters each) + one for
+                                            // the dummy bin 256 that scores outside the candidates go to
 constexpr int kCap = 64;                 // boundary-bin members ranked directly per row
 constexpr int kHalfCap = kCap / 2;       // of which each of the row's two threads keeps up to 32
 constexpr int kQStride = 528;            // staged Qbar rows: 512 bytes + 16 (conflict-free column reads)
@@ -486,9 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
     }
 
     uint32_t gs = 0;
-    float mx = -INFINITY, mn = INFINITY, l0 = 0.f, l1 = 0.f;
+    float mx = -INFINITY, mn = INFINITY, lq[4] = {0.f, 0.f, 0.f, 0.f};
     int arg = 0;
-    double s1 = 0.0, s2 = 0.0, thr = 0.0;
+    double s1 = 0.0, s2 = 0.0, s1b = 0.0, s2b = 0.0, thr = 0.0;
     float inv_w = 0.f, off = 0.f;
     int bstar = 0, krem = 0, nmem = 0, eq_seen = 0, n_loc = 0;
     bool fb = false;
@@ -580,23 +581,46 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
         const int o0 = c * kChunk + 32 * half;   // candidate of x[0]
         const int n_valid = a.n_cand - o0;        // x[j] is a candidate for j < n_valid
         uint32_t word = 0;                        // marks of candidates o0 .. o0 + 31
+        // The per-score work avoids long serial chains (tree reductions,
+        // bit masks, several accumulators): two row warps per scheduler hide
+        // little latency.
         if (kind == kPassRange) {
+          float hv[32], lv[32];
+          int hi_[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float s = x[j] * a.scale;
-            if (j < n_valid) {
-              if (s > mx || (s == mx && o0 + j < arg)) {   // the first maximal candidate in any visiting order
-                mx = s;
-                arg = o0 + j;
-              }
-              mn = fminf(mn, s);
-              if (kMode == kModeStats) {
-                const double sd = static_cast<double>(s);
-                s1 += sd;
+            const bool v = j < n_valid;
+            hv[j] = v ? s : -INFINITY;
+            lv[j] = v ? s : INFINITY;
+            hi_[j] = j;
+            if (kMode == kModeStats) {
+              const double sd = v ? static_cast<double>(s) : 0.0;
+              if (j & 1) {
                 s2 = fma(sd, sd, s2);
+                s1 += sd;
+              } else {
+                s2b = fma(sd, sd, s2b);
+                s1b += sd;
               }
             }
           }
+          // maximum with the lowest index among equal maxima, and minimum, as trees
+#pragma unroll
+          for (int w = 16; w >= 1; w >>= 1) {
+#pragma unroll
+            for (int j = 0; j < w; ++j) {
+              const bool tb = hv[j + w] > hv[j];      // the upper half wins only when strictly larger
+              hv[j] = tb ? hv[j + w] : hv[j];
+              hi_[j] = tb ? hi_[j + w] : hi_[j];
+              lv[j] = fminf(lv[j], lv[j + w]);
+            }
+          }
+          // the first maximal candidate in any visiting order
+          const bool better = hv[0] > mx || (hv[0] == mx && o0 + hi_[0] < arg);
+          mx = better ? hv[0] : mx;
+          arg = better ? o0 + hi_[0] : arg;
+          mn = fminf(mn, lv[0]);
         } else if (kind == kPassSoftmax) {
           uint32_t wh[16], wl[16];
 #pragma unroll
@@ -605,12 +629,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
             const bool va = 2 * i < n_valid, vb = 2 * i + 1 < n_valid;
             const float pa = va ? ex2_approx((sa - mx) * kLog2e) : 0.f;
             const float pb = vb ? ex2_approx((sb - mx) * kLog2e) : 0.f;
-            if (i & 1) l1 += pa + pb;
-            else l0 += pa + pb;
+            lq[i & 3] += pa + pb;
             split_pair(pa, pb, wh[i], wl[i]);
             if (kMode == kModeTopk) {
-              if (va) hist_add(hist, score_bin(sa, inv_w, off));
-              if (vb) hist_add(hist, score_bin(sb, inv_w, off));
+              hist_add(hist, va ? score_bin(sa, inv_w, off) : kBins);
+              hist_add(hist, vb ? score_bin(sb, inv_w, off) : kBins);
             } else {
               word |= (va && static_cast<double>(sa) >= thr ? 1u : 0u) << (2 * i);
               word |= (vb && static_cast<double>(sb) >= thr ? 1u : 0u) << (2 * i + 1);
@@ -626,17 +649,26 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
           if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[b]));
           if (kMode == kModeThresh && row_ok) bits_row[2 * c + half] = word;
         } else {   // collect
+          uint32_t memb = 0;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float s = x[j] * a.scale;
-            if (j < n_valid) {
-              const int bn = score_bin(s, inv_w, off);
-              if (bn > bstar) {
-                word |= 1u << j;
-              } else if (bn == bstar && !fb) {
-                if (n_loc < kHalfCap) member[(kHalfCap * half + n_loc) * kRows + r] = make_float2(s, __int_as_float(o0 + j));
-                ++n_loc;
-              }
+            const bool v = j < n_valid;
+            const int bn = score_bin(s, inv_w, off);
+            word |= (v && bn > bstar ? 1u : 0u) << j;
+            memb |= (v && bn == bstar ? 1u : 0u) << j;
+          }
+          // boundary members (a handful per row over the whole pass)
+          if (!fb) {
+            while (memb) {
+              const int j = __ffs(memb) - 1;
+              memb &= memb - 1;
+              float xj = 0.f;
+#pragma unroll
+              for (int u = 0; u < 32; ++u) xj = (u == j) ? x[u] : xj;
+              if (n_loc < kHalfCap)
+                member[(kHalfCap * half + n_loc) * kRows + r] = make_float2(xj * a.scale, __int_as_float(o0 + j));
+              ++n_loc;
             }
           }
           if (row_ok) bits_row[2 * c + half] = word;
@@ -672,6 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
             a.rowmax[row] = mx;
             a.rowarg[row] = arg;
           }
+          s1 += s1b;
+          s2 += s2b;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
             s1 += __shfl_xor_sync(0xffffffffu, s1, o);
@@ -693,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_tc_kernel(const __grid_con
           }
         }
       } else if (kind == kPassSoftmax) {
-        sm.xl[half][r] = l0 + l1;
+        sm.xl[half][r] = (lq[0] + lq[1]) + (lq[2] + lq[3]);
         rows_sync();                              // also: every histogram count of the pass has landed
         const float l = sm.xl[0][r] + sm.xl[1][r];
         if (ok) ok = warp_wait(sm, sm.o_full, 0, lane, a.err);
