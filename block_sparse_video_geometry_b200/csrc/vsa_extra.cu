@@ -16,15 +16,20 @@
 //    attention uses, so that a key tile arrives with one bulk copy.
 //  * pool_q_kernel: Qbar, the fp32 mean of the valid tokens of every tile.
 //  * extra_select_kernel: one CTA per (batch, head, 128 query tiles). Scoring
-//    128 query tiles against one 64-token key tile is one M = 128, N = 64
-//    tcgen05 product per split term: Qbar = hi + mid + lo in bf16 (24 mantissa
-//    bits, held in TMEM as the A operand), K exact in bf16, fp32 accumulation,
-//    so the scores carry fp32 rounding only (3 x 8 MMAs per key tile). The key
-//    tiles stream through shared memory in candidate order (four stages); each
-//    of 128 threads owns one query tile (TMEM lane r = query tile r of the
-//    block), skips the tiles its ascending selection list holds (a pointer
-//    walks the list), and keeps a running top-E in shared memory (an unordered
-//    array plus the position of its weakest entry, which a new token must beat).
+//    128 query tiles against a pair of 64-token key tiles is one M = 128,
+//    N = 128 tcgen05 product per split term: Qbar = hi + lo in bf16 (hi =
+//    bf16(x), lo = bf16(x - hi): x to a relative 2^-17, held in TMEM as the A
+//    operand), K exact in bf16, fp32 accumulation, so a score's error stays
+//    below 2^-17 of sum_d |q_d k_d|, the size of an fp32 FMA chain's rounding
+//    over 128 dims (2 x 8 MMAs per pair; a pair halves the MMA count of one
+//    tile at a time, whose N = 64 products ran at a third of the tensor rate).
+//    The pairs stream through shared memory (up to four stages; the CTAs of a
+//    head start at different tiles). Two sets of 128 threads read the scores:
+//    thread r of set s owns query tile r of the block (TMEM lane r) for tile
+//    s of every pair, skips the tiles the query tile selected (a bitmap in
+//    shared memory), and keeps a running top-E in shared memory (an unordered
+//    array plus the position of its weakest entry, which a new token must
+//    beat); at the end set 0 offers set 1's entries to its own list.
 
 #include <cuda_runtime.h>
 
@@ -40,26 +45,47 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kXThreads = 192;           // 6 warps: 0 copies, 1 MMAs, 2-5 one query tile per thread
+constexpr int kXThreads = 320;           // 10 warps: 0 copies, 1 MMAs, 2-9 two sets of one query tile per thread
 constexpr int kXRows = 128;
-constexpr int kXStages = 4;
-constexpr int kXMaxE = VSA_MAX_EXTRA_TOKENS;
+constexpr int kXStagesMax = 4;           // stages of a key tile pair (32 KB each)
 constexpr uint32_t kXTmemCols = 512;
-constexpr uint32_t kXColA = 0;           // Qbar split terms: 64 columns of bf16 pairs each
-constexpr uint32_t kXColD = 192;         // two score buffers of 64 fp32 columns
-constexpr uint32_t kXIdesc = idesc_bf16_f32(128, 64, 0, 0);
+constexpr uint32_t kXColA = 0;           // Qbar split terms hi, lo: 64 columns of bf16 pairs each
+constexpr uint32_t kXColD = 128;         // two score buffers of 128 fp32 columns (a key tile pair)
+constexpr uint32_t kXIdesc = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint64_t kXTimeoutNs = 4000000000ull;
 constexpr uint64_t kXDrainNs = 200000000ull;
 constexpr size_t kXHeader = 256;         // status word
+constexpr uint32_t kXSmemMax = 227u * 1024u;
 
-struct XSmem {
-  uint8_t k[kXStages][16384];
-  float val[kXMaxE * kXRows];            // top-E scores: entry e of row r at e * 128 + r
-  int32_t tok[kXMaxE * kXRows];
-  uint64_t k_full[kXStages], k_free[kXStages], d_full[2], d_free[2], a_ready, drain;
+// Fixed part of the shared memory; the stages, the two sets' top-E lists and
+// the selected-tile bitmap follow at offsets XSmemLayout gives.
+struct XHead {
+  uint64_t k_full[kXStagesMax], k_free[kXStagesMax], d_full[2], d_free[2], a_ready, drain;
   uint32_t tmem_base;
   int abort;
+  int cnt1[kXRows];                      // set 1's list length per row, for the merge
 };
+static_assert(sizeof(XHead) <= 1024, "stages start at byte 1024");
+
+// words of the per-row bitmap of selected candidate tiles
+__host__ __device__ inline int x_sel_words(int n_cand) { return (n_cand + 31) / 32; }
+// E rounded up to eight: the lists are read eight entries at a time
+__host__ __device__ inline int x_pad_e(int E) { return (E + 7) & ~7; }
+
+struct XSmemLayout {
+  int stages;
+  uint32_t val;                          // set s: scores at val + s * 8 ep * 128, tokens 4 ep * 128 bytes later
+  uint32_t sel;                          // bitmap: bit c of word w of row r in word w * 128 + r
+  uint32_t total;
+};
+inline XSmemLayout x_smem_layout(int stages, int E, int n_cand) {
+  XSmemLayout l;
+  l.stages = stages;
+  l.val = 1024u + static_cast<uint32_t>(stages) * 32768u;
+  l.sel = l.val + 2u * 8u * static_cast<uint32_t>(x_pad_e(E)) * kXRows;
+  l.total = l.sel + 4u * static_cast<uint32_t>(x_sel_words(n_cand)) * kXRows;
+  return l;
+}
 
 struct XArgs {
   DevLayout L;
@@ -68,17 +94,21 @@ struct XArgs {
   const int32_t* idx;
   const int32_t* cnt;
   int32_t kmax, H, c0, cand0, n_cand, E;
+  int32_t stages;
+  uint32_t off_val, off_sel;             // XSmemLayout offsets
   int32_t* out_idx;                      // [B, H, n_tiles, E]
   int32_t* out_cnt;                      // [B, H, n_tiles]
   int* err;
 };
 
-__device__ __forceinline__ void x_abort(XSmem& sm, int* err) {
+template <class XS>
+__device__ __forceinline__ void x_abort(XS& sm, int* err) {
   atomicExch(err, VSA_ERR_TIMEOUT);
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
-__device__ __forceinline__ bool x_warp_wait(XSmem& sm, uint64_t& bar, uint32_t parity, int lane, int* err) {
+template <class XS>
+__device__ __forceinline__ bool x_warp_wait(XS& sm, uint64_t& bar, uint32_t parity, int lane, int* err) {
   int ok = 1;
   if (lane == 0) {
     ok = mbar_wait(smem_u32(&bar), parity, &sm.abort, kXTimeoutNs) ? 1 : 0;
@@ -96,39 +126,147 @@ __device__ __forceinline__ float bf16_round(float x) {
   return __uint_as_float(r);
 }
 
-// The weakest entry of a row's full top-E: lowest score, and among equal
-// lowest scores the highest token index.
-__device__ __noinline__ void x_find_worst(const XSmem& sm, int r, int E, int& worst, float& wv, int& wt) {
-  worst = 0;
-  wv = sm.val[r];
-  wt = sm.tok[r];
-  for (int e = 1; e < E; ++e) {
-    const float v = sm.val[e * kXRows + r];
-    const int t = sm.tok[e * kXRows + r];
-    if (v < wv || (v == wv && t > wt)) {
-      worst = e;
-      wv = v;
-      wt = t;
+// (v, t) ranks below (wv, wt): lower score, or equal score and higher token
+// index. Tokens are distinct, so this is a total order on a row's entries.
+__device__ __forceinline__ bool x_weaker(float v, int t, float wv, int wt) { return v < wv || (v == wv && t > wt); }
+
+// The weakest entry of a row's full top-E (entry e at val[e * 128], tok[e * 128]).
+// The entries are read eight at a time (independent loads; the arrays hold a
+// multiple of eight) and reduced as a tree, so a replacement costs a few load
+// latencies, not E of them.
+__device__ __forceinline__ void x_find_worst(const float* val, const int* tok, int E, int& worst, float& wv, int& wt) {
+  worst = -1;
+  wv = INFINITY;
+  wt = -1;
+  for (int e0 = 0; e0 < E; e0 += 8) {
+    float v[8];
+    int t[8], w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = e0 + j < E;
+      v[j] = in ? val[(e0 + j) * kXRows] : INFINITY;
+      t[j] = in ? tok[(e0 + j) * kXRows] : -1;
+      w[j] = e0 + j;
+    }
+#pragma unroll
+    for (int h = 4; h >= 1; h >>= 1)
+#pragma unroll
+      for (int j = 0; j < h; ++j)
+        if (x_weaker(v[j + h], t[j + h], v[j], t[j])) {
+          v[j] = v[j + h];
+          t[j] = t[j + h];
+          w[j] = w[j + h];
+        }
+    if (worst < 0 || x_weaker(v[0], t[0], wv, wt)) {
+      worst = w[0];
+      wv = v[0];
+      wt = t[0];
     }
   }
 }
 
-// Offers (score, slot of key tile) to row r's top-E (called for scores that
-// may enter: the list is not full, or the score is at least the weakest).
-__device__ __noinline__ void x_offer(XSmem& sm, const int32_t* perm_tile, int r, int E, float s, int slot,
-                                     int& count, int& worst, float& wv, int& wt) {
-  const int t = perm_tile[slot];
+// Score of slot i (0..63) of a key tile held in two register arrays, by a
+// select tree on the bits of i (depth six, no dynamic register indexing).
+__device__ __forceinline__ float x_pick(const float (&x0)[32], const float (&x1)[32], int i) {
+  float l[32];
+  const bool b5 = (i & 32) != 0;
+#pragma unroll
+  for (int u = 0; u < 32; ++u) l[u] = b5 ? x1[u] : x0[u];
+#pragma unroll
+  for (int h = 16; h >= 1; h >>= 1) {
+    const bool b = (i & h) != 0;
+#pragma unroll
+    for (int u = 0; u < h; ++u) l[u] = b ? l[u + h] : l[u];
+  }
+  return l[0];
+}
+
+// Token of slot `slot` of a tile from its origin (conditioning tile: first
+// token; video tile: the cube corner), without a memory access.
+__device__ __forceinline__ int x_token(const DevLayout& L, int4 org, int slot) {
+  if (org.w != VSA_SEG_VIDEO) return org.x + slot;
+  const int t = org.x + (slot >> 4), h = org.y + ((slot >> 2) & 3), w = org.z + (slot & 3);
+  return static_cast<int>(L.video_start + (static_cast<int64_t>(t) * L.grid_h + h) * L.grid_w + w);
+}
+
+// Bit i of the result: slot i's score (x0[i], then x1[i - 32]) is at least
+// lim. Built as an OR tree, so no 32-long dependency chain.
+__device__ __forceinline__ unsigned long long x_mask_ge(const float (&x0)[32], const float (&x1)[32], float lim) {
+  uint32_t mq[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    mq[i] = ((x0[4 * i] >= lim ? 1u : 0u) << (4 * i)) | ((x0[4 * i + 1] >= lim ? 1u : 0u) << (4 * i + 1)) |
+            ((x0[4 * i + 2] >= lim ? 1u : 0u) << (4 * i + 2)) | ((x0[4 * i + 3] >= lim ? 1u : 0u) << (4 * i + 3));
+    mq[8 + i] = ((x1[4 * i] >= lim ? 1u : 0u) << (4 * i)) | ((x1[4 * i + 1] >= lim ? 1u : 0u) << (4 * i + 1)) |
+                ((x1[4 * i + 2] >= lim ? 1u : 0u) << (4 * i + 2)) | ((x1[4 * i + 3] >= lim ? 1u : 0u) << (4 * i + 3));
+  }
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      mq[i] |= mq[i + w];
+      mq[8 + i] |= mq[8 + i + w];
+    }
+  return static_cast<unsigned long long>(mq[8]) << 32 | mq[0];
+}
+
+// Narrows a key tile's candidate slots when more than E of them qualify: a
+// slot with at least E candidates of the same tile above it cannot be in the
+// top-E after the tile, so any bound lo with at least E candidates at or
+// above it filters the rest. lo is found by bisection between the
+// candidates' minimum and maximum score (a filter only: ties and the exact
+// order are left to the offers).
+__device__ __forceinline__ unsigned long long x_narrow(const float (&x0)[32], const float (&x1)[32],
+                                                       unsigned long long cand, int E) {
+  float t[32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u)
+    t[u] = fminf(((cand >> u) & 1ull) ? x0[u] : INFINITY, ((cand >> (32 + u)) & 1ull) ? x1[u] : INFINITY);
+#pragma unroll
+  for (int h = 16; h >= 1; h >>= 1)
+#pragma unroll
+    for (int u = 0; u < h; ++u) t[u] = fminf(t[u], t[u + h]);
+  float lo = t[0];
+#pragma unroll
+  for (int u = 0; u < 32; ++u)
+    t[u] = fmaxf(((cand >> u) & 1ull) ? x0[u] : -INFINITY, ((cand >> (32 + u)) & 1ull) ? x1[u] : -INFINITY);
+#pragma unroll
+  for (int h = 16; h >= 1; h >>= 1)
+#pragma unroll
+    for (int u = 0; u < h; ++u) t[u] = fmaxf(t[u], t[u + h]);
+  float hi = t[0];
+  for (int it = 0; it < 10; ++it) {              // invariant: at least E candidates at or above lo
+    const float mid = 0.5f * (lo + hi);
+    if (__popcll(x_mask_ge(x0, x1, mid) & cand) >= E) lo = mid;
+    else hi = mid;
+  }
+  return x_mask_ge(x0, x1, lo) & cand;
+}
+
+// Offers (score, token) to a row's top-E (called for scores that may enter:
+// the list is not full, or the score is at least the weakest).
+__device__ __forceinline__ void x_offer(float* val, int* tok, int E, float s, int t, int& count, int& worst,
+                                        float& wv, int& wt) {
   if (count < E) {
-    sm.val[count * kXRows + r] = s;
-    sm.tok[count * kXRows + r] = t;
-    if (++count == E) x_find_worst(sm, r, E, worst, wv, wt);
+    val[count * kXRows] = s;
+    tok[count * kXRows] = t;
+    if (++count == E) x_find_worst(val, tok, E, worst, wv, wt);
     return;
   }
-  if (s > wv || (s == wv && t < wt)) {
-    sm.val[worst * kXRows + r] = s;
-    sm.tok[worst * kXRows + r] = t;
-    x_find_worst(sm, r, E, worst, wv, wt);
+  if (x_weaker(wv, wt, s, t)) {
+    val[worst * kXRows] = s;
+    tok[worst * kXRows] = t;
+    x_find_worst(val, tok, E, worst, wv, wt);
   }
+}
+
+__device__ __forceinline__ void x_rows_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Position t of a CTA's key tile stream -> candidate index (the CTAs of a head
+// start at different tiles, spreading their reads of the same tiles in time).
+__device__ __forceinline__ int x_rotate(int t, int rot, int n_cand) {
+  const int tt = t + rot;
+  return tt >= n_cand ? tt - n_cand : tt;
 }
 
 __global__ void __launch_bounds__(kXThreads, 1) extra_select_kernel(const __grid_constant__ XArgs a) {
@@ -137,21 +275,25 @@ __global__ void __launch_bounds__(kXThreads, 1) extra_select_kernel(const __grid
     if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
     return;
   }
-  XSmem& sm = *reinterpret_cast<XSmem*>(smem_raw);
+  XHead& sm = *reinterpret_cast<XHead*>(smem_raw);
+  uint8_t* const stage0 = smem_raw + 1024;
+  const int S = a.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t bh = static_cast<size_t>(blockIdx.z) * a.H + blockIdx.y;
   const int qt0 = a.c0 + blockIdx.x * kXRows;
   const int n_tiles = a.L.n_tiles;
+  const int n_pairs = (a.n_cand + 1) >> 1;
+  const int rot = static_cast<int>((static_cast<long long>(blockIdx.x) * a.n_cand) / gridDim.x);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kXStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&sm.k_full[s]), 1);
       mbar_init(smem_u32(&sm.k_free[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.d_full[i]), 1);
-      mbar_init(smem_u32(&sm.d_free[i]), 4);    // one arrival per row warp
+      mbar_init(smem_u32(&sm.d_free[i]), 8);    // one arrival per row warp
     }
-    mbar_init(smem_u32(&sm.a_ready), 4);
+    mbar_init(smem_u32(&sm.a_ready), 8);
     mbar_init(smem_u32(&sm.drain), 1);
     sm.abort = 0;
     fence_mbar_init();
@@ -166,45 +308,55 @@ __global__ void __launch_bounds__(kXThreads, 1) extra_select_kernel(const __grid
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == 0) {
-    // ---------------------------------------------------- key tile copies
+    // ------------------------------------------- key tile pair copies
+    // stage layout [d half][tile 2p, tile 2p + 1][64 slots][128 B]: each d
+    // half of the pair is one 128-row K-major operand of the MMA
     uint32_t issued = 0;
     bool ok = true;
-    for (int t = 0; t < a.n_cand; ++t) {
-      const int st = t % kXStages;
-      if (t >= kXStages && !(ok = x_warp_wait(sm, sm.k_free[st], ((t / kXStages) - 1) & 1, lane, a.err))) break;
+    for (int p = 0; p < n_pairs; ++p) {
+      const int st = p % S;
+      if (p >= S && !(ok = x_warp_wait(sm, sm.k_free[st], ((p / S) - 1) & 1, lane, a.err))) break;
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sm.k_full[st]);
-        mbar_arrive_expect_tx(bar, 16384);
-        bulk_load(smem_u32(sm.k[st]), a.ktm + (bh * n_tiles + a.cand0 + t) * 16384u, 16384, bar);
+        const uint32_t dst = smem_u32(stage0 + st * 32768);
+        const int nt = 2 * p + 1 < a.n_cand ? 2 : 1;
+        mbar_arrive_expect_tx(bar, 16384u * nt);
+        for (int j = 0; j < nt; ++j) {
+          const uint8_t* src = a.ktm + (bh * n_tiles + a.cand0 + x_rotate(2 * p + j, rot, a.n_cand)) * 16384u;
+          bulk_load(dst + 8192u * j, src, 8192, bar);
+          bulk_load(dst + 16384u + 8192u * j, src + 8192, 8192, bar);
+        }
       }
       __syncwarp();
       ++issued;
     }
     if (!ok && lane == 0) {
-      for (uint32_t i = (issued > kXStages ? issued - kXStages : 0u); i < issued; ++i)
-        mbar_wait(smem_u32(&sm.k_full[i % kXStages]), (i / kXStages) & 1, nullptr, kXDrainNs);
+      for (uint32_t i = (issued > static_cast<uint32_t>(S) ? issued - S : 0u); i < issued; ++i)
+        mbar_wait(smem_u32(&sm.k_full[i % S]), (i / S) & 1, nullptr, kXDrainNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMAs
-    // D(t) = sum over the three split terms of Qbar_term K(t)^T into score
-    // buffer t & 1, once the row warps have read D(t - 2) out of it.
+    // D(p) = sum over the two split terms of Qbar_term [K(2p); K(2p+1)]^T into
+    // score buffer p & 1, once the row warps have read D(p - 2) out of it.
+    // (A missing second tile of an odd count leaves columns 64..127 stale;
+    // nothing reads them.)
     if (lane == 0) {
       bool ok = mbar_wait(smem_u32(&sm.a_ready), 0, &sm.abort, kXTimeoutNs);
-      for (int t = 0; ok && t < a.n_cand; ++t) {
-        const int st = t % kXStages;
-        if (!(ok = mbar_wait(smem_u32(&sm.k_full[st]), (t / kXStages) & 1, &sm.abort, kXTimeoutNs))) break;
-        if (t >= 2 && !(ok = mbar_wait(smem_u32(&sm.d_free[t & 1]), ((t >> 1) - 1) & 1, &sm.abort, kXTimeoutNs)))
+      for (int p = 0; ok && p < n_pairs; ++p) {
+        const int st = p % S;
+        if (!(ok = mbar_wait(smem_u32(&sm.k_full[st]), (p / S) & 1, &sm.abort, kXTimeoutNs))) break;
+        if (p >= 2 && !(ok = mbar_wait(smem_u32(&sm.d_free[p & 1]), ((p >> 1) - 1) & 1, &sm.abort, kXTimeoutNs)))
           break;
         tc_fence_after();
-        const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
-        const uint32_t d = tmem + kXColD + 64u * (t & 1);
+        const uint64_t kd = smem_desc_sw128(smem_u32(stage0 + st * 32768), 16, 1024);
+        const uint32_t d = tmem + kXColD + 128u * (p & 1);
 #pragma unroll
-        for (int term = 0; term < 3; ++term)
+        for (int term = 0; term < 2; ++term)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(d, tmem + kXColA + 64u * term + kk * 8, kd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kXIdesc,
+            umma_ts(d, tmem + kXColA + 64u * term + kk * 8, kd + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2, kXIdesc,
                     (term | kk) ? 1u : 0u);
-        umma_commit(smem_u32(&sm.d_full[t & 1]));
+        umma_commit(smem_u32(&sm.d_full[p & 1]));
         umma_commit(smem_u32(&sm.k_free[st]));
       }
       if (!ok) x_abort(sm, a.err);
@@ -213,99 +365,120 @@ __global__ void __launch_bounds__(kXThreads, 1) extra_select_kernel(const __grid
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ one query tile per thread
+    // -------------------------------- one query tile per thread, two sets
+    // set 0 (warps 2-5) scores the first tile of every pair, set 1 (warps
+    // 6-9) the second; each keeps its own top-E, merged at the end
+    const int set = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int qt = qt0 + r;
     const bool row_ok = qt < n_tiles;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const size_t row = bh * n_tiles + (row_ok ? qt : 0);
-    // Qbar of this query tile, split into three bf16 terms, as the A operand
+    const int ep = x_pad_e(a.E);
+    float* const val = reinterpret_cast<float*>(smem_raw + a.off_val) + set * 2 * ep * kXRows + r;
+    int* const tok = reinterpret_cast<int*>(val + ep * kXRows);
+    uint32_t* const sel = reinterpret_cast<uint32_t*>(smem_raw + a.off_sel) + r;
+    // Qbar of this query tile, split into two bf16 terms, as the A operand:
+    // set s writes dims 64 s .. 64 s + 63
     {
-      const float* src = a.qbar + row * kHeadDim;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {            // 64 dims = 32 bf16 pairs = 32 columns per chunk
-        uint32_t w0[32], w1[32], w2[32];
+      const float* src = a.qbar + row * kHeadDim + 64 * set;
+      uint32_t w0[32], w1[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          uint32_t hi[2], mid[2], lo[2];
+      for (int i = 0; i < 32; ++i) {
+        uint32_t hi[2], lo[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float x = row_ok ? src[64 * c + 2 * i + e] : 0.f;
-            const float hv = bf16_round(x);
-            const float mv = bf16_round(x - hv);
-            const float lv = bf16_round(x - hv - mv);
-            hi[e] = bf16_bits(hv);
-            mid[e] = bf16_bits(mv);
-            lo[e] = bf16_bits(lv);
-          }
-          w0[i] = hi[0] | (hi[1] << 16);
-          w1[i] = mid[0] | (mid[1] << 16);
-          w2[i] = lo[0] | (lo[1] << 16);
+        for (int e = 0; e < 2; ++e) {
+          const float x = row_ok ? src[2 * i + e] : 0.f;
+          const float hv = bf16_round(x);
+          hi[e] = bf16_bits(hv);
+          lo[e] = bf16_bits(bf16_round(x - hv));
         }
-        tmem_st32x32(lane_addr + kXColA + 0 * 64 + 32 * c, w0);
-        tmem_st32x32(lane_addr + kXColA + 1 * 64 + 32 * c, w1);
-        tmem_st32x32(lane_addr + kXColA + 2 * 64 + 32 * c, w2);
+        w0[i] = hi[0] | (hi[1] << 16);
+        w1[i] = lo[0] | (lo[1] << 16);
       }
+      tmem_st32x32(lane_addr + kXColA + 0 * 64 + 32 * set, w0);
+      tmem_st32x32(lane_addr + kXColA + 1 * 64 + 32 * set, w1);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.a_ready));
     }
-    // walk the candidate key tiles; skip the ones this query tile selected
-    const int n_sel = row_ok ? min(max(a.cnt[row], 0), a.kmax) : 0;
-    const int32_t* list = a.idx + row * a.kmax;
-    int p = 0;
-    int nxt = n_sel > 0 ? list[0] : INT_MAX;
+    // the tiles this query tile selected, as a bitmap in shared memory (set 0
+    // builds it); entries outside [0, n_cand) are ignored
+    if (set == 0) {
+      const int n_words = x_sel_words(a.n_cand);
+      for (int w = 0; w < n_words; ++w) sel[w * kXRows] = 0u;
+      const int n_sel = row_ok ? min(max(a.cnt[row], 0), a.kmax) : 0;
+      const int32_t* list = a.idx + row * a.kmax;
+      for (int i = 0; i < n_sel; ++i) {
+        const int cs = list[i];
+        if (cs >= 0 && cs < a.n_cand) sel[(cs >> 5) * kXRows] |= 1u << (cs & 31);
+      }
+    }
+    x_rows_sync();
     int count = 0, worst = 0, wt = 0;
     float wv = -INFINITY;
-    bool ok = true;
-    for (int t = 0; t < a.n_cand; ++t) {
-      if (!(ok = x_warp_wait(sm, sm.d_full[t & 1], (t >> 1) & 1, lane, a.err))) break;
+    // the valid-slot mask and origin of this set's tiles, loaded two pairs
+    // ahead (a load from L2 takes longer than a pair's scores)
+    unsigned long long vm_n[2];
+    int4 org_n[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int t = 2 * j + set;
+      const int tile = a.cand0 + (t < a.n_cand ? x_rotate(t, rot, a.n_cand) : 0);
+      vm_n[j] = t < a.n_cand ? a.L.valid[tile] : 0ull;
+      org_n[j] = t < a.n_cand ? a.L.origin[tile] : make_int4(0, 0, 0, 0);
+    }
+    for (int p = 0; p < n_pairs; ++p) {
+      const int t = 2 * p + set;
+      if (t >= a.n_cand) break;                  // an odd count's last pair has no second tile
+      const int tt = x_rotate(t, rot, a.n_cand);
+      const unsigned long long vm = vm_n[0];
+      const int4 org = org_n[0];
+      vm_n[0] = vm_n[1];
+      org_n[0] = org_n[1];
+      if (t + 4 < a.n_cand) {
+        const int tile = a.cand0 + x_rotate(t + 4, rot, a.n_cand);
+        vm_n[1] = a.L.valid[tile];
+        org_n[1] = a.L.origin[tile];
+      }
+      if (!x_warp_wait(sm, sm.d_full[p & 1], (p >> 1) & 1, lane, a.err)) break;
       tc_fence_after();
       float x0[32], x1[32];
-      tmem_ld32x32f(lane_addr + kXColD + 64u * (t & 1), x0);
-      tmem_ld32x32f(lane_addr + kXColD + 64u * (t & 1) + 32, x1);
+      const uint32_t dcol = kXColD + 128u * (p & 1) + 64u * set;
+      tmem_ld32x32f(lane_addr + dcol, x0);
+      tmem_ld32x32f(lane_addr + dcol + 32, x1);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.d_free[t & 1]));
-      while (nxt < t) nxt = ++p < n_sel ? list[p] : INT_MAX;   // lists are ascending (anything else is skipped over)
-      if (nxt == t) {
-        nxt = ++p < n_sel ? list[p] : INT_MAX;
-        continue;
-      }
-      if (!row_ok) continue;
-      const int tile = a.cand0 + t;
-      const unsigned long long vm = a.L.valid[tile];
-      const int32_t* perm_tile = a.L.perm + tile * kTile;
+      if (lane == 0) mbar_arrive(smem_u32(&sm.d_free[p & 1]));
+      if (((sel[(tt >> 5) * kXRows] >> (tt & 31)) & 1u) || !row_ok) continue;
       // slots that may enter the top-E: a branch-free mask first (after the
       // first tiles almost none qualify, and a branch per slot costs far more
       // than the compare), then one offer per set bit in slot order
-      const float lim = count < a.E ? -INFINITY : wv;
-      uint32_t m0 = 0, m1 = 0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        m0 |= (x0[i] >= lim ? 1u : 0u) << i;
-        m1 |= (x1[i] >= lim ? 1u : 0u) << i;
-      }
-      unsigned long long cand = (static_cast<unsigned long long>(m1) << 32 | m0) & vm;
+      unsigned long long cand = x_mask_ge(x0, x1, count < a.E ? -INFINITY : wv) & vm;
+      if (__popcll(cand) > a.E) cand = x_narrow(x0, x1, cand, a.E);   // early tiles: most slots qualify
       while (cand) {
         const int i = __ffsll(static_cast<long long>(cand)) - 1;
         cand &= cand - 1;
-        // the scores stay in registers: pick slot i's without dynamic indexing
-        float xi = 0.f;
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          xi = (i == u) ? x0[u] : xi;
-          xi = (i == 32 + u) ? x1[u] : xi;
-        }
-        if (count < a.E || xi >= wv) x_offer(sm, perm_tile, r, a.E, xi, i, count, worst, wv, wt);
+        const float xi = x_pick(x0, x1, i);   // the scores stay in registers
+        if (count < a.E || xi >= wv) x_offer(val, tok, a.E, xi, x_token(a.L, org, i), count, worst, wv, wt);
       }
     }
-    if (ok && row_ok) {
+    // merge: set 0 offers set 1's entries to its own list, then writes it out
+    if (set == 1) sm.cnt1[r] = count;
+    x_rows_sync();
+    if (set == 0 && row_ok && !*reinterpret_cast<volatile int*>(&sm.abort)) {
+      const float* val1 = val + 2 * ep * kXRows;
+      const int* tok1 = tok + 2 * ep * kXRows;
+      const int n1 = sm.cnt1[r];
+      for (int e = 0; e < n1; ++e) {
+        const float s1 = val1[e * kXRows];
+        if (count < a.E || s1 >= wv) x_offer(val, tok, a.E, s1, tok1[e * kXRows], count, worst, wv, wt);
+      }
       int32_t* dst = a.out_idx + row * a.E;
-      for (int e = 0; e < count; ++e) dst[e] = sm.tok[e * kXRows + r];
+      for (int e = 0; e < count; ++e) dst[e] = tok[e * kXRows];
       a.out_cnt[row] = count;
     }
   }
@@ -451,10 +624,22 @@ vsa_status vsa_extra_tokens_select(const vsa_layout* L, const vsa_params* p, int
   if (e != cudaSuccess) return cuda_fail("vsa_extra_tokens_select: permute/pool launch", e);
   const int rows = L->n_tiles - a.c0;
   if (rows > 0) {
-    const size_t smem = sizeof(XSmem);
-    e = cudaFuncSetAttribute(extra_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    // as many key tile pair stages as fit next to the two top-E lists and the
+    // bitmap (the copies take thousands of cycles to land), at most four
+    int stages = kXStagesMax;
+    while (stages > 1 && x_smem_layout(stages, a.E, cand.count).total > kXSmemMax) --stages;
+    const XSmemLayout sl = x_smem_layout(stages, a.E, cand.count);
+    if (sl.total > kXSmemMax) {
+      set_detail("vsa_extra_tokens_select: the candidate bitmap and the top-E lists exceed shared memory");
+      return VSA_ERR_UNSUPPORTED;
+    }
+    a.stages = stages;
+    a.off_val = sl.val;
+    a.off_sel = sl.sel;
+    e = cudaFuncSetAttribute(extra_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sl.total));
     if (e != cudaSuccess) return cuda_fail("vsa_extra_tokens_select: cudaFuncSetAttribute", e);
-    extra_select_kernel<<<dim3((rows + kXRows - 1) / kXRows, H, B), kXThreads, smem, stream>>>(a);
+    extra_select_kernel<<<dim3((rows + kXRows - 1) / kXRows, H, B), kXThreads, sl.total, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("vsa_extra_tokens_select: launch", e);
   }

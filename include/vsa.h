@@ -321,9 +321,13 @@ vsa_status vsa_extra_tokens_workspace_size(const vsa_layout* layout, int32_t B, 
  *                   its first word is the status that vsa_extra_tokens_status
  *                   reads (a kernel wait that ran out).
  * Scores: fp32 accumulation of the exact bf16 keys against the fp32 pooled
- * query split into three bf16 terms (tensor cores), so the chosen set matches
- * an fp64 evaluation except where two scores tie within fp32 rounding.
- * Errors: INVALID_ARG when params->extra_tokens is 0 (nothing to choose). */
+ * query split into two bf16 terms (tensor cores; the query to a relative
+ * 2^-17), so the chosen set matches an fp64 evaluation except where two
+ * scores tie within about fp32 rounding.
+ * Errors: INVALID_ARG when params->extra_tokens is 0 (nothing to choose);
+ * UNSUPPORTED when a bitmap of the candidate tiles, two top-E lists and one
+ * 32 KB key stage per 128 query tiles exceed 227 KB of shared memory (more
+ * than about 10k candidate tiles at E = 16, 4.2k at E = 64). */
 vsa_status vsa_extra_tokens_select(const vsa_layout* layout, const vsa_params* params,
                                    int32_t B, int32_t H, const void* q, const void* k,
                                    int64_t stride_b, int64_t stride_s, int64_t stride_h,

@@ -114,3 +114,29 @@ def test_5s_extra_tokens(cuda_ok):
         C.note_near_ties(len(near_x))
         gpu_extra = {qt: res["extra_idx"][0, h, qt, :E] for qt in tiles}
         C.compare_outputs(ho, res, 0, h, tiles, near_tie=near, extra=gpu_extra)
+
+
+def test_10s_extra_tokens_e64(cuda_ok):
+    """extra_tokens on the 10 s clip with E = 64: the bitmap of ~3.8k candidate
+    tiles and two 64-entry top-E lists leave shared memory for a single key
+    tile pair stage, the smallest pipeline the kernel runs."""
+    wl = W.WORKLOADS["10s"]
+    E = 64
+    lay = C.oracle_layout(wl)
+    q, k, v, g = C.inputs(wl, lay)
+    prm = C.params_of(wl, extra_tokens=E)
+    assert prm["sink"] == O.SINK_EXACT_KV_AND_ROWS   # dense conditioning rows take no extra tokens
+    res = C.gpu_forward(wl, (q, k, v, g), prm)
+    assert res["status"] == vsa.OK and res["extra_status"] == vsa.OK
+    nc = lay.n_cond_tiles
+    assert np.all(res["extra_cnt"][:, :, :nc] == 0)
+    assert res["extra_cnt"][:, :, nc:].min() == E and res["extra_cnt"][:, :, nc:].max() == E
+    rng = np.random.default_rng(5)
+    h = 11
+    ho = C.HeadOracle(wl, lay, (q, k, v, g), 0, h, prm)
+    near = C.compare_selection(ho, res["idx"][0, h], res["cnt"][0, h])
+    tiles = sorted(set(sample_tiles(lay, rng, 3)) | set(list(near)[:2]))
+    near_x = C.compare_extra(ho, res["extra_idx"][0, h], res["extra_cnt"][0, h], tiles, near)
+    C.note_near_ties(len(near_x))
+    gpu_extra = {qt: res["extra_idx"][0, h, qt, :E] for qt in tiles}
+    C.compare_outputs(ho, res, 0, h, tiles, near_tie=near, extra=gpu_extra)
