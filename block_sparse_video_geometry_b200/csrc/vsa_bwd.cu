@@ -26,15 +26,18 @@
 //  * dkv_kernel: one CTA per (batch, head, key tile) walking the query tiles
 //    that attend it (all of them for conditioning keys; for a candidate tile,
 //    dense conditioning rows plus the transpose of the selection lists, built
-//    on the GPU by a counting sort); S^T = K Q^T and dP^T = V dO^T with K and
-//    V in TMEM and Q, dO bulk-copied tile-major tiles, then dV += P^T dO and
+//    on the GPU by a counting sort); S^T = K Q^T and dP^T = V dO^T with K, V,
+//    Q and dO as bulk-copied shared-memory tiles, then dV += P^T dO and
 //    dK += dS^T Q with P^T, dS^T (bf16) in TMEM.
+//  * Both are warp-specialised pipelines: a copy warp keeps four 32 KB stages
+//    in flight, an MMA warp issues step j + 1's two products before step j's
+//    accumulation, and eight warps run the elementwise step on the other of
+//    two TMEM score buffers meanwhile (two per TMEM quadrant, each half of a
+//    thread pair's 32 columns: 16 exponentials per thread and step).
 //  * The coarse branch runs on CUDA cores in fp32 (like its forward):
 //    dOc and dg in one pass over the tokens, a row pass per 64 query tiles
 //    (softmax statistics, P, dS, dQbar), a column pass per 64 candidate tiles
 //    (dKbar, dVbar), and a scatter through the pooling.
-//  Both fine kernels run their MMAs and the elementwise step in turn (one CTA
-//  per SM, bulk copies of the next tiles in flight meanwhile).
 
 #include <cuda_runtime.h>
 
@@ -50,34 +53,39 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBThreads = 128;
+constexpr int kBThreads = 352;           // warp 0 copies, warps 1 and 10 MMAs, warps 2-9 the elementwise step
+constexpr int kBStages = 4;              // copy stages of 32 KB
 constexpr uint32_t kBTmemCols = 512;
 constexpr uint32_t kTB = 16384;          // one tile of Q, K, V or dO: [d half][64 rows][128 B]
 constexpr uint64_t kBTimeoutNs = 4000000000ull;
 constexpr uint64_t kBDrainNs = 200000000ull;
 constexpr size_t kBHeader = 256;         // status word
-constexpr size_t kBSmem = 120 * 1024;    // requested so that one CTA holds an SM (512 TMEM columns)
 
-// TMEM columns (lanes 0-15 of every quadrant: M = 64)
-//  dq_kernel : Q 0-63, dO 64-127, S / dS 128-191, dP 192-255, dQ 256-383
-//  dkv_kernel: K 0-63, V 64-127, S^T / P^T 128-191, dP^T / dS^T 192-255, dK 256-383, dV 384-511
-constexpr uint32_t kColA0 = 0, kColA1 = 64, kColS = 128, kColP = 192, kColAcc0 = 256, kColAcc1 = 384;
+// TMEM columns (lanes 0-15 of every quadrant: M = 64); S and dP are double
+// buffered so that step j + 1's products run during step j's elementwise work
+//  dq_kernel : Q 0-63, dO 64-127, S / dS [b] 128 + 128 b, dP [b] 192 + 128 b, dQ 384-511
+//  dkv_kernel: S^T / P^T [b] 128 b, dP^T / dS^T [b] 64 + 128 b, dK 256-383, dV 384-511
+//              (K and V stay in shared memory as A operands)
+constexpr uint32_t kQColQ = 0, kQColDO = 64, kQColS = 128, kQColP = 192, kQColAcc = 384;
+constexpr uint32_t kKColS = 0, kKColP = 64, kKColDK = 256, kKColDV = 384;
 
-struct BSmem {
-  uint8_t t0[2][kTB];                    // dq: K stages; dkv: Q stages
-  uint8_t t1[2][kTB];                    // dq: V stages; dkv: dO stages
-  float rowstat[2][2][64];               // dkv: lse and D of the query tile of each stage
-  uint64_t full[2], mma_done, acc_done;
+// Shared memory: this header, then (1024-byte aligned) the tiles.
+//  dq_kernel : stage s (K then V of a key tile) at 1024 + 32 KB s
+//  dkv_kernel: the key tile's K and V at 1024, stage s (Q then dO of a query
+//              tile) at 1024 + 32 KB (s + 1), then the stages' row statistics
+struct BHead {
+  uint64_t full[kBStages], free_[kBStages], s_full[2], p_full[2], ds_ready[2], a_ready, acc_done;
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(BHead) <= 1024, "tiles start at byte 1024");
+constexpr size_t kDqSmem = 1024 + kBStages * 2 * kTB;
+constexpr size_t kDkvSmem = 1024 + 2 * kTB + kBStages * 2 * kTB + kBStages * 2 * 64 * sizeof(float);
 
 struct BArgs {
   DevLayout L;
   int32_t H, sink, n_cond, cand0, n_cand, kmax, c0;     // c0 = dense conditioning rows (0 unless rows mode)
   const uint16_t* q;                     // natural layout [B, S, H, 128]
-  const uint16_t* k;
-  const uint16_t* v;
   const uint16_t* dout;
   int64_t sb, ss, sh;                    // strides of q, k, v
   int64_t d_sb, d_ss, d_sh;              // strides of dO
@@ -98,16 +106,66 @@ struct BArgs {
   int* err;
 };
 
-__device__ __forceinline__ void b_abort(BSmem& sm, int* err) {
+__device__ __forceinline__ void b_abort(BHead& sm, int* err) {
   atomicExch(err, VSA_ERR_TIMEOUT);
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
-// every thread of the block waits (bounded) on a barrier phase
-__device__ __forceinline__ bool b_wait(BSmem& sm, uint64_t& bar, uint32_t parity, int* err) {
+// the calling threads wait (bounded) on a barrier phase; a phase that has
+// already completed is taken with a non-suspending test first (a try_wait on
+// it still costs a few hundred cycles)
+__device__ __forceinline__ bool b_wait(BHead& sm, uint64_t& bar, uint32_t parity, int* err) {
+  if (mbar_test_wait(smem_u32(&bar), parity)) return true;
   const bool ok = mbar_wait(smem_u32(&bar), parity, &sm.abort, kBTimeoutNs);
   if (!ok) b_abort(sm, err);
   return ok;
+}
+
+// a_ready_count: arrivals that complete a_ready (dq: the eight elementwise
+// warps after writing Q and dO into TMEM; dkv: the copy of K and V);
+// free_count: MMA warps whose accumulation reads a stage
+__device__ __forceinline__ void b_init(BHead& sm, uint32_t a_ready_count, uint32_t free_count) {
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 1);
+      mbar_init(smem_u32(&sm.free_[s]), free_count);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.p_full[i]), 1);
+      mbar_init(smem_u32(&sm.ds_ready[i]), 8);   // one arrival per elementwise warp
+    }
+    mbar_init(smem_u32(&sm.a_ready), a_ready_count);
+    mbar_init(smem_u32(&sm.acc_done), 2);       // both MMA warps, after their last MMA
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kBTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+// Copy-warp loop (lane 0): step j's tiles into stage j % kBStages once the
+// MMAs of step j - kBStages released it; on a failed wait, lets the copies in
+// flight land before returning.
+template <class Issue>
+__device__ __forceinline__ void b_copy_loop(BHead& sm, int n, int* err, Issue issue) {
+  int issued = 0;
+  bool ok = true;
+  for (int j = 0; j < n; ++j) {
+    const int st = j % kBStages;
+    if (j >= kBStages && !(ok = b_wait(sm, sm.free_[st], ((j / kBStages) - 1) & 1, err))) break;
+    issue(j, st, smem_u32(&sm.full[st]));
+    ++issued;
+  }
+  if (!ok)
+    for (int i = max(0, issued - kBStages); i < issued; ++i)
+      mbar_wait(smem_u32(&sm.full[i % kBStages]), (i / kBStages) & 1, nullptr, kBDrainNs);
 }
 
 // 64-row tile of a natural-layout [B, S, H, 128] tensor into TMEM as an M = 64
@@ -131,7 +189,7 @@ __device__ __forceinline__ void rows_to_tmem(const uint16_t* base, const int32_t
 // Key tile of step jj of query tile qt's key set in the forward: dense rows
 // all tiles; otherwise the conditioning tiles (unless the sink is off), then
 // the selection list.
-__device__ __forceinline__ int dq_step_tile(const BArgs& a, int qt, size_t row, int jj, bool dense, int n_fixed) {
+__device__ __forceinline__ int dq_step_tile(const BArgs& a, size_t row, int jj, bool dense, int n_fixed) {
   if (dense || jj < n_fixed) return jj;
   const int c = a.idx[row * a.kmax + (jj - n_fixed)];
   return a.cand0 + min(max(c, 0), a.n_cand - 1);
@@ -146,126 +204,133 @@ __device__ __forceinline__ int dkv_step_tile(const BArgs& a, const int32_t* list
 }
 
 // -------------------------------------------------------------------- dQ
+// Per step j (key tile t_j): S = Q K^T and dP = dO V^T into buffer j & 1;
+// the elementwise warps turn them into dS = P (dP - D) (bf16, over S); then
+// dQ += dS K. The MMA warp issues S(j), dP(j) before dQ(j - 1), so the tensor
+// pipe has the next products queued while the elementwise step runs.
 __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant__ BArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
     return;
   }
-  BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hf = lane >> 4;
+  BHead& sm = *reinterpret_cast<BHead*>(smem_raw);
+  uint8_t* const stage0 = smem_raw + 1024;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const size_t bh = static_cast<size_t>(b) * a.H + h;
   const size_t row = bh * a.L.n_tiles + qt;
   const bool dense = qt < a.c0;
   const int n_fixed = (a.sink == VSA_SINK_OFF || dense) ? 0 : a.n_cond;
   const int n = dense ? a.L.n_tiles : n_fixed + min(max(a.cnt[row], 1), a.kmax);
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&sm.full[0]), 1);
-    mbar_init(smem_u32(&sm.full[1]), 1);
-    mbar_init(smem_u32(&sm.mma_done), 1);
-    mbar_init(smem_u32(&sm.acc_done), 1);
-    sm.abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(&sm.tmem_base), kBTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  b_init(sm, 8, 1);
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // lanes 32 w .. 32 w + 15
-  const int r = warp * 16 + (lane & 15);
-  const int32_t* perm_q = a.L.perm + qt * kTile;
-  rows_to_tmem(a.q + b * a.sb + h * a.sh, perm_q, a.ss, r, hf, lane_addr + kColA0);
-  rows_to_tmem(a.dout + b * a.d_sb + h * a.d_sh, perm_q, a.d_ss, r, hf, lane_addr + kColA1);
-  tmem_wait_st();
-  const float lse = a.lse[row * kTile + r];
-  const float dd = a.dd[row * kTile + r];
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint8_t* head_kv = a.kv + bh * a.L.n_tiles * 32768u;
-  auto issue = [&](int jj) {           // K and V of step jj into stage jj & 1
-    const int t = dq_step_tile(a, qt, row, jj, dense, n_fixed);
-    const uint32_t bar = smem_u32(&sm.full[jj & 1]);
-    mbar_arrive_expect_tx(bar, 2 * kTB);
-    bulk_load(smem_u32(sm.t0[jj & 1]), head_kv + static_cast<size_t>(t) * 32768u, kTB, bar);
-    bulk_load(smem_u32(sm.t1[jj & 1]), head_kv + static_cast<size_t>(t) * 32768u + kTB, kTB, bar);
-  };
-  if (threadIdx.x == 0) {
-    issue(0);
-    if (n > 1) issue(1);
-  }
-  bool ok = true;
-  int issued = n > 1 ? 2 : 1;
-  for (int jj = 0; jj < n; ++jj) {
-    const int st = jj & 1;
-    if (!(ok = b_wait(sm, sm.full[st], (jj >> 1) & 1, a.err))) break;
-    const int t = dq_step_tile(a, qt, row, jj, dense, n_fixed);
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      // S = Q K^T and dP = dO V^T (V K-major like K: [keys][d])
-      const uint64_t kd = smem_desc_sw128(smem_u32(sm.t0[st]), 16, 1024);
-      const uint64_t vd = smem_desc_sw128(smem_u32(sm.t1[st]), 16, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t off = (kk >> 2) * (8192 >> 4) + (kk & 3) * 2;
-        umma_ts(tmem + kColS, tmem + kColA0 + kk * 8, kd + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
-        umma_ts(tmem + kColP, tmem + kColA1 + kk * 8, vd + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
-      }
-      umma_commit(smem_u32(&sm.mma_done));
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint8_t* head_kv = a.kv + bh * a.L.n_tiles * 32768u;
+      b_copy_loop(sm, n, a.err, [&](int j, int st, uint32_t bar) {
+        const int t = dq_step_tile(a, row, j, dense, n_fixed);
+        const uint32_t dst = smem_u32(stage0 + st * 2 * kTB);
+        mbar_arrive_expect_tx(bar, 2 * kTB);
+        bulk_load(dst, head_kv + static_cast<size_t>(t) * 32768u, kTB, bar);
+        bulk_load(dst + kTB, head_kv + static_cast<size_t>(t) * 32768u + kTB, kTB, bar);
+      });
     }
-    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj) & 1, a.err))) break;
-    tc_fence_after();
-    float s[32], dp[32];
-    tmem_ld16x2_32f<32>(lane_addr + kColS, s);
-    tmem_ld16x2_32f<32>(lane_addr + kColP, dp);
-    tmem_wait_ld();
-    const unsigned long long vm = a.L.valid[t];
-    const uint32_t vbits = static_cast<uint32_t>(vm >> (32 * hf));
-    uint32_t w[16];
+    __syncwarp();
+  } else if (warp == 1 || warp == 10) {
+    // two MMA issuers, so that the tensor pipe interleaves two independent
+    // chains: warp 1 S = Q K^T and dQ += dS K, warp 10 dP = dO V^T (V K-major
+    // like K: [keys][d]); buffer j & 1 is rewritten only after the
+    // elementwise warps released step j - 2 (warp 1: its dQ(j - 2) precedes
+    // in issue order; warp 10: it waits for ds_ready(j - 2))
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(64, 64, 0, 0), kIdQ = idesc_bf16_f32(64, 128, 0, 1);
+      const bool is_s = warp == 1;
+      bool ok = b_wait(sm, sm.a_ready, 0, a.err);
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % kBStages;
+          const uint32_t bs = 128u * (j & 1);
+          if (!(ok = b_wait(sm, sm.full[st], (j / kBStages) & 1, a.err))) break;
+          if (!is_s && j >= 2 && !(ok = b_wait(sm, sm.ds_ready[j & 1], ((j >> 1) - 1) & 1, a.err))) break;
+          tc_fence_after();
+          const uint64_t bd = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB + (is_s ? 0u : kTB)), 16, 1024);
+          const uint32_t dcol = (is_s ? kQColS : kQColP) + bs, acol = is_s ? kQColQ : kQColDO;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float ds[2];
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + dcol, tmem + acol + kk * 8, bd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdS, kk > 0);
+          umma_commit(smem_u32(is_s ? &sm.s_full[j & 1] : &sm.p_full[j & 1]));
+        }
+        if (is_s && j >= 1) {
+          const int jp = j - 1, stp = jp % kBStages;
+          if (!(ok = b_wait(sm, sm.ds_ready[jp & 1], (jp >> 1) & 1, a.err))) break;
+          tc_fence_after();
+          // dQ += dS K: dS (A) in TMEM, K as the MN-major B operand ([keys][d])
+          const uint64_t kmn = smem_desc_sw128(smem_u32(stage0 + stp * 2 * kTB), 8192, 1024);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int key = 2 * i + e;
-        const float p = ((vbits >> key) & 1u) ? ex2_approx(fmaf(s[key], a.c_log2, -lse)) : 0.f;
-        ds[e] = p * (dp[key] - dd);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + kQColAcc, tmem + kQColS + 128u * (jp & 1) + kk * 8, kmn + kk * (2048 >> 4), kIdQ,
+                    (jp > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&sm.free_[stp]));   // dP(jp) completed before the elementwise step released it
+        }
       }
-      w[i] = pack_bf16x2(ds[0], ds[1]);
+      umma_commit(smem_u32(&sm.acc_done));     // every MMA issued, also on a failed wait
+      mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
     }
-    tmem_st16x2_16<16>(lane_addr + kColS, w);    // dS (bf16 pairs) over S
+    __syncwarp();
+  } else {
+    // thread (row r, half hf) of column set cs: keys 32 hf + 16 cs .. + 15
+    const int qd = warp & 3, hf = lane >> 4, cs = (warp - 2) >> 2;
+    const int r = qd * 16 + (lane & 15);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(qd * 32) << 16);   // lanes 32 qd .. 32 qd + 15
+    const int32_t* perm_q = a.L.perm + qt * kTile;
+    if (cs == 0) rows_to_tmem(a.q + b * a.sb + h * a.sh, perm_q, a.ss, r, hf, lane_addr + kQColQ);
+    else rows_to_tmem(a.dout + b * a.d_sb + h * a.d_sh, perm_q, a.d_ss, r, hf, lane_addr + kQColDO);
     tmem_wait_st();
     tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.a_ready));
+    const float lse = a.lse[row * kTile + r];
+    const float dd = a.dd[row * kTile + r];
+    unsigned long long vm_next = a.L.valid[dq_step_tile(a, row, 0, dense, n_fixed)];
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const unsigned long long vm = vm_next;
+      if (j + 1 < n) vm_next = a.L.valid[dq_step_tile(a, row, j + 1, dense, n_fixed)];
+      const uint32_t bs = 128u * (j & 1);
+      if (!(ok = b_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, a.err))) break;
+      if (!(ok = b_wait(sm, sm.p_full[j & 1], (j >> 1) & 1, a.err))) break;
       tc_fence_after();
-      // dQ += dS K: dS (A) in TMEM, K as the MN-major B operand ([keys][d])
-      const uint64_t kmn = smem_desc_sw128(smem_u32(sm.t0[st]), 8192, 1024);
+      float s[16], dp[16];
+      tmem_ld16x2_16f<32>(lane_addr + kQColS + bs + 16 * cs, s);
+      tmem_ld16x2_16f<32>(lane_addr + kQColP + bs + 16 * cs, dp);
+      tmem_wait_ld();
+      const uint32_t vbits = static_cast<uint32_t>(vm >> (32 * hf + 16 * cs));
+      uint32_t w[8];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        umma_ts(tmem + kColAcc0, tmem + kColS + kk * 8, kmn + kk * (2048 >> 4), idesc_bf16_f32(64, 128, 0, 1),
-                (jj > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(smem_u32(&sm.mma_done));
+      for (int i = 0; i < 8; ++i) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = 2 * i + e;
+          const float p = ((vbits >> key) & 1u) ? ex2_approx(fmaf(s[key], a.c_log2, -lse)) : 0.f;
+          ds[e] = p * (dp[key] - dd);
+        }
+        w[i] = pack_bf16x2(ds[0], ds[1]);
+      }
+      tmem_st16x2_8<16>(lane_addr + kQColS + bs + 8 * cs, w);    // dS (bf16 pairs) over S
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.ds_ready[j & 1]));
     }
-    // the stage is free (and S may be overwritten) once dQ += dS K completed
-    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj + 1) & 1, a.err))) break;
-    if (threadIdx.x == 0 && jj + 2 < n) {
-      issue(jj + 2);
-      ++issued;
-    }
-  }
-  if (ok) {
-    tc_fence_after();
-    const int tok = perm_q[r];
-#pragma unroll 1
-    for (int ch = 0; ch < 2; ++ch) {
+    if (ok && (ok = b_wait(sm, sm.acc_done, 0, a.err))) {
+      tc_fence_after();
+      const int tok = perm_q[r];
+      const int ch = cs;                               // dims 64 hf + 32 cs .. + 31
       float y[32];
-      tmem_ld16x2_32f<64>(lane_addr + kColAcc0 + 32 * ch, y);
+      tmem_ld16x2_32f<64>(lane_addr + kQColAcc + 32 * ch, y);
       tmem_wait_ld();
       if (tok >= 0) {
         float4* dst = reinterpret_cast<float4*>(a.dq + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
@@ -275,30 +340,31 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
           dst[i / 4] = make_float4(y[i] * a.scale, y[i + 1] * a.scale, y[i + 2] * a.scale, y[i + 3] * a.scale);
       }
     }
-  } else if (threadIdx.x == 0) {
-    // let every issued copy land before the block exits
-    for (int i = max(0, issued - 2); i < issued; ++i)
-      mbar_wait(smem_u32(&sm.full[i & 1]), (i >> 1) & 1, nullptr, kBDrainNs);
-    umma_commit(smem_u32(&sm.acc_done));
-    mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kBTmemCols);
   }
 }
 
 // -------------------------------------------------------------- dK and dV
+// Per step j (query tile q_j): S^T = K Q^T and dP^T = V dO^T into buffer
+// j & 1 (K and V of this CTA's key tile in shared memory as A operands); the
+// elementwise warps write P^T and dS^T = P^T (dP^T - D) (bf16, in place); then
+// dV += P^T dO and dK += dS^T Q, issued after the next step's products.
 __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant__ BArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
     return;
   }
-  BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hf = lane >> 4;
+  BHead& sm = *reinterpret_cast<BHead*>(smem_raw);
+  uint8_t* const kvt = smem_raw + 1024;
+  uint8_t* const stage0 = kvt + 2 * kTB;
+  float* const rowstat = reinterpret_cast<float*>(stage0 + kBStages * 2 * kTB);   // [stage][lse, D][64]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const size_t bh = static_cast<size_t>(b) * a.H + h;
   const int n_tiles = a.L.n_tiles;
@@ -313,144 +379,139 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant
     list = a.csr_list + off[c];
     n = a.c0 + (off[c + 1] - off[c]);
   }
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&sm.full[0]), 1);
-    mbar_init(smem_u32(&sm.full[1]), 1);
-    mbar_init(smem_u32(&sm.mma_done), 1);
-    mbar_init(smem_u32(&sm.acc_done), 1);
-    sm.abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(&sm.tmem_base), kBTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  b_init(sm, 1, 2);
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  const int r = warp * 16 + (lane & 15);            // key slot of this thread
-  const int32_t* perm_k = a.L.perm + kt * kTile;
-  rows_to_tmem(a.k + b * a.sb + h * a.sh, perm_k, a.ss, r, hf, lane_addr + kColA0);
-  rows_to_tmem(a.v + b * a.sb + h * a.sh, perm_k, a.ss, r, hf, lane_addr + kColA1);
-  tmem_wait_st();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  auto issue = [&](int jj) {           // Q, dO and the row statistics of step jj into stage jj & 1
-    const int qt = dkv_step_tile(a, list, jj, all_rows);
-    const size_t tq = bh * n_tiles + qt;
-    const uint32_t bar = smem_u32(&sm.full[jj & 1]);
-    mbar_arrive_expect_tx(bar, 2 * kTB + 2 * 256);
-    bulk_load(smem_u32(sm.t0[jj & 1]), a.qtm + tq * kTB, kTB, bar);
-    bulk_load(smem_u32(sm.t1[jj & 1]), a.dotm + tq * kTB, kTB, bar);
-    bulk_load(smem_u32(sm.rowstat[jj & 1][0]), a.lse + tq * kTile, 256, bar);
-    bulk_load(smem_u32(sm.rowstat[jj & 1][1]), a.dd + tq * kTile, 256, bar);
-  };
-  if (threadIdx.x == 0) {
-    if (n > 0) issue(0);
-    if (n > 1) issue(1);
-  }
-  bool ok = true;
-  int issued = min(n, 2);
-  for (int jj = 0; jj < n; ++jj) {
-    const int st = jj & 1;
-    if (!(ok = b_wait(sm, sm.full[st], (jj >> 1) & 1, a.err))) break;
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      // S^T = K Q^T and dP^T = V dO^T: K, V (A) in TMEM, Q and dO K-major
-      const uint64_t qd = smem_desc_sw128(smem_u32(sm.t0[st]), 16, 1024);
-      const uint64_t od = smem_desc_sw128(smem_u32(sm.t1[st]), 16, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t off = (kk >> 2) * (8192 >> 4) + (kk & 3) * 2;
-        umma_ts(tmem + kColS, tmem + kColA0 + kk * 8, qd + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
-        umma_ts(tmem + kColP, tmem + kColA1 + kk * 8, od + off, idesc_bf16_f32(64, 64, 0, 0), kk > 0);
-      }
-      umma_commit(smem_u32(&sm.mma_done));
-    }
-    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj) & 1, a.err))) break;
-    tc_fence_after();
-    float s[32], dp[32];
-    tmem_ld16x2_32f<32>(lane_addr + kColS, s);
-    tmem_ld16x2_32f<32>(lane_addr + kColP, dp);
-    tmem_wait_ld();
-    uint32_t wp[16], wd[16];
-    const float* lse = sm.rowstat[st][0] + 32 * hf;     // queries 32 hf .. 32 hf + 31 (columns of this thread)
-    const float* dd = sm.rowstat[st][1] + 32 * hf;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float p[2], ds[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int qi = 2 * i + e;
-        p[e] = ex2_approx(fmaf(s[qi], a.c_log2, -lse[qi]));    // padding query rows: lse = +inf, P = 0
-        ds[e] = p[e] * (dp[qi] - dd[qi]);
-      }
-      wp[i] = pack_bf16x2(p[0], p[1]);
-      wd[i] = pack_bf16x2(ds[0], ds[1]);
-    }
-    tmem_st16x2_16<16>(lane_addr + kColS, wp);          // P^T over S^T
-    tmem_st16x2_16<16>(lane_addr + kColP, wd);          // dS^T over dP^T
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      // dV += P^T dO and dK += dS^T Q: dO and Q as MN-major B operands ([queries][d])
-      const uint64_t omn = smem_desc_sw128(smem_u32(sm.t1[st]), 8192, 1024);
-      const uint64_t qmn = smem_desc_sw128(smem_u32(sm.t0[st]), 8192, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        umma_ts(tmem + kColAcc1, tmem + kColS + kk * 8, omn + kk * (2048 >> 4), idesc_bf16_f32(64, 128, 0, 1),
-                (jj > 0 || kk > 0) ? 1u : 0u);
-        umma_ts(tmem + kColAcc0, tmem + kColP + kk * 8, qmn + kk * (2048 >> 4), idesc_bf16_f32(64, 128, 0, 1),
-                (jj > 0 || kk > 0) ? 1u : 0u);
-      }
-      umma_commit(smem_u32(&sm.mma_done));
-    }
-    if (!(ok = b_wait(sm, sm.mma_done, (2 * jj + 1) & 1, a.err))) break;
-    if (threadIdx.x == 0 && jj + 2 < n) {
-      issue(jj + 2);
-      ++issued;
-    }
-  }
-  if (ok) {
-    tc_fence_after();
-    const int tok = perm_k[r];
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {          // dK (scaled), dV
-      float* dst_base = which == 0 ? a.dk : a.dv;
-      const float f = which == 0 ? a.scale : 1.0f;
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        float y[32];
-        if (n > 0) {
-          tmem_ld16x2_32f<64>(lane_addr + (which == 0 ? kColAcc0 : kColAcc1) + 32 * ch, y);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = 0.f;
-        }
-        if (tok >= 0) {
-          float4* dst = reinterpret_cast<float4*>(dst_base + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
-                                                  h * a.o_sh + 64 * hf + 32 * ch);
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            dst[i / 4] = make_float4(y[i] * f, y[i + 1] * f, y[i + 2] * f, y[i + 3] * f);
-        }
-      }
-    }
-  } else if (threadIdx.x == 0) {
-    for (int i = max(0, issued - 2); i < issued; ++i)
-      mbar_wait(smem_u32(&sm.full[i & 1]), (i >> 1) & 1, nullptr, kBDrainNs);
-    umma_commit(smem_u32(&sm.acc_done));
-    mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
-  }
-  tc_fence_before();
-  __syncthreads();
+
   if (warp == 0) {
+    if (lane == 0) {
+      // K and V of the key tile once (a_ready), then Q, dO and the row
+      // statistics of every attending query tile
+      mbar_arrive_expect_tx(smem_u32(&sm.a_ready), 2 * kTB);
+      bulk_load(smem_u32(kvt), a.kv + (bh * n_tiles + kt) * 32768u, 2 * kTB, smem_u32(&sm.a_ready));
+      b_copy_loop(sm, n, a.err, [&](int j, int st, uint32_t bar) {
+        const size_t tq = bh * n_tiles + dkv_step_tile(a, list, j, all_rows);
+        const uint32_t dst = smem_u32(stage0 + st * 2 * kTB);
+        mbar_arrive_expect_tx(bar, 2 * kTB + 2 * 256);
+        bulk_load(dst, a.qtm + tq * kTB, kTB, bar);
+        bulk_load(dst + kTB, a.dotm + tq * kTB, kTB, bar);
+        bulk_load(smem_u32(rowstat + st * 128), a.lse + tq * kTile, 256, bar);
+        bulk_load(smem_u32(rowstat + st * 128 + 64), a.dd + tq * kTile, 256, bar);
+      });
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp == 10) {
+    // two MMA issuers: warp 1 S^T = K Q^T and dV += P^T dO, warp 10
+    // dP^T = V dO^T and dK += dS^T Q (K, V, Q and dO K-major in shared memory
+    // for the products; dO and Q as MN-major B operands, [queries][d], for
+    // the accumulations); each rewrites its half of buffer j & 1 only after
+    // its own accumulation of step j - 2, and both release a stage
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(64, 64, 0, 0), kIdA = idesc_bf16_f32(64, 128, 0, 1);
+      const bool is_s = warp == 1;
+      const uint64_t ad = smem_desc_sw128(smem_u32(kvt + (is_s ? 0u : kTB)), 16, 1024);
+      bool ok = b_wait(sm, sm.a_ready, 0, a.err);
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % kBStages;
+          const uint32_t bs = 128u * (j & 1);
+          if (!(ok = b_wait(sm, sm.full[st], (j / kBStages) & 1, a.err))) break;
+          tc_fence_after();
+          const uint64_t bd = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB + (is_s ? 0u : kTB)), 16, 1024);
+          const uint32_t dcol = (is_s ? kKColS : kKColP) + bs;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t off = (kk >> 2) * (8192 >> 4) + (kk & 3) * 2;
+            umma_ss(tmem + dcol, ad + off, bd + off, kIdS, kk > 0);
+          }
+          umma_commit(smem_u32(is_s ? &sm.s_full[j & 1] : &sm.p_full[j & 1]));
+        }
+        if (j >= 1) {
+          const int jp = j - 1, stp = jp % kBStages;
+          const uint32_t bp = 128u * (jp & 1);
+          if (!(ok = b_wait(sm, sm.ds_ready[jp & 1], (jp >> 1) & 1, a.err))) break;
+          tc_fence_after();
+          // warp 1: dV += P^T dO; warp 10: dK += dS^T Q
+          const uint64_t bmn = smem_desc_sw128(smem_u32(stage0 + stp * 2 * kTB + (is_s ? kTB : 0u)), 8192, 1024);
+          const uint32_t acc = is_s ? kKColDV : kKColDK, acol = (is_s ? kKColS : kKColP) + bp;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + acc, tmem + acol + kk * 8, bmn + kk * (2048 >> 4), kIdA, (jp > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&sm.free_[stp]));
+        }
+      }
+      umma_commit(smem_u32(&sm.acc_done));     // every MMA issued, also on a failed wait
+      mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // thread (key slot r, half hf) of column set cs: queries 32 hf + 16 cs .. + 15
+    const int qd = warp & 3, hf = lane >> 4, cs = (warp - 2) >> 2;
+    const int r = qd * 16 + (lane & 15);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kBStages;
+      const uint32_t bs = 128u * (j & 1);
+      if (!(ok = b_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, a.err))) break;
+      if (!(ok = b_wait(sm, sm.p_full[j & 1], (j >> 1) & 1, a.err))) break;
+      tc_fence_after();
+      float s[16], dp[16];
+      tmem_ld16x2_16f<32>(lane_addr + kKColS + bs + 16 * cs, s);
+      tmem_ld16x2_16f<32>(lane_addr + kKColP + bs + 16 * cs, dp);
+      tmem_wait_ld();
+      uint32_t wp[8], wd[8];
+      const float* lse = rowstat + st * 128 + 32 * hf + 16 * cs;     // the queries of this thread's columns
+      const float* dd = rowstat + st * 128 + 64 + 32 * hf + 16 * cs;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float p[2], ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int qi = 2 * i + e;
+          p[e] = ex2_approx(fmaf(s[qi], a.c_log2, -lse[qi]));    // padding query rows: lse = +inf, P = 0
+          ds[e] = p[e] * (dp[qi] - dd[qi]);
+        }
+        wp[i] = pack_bf16x2(p[0], p[1]);
+        wd[i] = pack_bf16x2(ds[0], ds[1]);
+      }
+      tmem_st16x2_8<16>(lane_addr + kKColS + bs + 8 * cs, wp);     // P^T over S^T
+      tmem_st16x2_8<16>(lane_addr + kKColP + bs + 8 * cs, wd);     // dS^T over dP^T
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.ds_ready[j & 1]));
+    }
+    if (ok && (ok = b_wait(sm, sm.acc_done, 0, a.err))) {
+      tc_fence_after();
+      const int tok = a.L.perm[kt * kTile + r];
+      {
+        const int which = cs;                            // set 0: dK (scaled), set 1: dV
+        float* dst_base = which == 0 ? a.dk : a.dv;
+        const float f = which == 0 ? a.scale : 1.0f;
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          float y[32];
+          if (n > 0) {
+            tmem_ld16x2_32f<64>(lane_addr + (which == 0 ? kKColDK : kKColDV) + 32 * ch, y);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[i] = 0.f;
+          }
+          if (tok >= 0) {
+            float4* dst = reinterpret_cast<float4*>(dst_base + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
+                                                    h * a.o_sh + 64 * hf + 32 * ch);
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              dst[i / 4] = make_float4(y[i] * f, y[i + 1] * f, y[i + 2] * f, y[i + 3] * f);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kBTmemCols);
   }
@@ -1026,8 +1087,6 @@ vsa_status vsa_sparse_attn_bwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.kmax = kmax;
   a.c0 = c0;
   a.q = static_cast<const uint16_t*>(q);
-  a.k = static_cast<const uint16_t*>(k);
-  a.v = static_cast<const uint16_t*>(v);
   a.dout = static_cast<const uint16_t*>(dout);
   a.sb = sb;
   a.ss = ss;
@@ -1053,12 +1112,12 @@ vsa_status vsa_sparse_attn_bwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.scale = scale;
   a.c_log2 = scale * 1.4426950408889634f;
   a.err = static_cast<int*>(workspace);
-  for (auto kern : {dq_kernel, dkv_kernel}) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kBSmem));
-    if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute", e);
-  }
-  dq_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kBSmem, stream>>>(a);
-  dkv_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kBSmem, stream>>>(a);
+  e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDqSmem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dq)", e);
+  e = cudaFuncSetAttribute(dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDkvSmem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dkv)", e);
+  dq_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kDqSmem, stream>>>(a);
+  dkv_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kDkvSmem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: fine-branch launch", e);
 
