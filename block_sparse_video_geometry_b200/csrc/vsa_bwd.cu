@@ -106,6 +106,16 @@ struct BArgs {
   int* err;
 };
 
+// 16 lanes x 8 consecutive 32-bit columns per half-warp (16x32bx2 shape: the
+// upper half-warp at column offset `split`)
+template <int split>
+__device__ __forceinline__ void tmem_st16x2_8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], %1, {%2, %3, %4, %5, %6, %7, %8, %9};" ::"r"(taddr), "n"(split),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void b_abort(BHead& sm, int* err) {
   atomicExch(err, VSA_ERR_TIMEOUT);
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
