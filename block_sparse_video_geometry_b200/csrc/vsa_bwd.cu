@@ -30,10 +30,16 @@
 //    Q and dO as bulk-copied shared-memory tiles, then dV += P^T dO and
 //    dK += dS^T Q with P^T, dS^T (bf16) in TMEM.
 //  * Both are warp-specialised pipelines: a copy warp keeps four 32 KB stages
-//    in flight, an MMA warp issues step j + 1's two products before step j's
-//    accumulation, and eight warps run the elementwise step on the other of
-//    two TMEM score buffers meanwhile (two per TMEM quadrant, each half of a
-//    thread pair's 32 columns: 16 exponentials per thread and step).
+//    in flight; the MMAs are spread over several issuing warps (each
+//    tcgen05.mma holds its thread for tens of cycles, so one thread issuing a
+//    step's 20-24 MMAs was the bound; dq: S, dP and dQ on three warps, dkv:
+//    S^T with dV and dP^T with dK on two); the products of step j + 1 and the
+//    accumulations of step j run while eight warps do the elementwise step of
+//    the other of two TMEM score buffers (two per TMEM quadrant, each half of
+//    a thread pair's 32 columns: 16 exponentials per thread and step). A
+//    product rewrites its buffer only after the accumulation that read it two
+//    steps earlier has completed (dq: acc_a) or was issued before it by the
+//    same thread (dkv).
 //  * The coarse branch runs on CUDA cores in fp32 (like its forward):
 //    dOc and dg in one pass over the tokens, a row pass per 64 query tiles
 //    (softmax statistics, P, dS, dQbar), a column pass per 64 candidate tiles
@@ -53,7 +59,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBThreads = 352;           // warp 0 copies, warps 1 and 10 MMAs, warps 2-9 the elementwise step
+constexpr int kBThreads = 416;           // warp 0 copies, warps 1 and 10-12 MMAs, warps 2-9 the elementwise step
 constexpr int kBStages = 4;              // copy stages of 32 KB
 constexpr uint32_t kBTmemCols = 512;
 constexpr uint32_t kTB = 16384;          // one tile of Q, K, V or dO: [d half][64 rows][128 B]
@@ -74,7 +80,7 @@ constexpr uint32_t kKColS = 0, kKColP = 64, kKColDK = 256, kKColDV = 384;
 //  dkv_kernel: the key tile's K and V at 1024, stage s (Q then dO of a query
 //              tile) at 1024 + 32 KB (s + 1), then the stages' row statistics
 struct BHead {
-  uint64_t full[kBStages], free_[kBStages], s_full[2], p_full[2], ds_ready[2], a_ready, acc_done;
+  uint64_t full[kBStages], free_[kBStages], s_full[2], p_full[2], ds_ready[2], acc_a[2], a_ready, acc_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -144,10 +150,11 @@ __device__ __forceinline__ void b_init(BHead& sm, uint32_t a_ready_count, uint32
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
       mbar_init(smem_u32(&sm.p_full[i]), 1);
+      mbar_init(smem_u32(&sm.acc_a[i]), 1);      // dq: dQ of the step that used buffer i completed
       mbar_init(smem_u32(&sm.ds_ready[i]), 8);   // one arrival per elementwise warp
     }
     mbar_init(smem_u32(&sm.a_ready), a_ready_count);
-    mbar_init(smem_u32(&sm.acc_done), 2);       // both MMA warps, after their last MMA
+    mbar_init(smem_u32(&sm.acc_done), 4);       // the four MMA warps, after their last MMA
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -248,22 +255,23 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
       });
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 10) {
-    // two MMA issuers, so that the tensor pipe interleaves two independent
-    // chains: warp 1 S = Q K^T and dQ += dS K, warp 10 dP = dO V^T (V K-major
-    // like K: [keys][d]); buffer j & 1 is rewritten only after the
-    // elementwise warps released step j - 2 (warp 1: its dQ(j - 2) precedes
-    // in issue order; warp 10: it waits for ds_ready(j - 2))
+  } else if (warp == 1 || warp >= 10) {
+    // one issuing thread per MMA chain: warp 1 S = Q K^T, warp 10 dP = dO V^T
+    // (V K-major like K: [keys][d]), warp 11 dQ += dS K (K as the MN-major B
+    // operand); warp 12 has nothing to issue here. S(j) overwrites dS(j - 2):
+    // it waits for dQ(j - 2) to complete (acc_a); dP(j) overwrites dP(j - 2):
+    // it waits for the elementwise step to release it (ds_ready).
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(64, 64, 0, 0), kIdQ = idesc_bf16_f32(64, 128, 0, 1);
-      const bool is_s = warp == 1;
       bool ok = b_wait(sm, sm.a_ready, 0, a.err);
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
+      if (warp == 1 || warp == 10) {
+        const bool is_s = warp == 1;
+        for (int j = 0; ok && j < n; ++j) {
           const int st = j % kBStages;
           const uint32_t bs = 128u * (j & 1);
           if (!(ok = b_wait(sm, sm.full[st], (j / kBStages) & 1, a.err))) break;
-          if (!is_s && j >= 2 && !(ok = b_wait(sm, sm.ds_ready[j & 1], ((j >> 1) - 1) & 1, a.err))) break;
+          if (j >= 2 && !(ok = b_wait(sm, is_s ? sm.acc_a[j & 1] : sm.ds_ready[j & 1], ((j >> 1) - 1) & 1, a.err)))
+            break;
           tc_fence_after();
           const uint64_t bd = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB + (is_s ? 0u : kTB)), 16, 1024);
           const uint32_t dcol = (is_s ? kQColS : kQColP) + bs, acol = is_s ? kQColQ : kQColDO;
@@ -272,17 +280,18 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
             umma_ts(tmem + dcol, tmem + acol + kk * 8, bd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdS, kk > 0);
           umma_commit(smem_u32(is_s ? &sm.s_full[j & 1] : &sm.p_full[j & 1]));
         }
-        if (is_s && j >= 1) {
-          const int jp = j - 1, stp = jp % kBStages;
-          if (!(ok = b_wait(sm, sm.ds_ready[jp & 1], (jp >> 1) & 1, a.err))) break;
+      } else if (warp == 11) {
+        for (int j = 0; ok && j < n; ++j) {
+          const int st = j % kBStages;
+          if (!(ok = b_wait(sm, sm.ds_ready[j & 1], (j >> 1) & 1, a.err))) break;
           tc_fence_after();
-          // dQ += dS K: dS (A) in TMEM, K as the MN-major B operand ([keys][d])
-          const uint64_t kmn = smem_desc_sw128(smem_u32(stage0 + stp * 2 * kTB), 8192, 1024);
+          const uint64_t kmn = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB), 8192, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tmem + kQColAcc, tmem + kQColS + 128u * (jp & 1) + kk * 8, kmn + kk * (2048 >> 4), kIdQ,
-                    (jp > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(smem_u32(&sm.free_[stp]));   // dP(jp) completed before the elementwise step released it
+            umma_ts(tmem + kQColAcc, tmem + kQColS + 128u * (j & 1) + kk * 8, kmn + kk * (2048 >> 4), kIdQ,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&sm.acc_a[j & 1]));
+          umma_commit(smem_u32(&sm.free_[st]));   // S(j), dP(j) completed before the elementwise step released it
         }
       }
       umma_commit(smem_u32(&sm.acc_done));     // every MMA issued, also on a failed wait
@@ -409,13 +418,16 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant
       });
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 10) {
+  } else if (warp == 1 || warp >= 10) {
     // two MMA issuers: warp 1 S^T = K Q^T and dV += P^T dO, warp 10
     // dP^T = V dO^T and dK += dS^T Q (K, V, Q and dO K-major in shared memory
     // for the products; dO and Q as MN-major B operands, [queries][d], for
     // the accumulations); each rewrites its half of buffer j & 1 only after
-    // its own accumulation of step j - 2, and both release a stage
-    if (lane == 0) {
+    // its own accumulation of step j - 2 (one thread's MMAs run in issue
+    // order), and both release a stage. (Separate warps for the
+    // accumulations made the products wait for their completion: slower.)
+    // Warps 11 and 12 have nothing to issue here.
+    if (lane == 0 && (warp == 1 || warp == 10)) {
       constexpr uint32_t kIdS = idesc_bf16_f32(64, 64, 0, 0), kIdA = idesc_bf16_f32(64, 128, 0, 1);
       const bool is_s = warp == 1;
       const uint64_t ad = smem_desc_sw128(smem_u32(kvt + (is_s ? 0u : kTB)), 16, 1024);
@@ -450,6 +462,9 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant
         }
       }
       umma_commit(smem_u32(&sm.acc_done));     // every MMA issued, also on a failed wait
+      mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+    } else if (lane == 0) {
+      umma_commit(smem_u32(&sm.acc_done));     // no MMAs: arrives at once
       mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
     }
     __syncwarp();
