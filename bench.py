@@ -435,6 +435,39 @@ def run_ours(args):
         select()
         attend()
 
+    if args.profile_call is not None:
+        # warmup + steps calls of one entry point and nothing timed: the run a
+        # kernel profiler captures (the backward and the token ranking are not
+        # in the headline step)
+        if args.profile_call == "backward":
+            gen = torch.Generator(device=dev).manual_seed(77)
+            dout = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+            grads = [torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3)]
+            dg = torch.empty(g.shape, dtype=torch.float32, device=dev)
+            ws = torch.empty(lay.sparse_attn_bwd_workspace_size(wl.B, wl.H, params), dtype=torch.uint8, device=dev)
+            select()
+            call = lambda: vsa.sparse_attn_bwd(lay, params, q, k, v, g, fwd.idx, fwd.cnt, fwd.kmax, fwd.o_coarse,
+                                               dout, *grads, dg, ws, stream)
+
+            def check():
+                if vsa.sparse_attn_bwd_status(ws, stream) != vsa.OK:
+                    raise RuntimeError("backward: a kernel wait ran out")
+        else:
+            call = select if args.profile_call == "select" else step
+
+            def check():
+                check_failures(fwd, stream, "profiled calls")
+                if vsa.coarse_select_status(fwd.ws_select, stream) != vsa.OK or (
+                        args.extra_tokens > 0 and vsa.extra_tokens_status(fwd.ws_extra, stream) != vsa.OK):
+                    raise RuntimeError("profiled calls: a selection kernel wait ran out")
+        for _ in range(args.warmup + args.steps):
+            call()
+        torch.cuda.synchronize()
+        check()
+        print(json.dumps({"profile_call": args.profile_call, "workload": args.workload,
+                          "extra_tokens": args.extra_tokens, "calls": args.warmup + args.steps}), flush=True)
+        return
+
     for _ in range(args.warmup):
         step()
     check_failures(fwd, stream, "warm-up")
@@ -634,6 +667,9 @@ def main():
     ap.add_argument("--extra-tokens", type=int, default=0,
                     help="extra_tokens E (0..64): the E best tokens beyond each query tile's selected tiles")
     ap.add_argument("--ref-tiles", type=int, default=48)
+    ap.add_argument("--profile-call", choices=["step", "select", "backward"], default=None,
+                    help="only run warmup + steps calls of one entry point (selection incl. the token ranking, "
+                         "the whole step, or the backward) for a kernel profiler; prints no bench line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the torch SDPA comparator")
     ap.add_argument("--no-configs", action="store_true",
