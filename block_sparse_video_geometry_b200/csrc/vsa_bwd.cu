@@ -23,12 +23,13 @@
 //    in TMEM and K, V bulk-copied tiles (the forward's tile-major copies), the
 //    fp32 elementwise step writes dS as bf16 over S in TMEM, and
 //    dQ += dS K accumulates in TMEM (K as the MN-major B operand).
-//  * dkv_kernel: one CTA per (batch, head, key tile) walking the query tiles
-//    that attend it (all of them for conditioning keys; for a candidate tile,
-//    dense conditioning rows plus the transpose of the selection lists, built
-//    on the GPU by a counting sort); S^T = K Q^T and dP^T = V dO^T with K, V,
-//    Q and dO as bulk-copied shared-memory tiles, then dV += P^T dO and
-//    dK += dS^T Q with P^T, dS^T (bf16) in TMEM.
+//  * dkv_kernel: one CTA per (batch, head, candidate key tile) walking the
+//    query tiles that attend it (dense conditioning rows plus the transpose of
+//    the selection lists, built on the GPU by a counting sort); S^T = K Q^T
+//    and dP^T = V dO^T with K, V, Q and dO as bulk-copied shared-memory tiles,
+//    then dV += P^T dO and dK += dS^T Q with P^T, dS^T (bf16) in TMEM.
+//  * dkv_pair_kernel: the conditioning key tiles (sink on), which every query
+//    tile attends, two per CTA as M = 128 products over the same query steps.
 //  * Both are warp-specialised pipelines: a copy warp keeps four 32 KB stages
 //    in flight; the MMAs are spread over several issuing warps (each
 //    tcgen05.mma holds its thread for tens of cycles, so one thread issuing a
@@ -81,6 +82,7 @@ constexpr uint32_t kKColS = 0, kKColP = 64, kKColDK = 256, kKColDV = 384;
 //              tile) at 1024 + 32 KB (s + 1), then the stages' row statistics
 struct BHead {
   uint64_t full[kBStages], free_[kBStages], s_full[2], p_full[2], ds_ready[2], acc_a[2], a_ready, acc_done;
+  uint64_t qpair[4];                     // dkv_pair_kernel: the two warps of a lane quadrant, once per step
   uint32_t tmem_base;
   int abort;
 };
@@ -154,6 +156,7 @@ __device__ __forceinline__ void b_init(BHead& sm, uint32_t a_ready_count, uint32
       mbar_init(smem_u32(&sm.ds_ready[i]), 8);   // one arrival per elementwise warp
     }
     mbar_init(smem_u32(&sm.a_ready), a_ready_count);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&sm.qpair[i]), 2);
     mbar_init(smem_u32(&sm.acc_done), 4);       // the four MMA warps, after their last MMA
     sm.abort = 0;
     fence_mbar_init();
@@ -212,12 +215,10 @@ __device__ __forceinline__ int dq_step_tile(const BArgs& a, size_t row, int jj, 
   return a.cand0 + min(max(c, 0), a.n_cand - 1);
 }
 
-// Query tile of step jj of key tile kt's attending set: all query tiles for a
-// conditioning key tile (sink on); otherwise dense conditioning rows, then the
-// query tiles whose lists hold the tile.
-__device__ __forceinline__ int dkv_step_tile(const BArgs& a, const int32_t* list, int jj, bool all_rows) {
-  if (all_rows || jj < a.c0) return jj;
-  return list[jj - a.c0];
+// Query tile of step jj of candidate key tile kt's attending set: the dense
+// conditioning rows, then the query tiles whose lists hold the tile.
+__device__ __forceinline__ int dkv_step_tile(const BArgs& a, const int32_t* list, int jj) {
+  return jj < a.c0 ? jj : list[jj - a.c0];
 }
 
 // -------------------------------------------------------------------- dQ
@@ -385,19 +386,13 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant
   float* const rowstat = reinterpret_cast<float*>(stage0 + kBStages * 2 * kTB);   // [stage][lse, D][64]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (a.sink != VSA_SINK_OFF && kt < a.n_cond) return;   // dkv_pair_kernel's key tiles
   const size_t bh = static_cast<size_t>(b) * a.H + h;
   const int n_tiles = a.L.n_tiles;
-  const bool all_rows = a.sink != VSA_SINK_OFF && kt < a.n_cond;
-  const int c = kt - a.cand0;                       // candidate ordinal when not all_rows
-  const int32_t* list = nullptr;
-  int n;
-  if (all_rows) {
-    n = n_tiles;
-  } else {
-    const int32_t* off = a.csr_off + bh * (a.n_cand + 1);
-    list = a.csr_list + off[c];
-    n = a.c0 + (off[c + 1] - off[c]);
-  }
+  const int c = kt - a.cand0;                       // candidate ordinal
+  const int32_t* off = a.csr_off + bh * (a.n_cand + 1);
+  const int32_t* list = a.csr_list + off[c];
+  const int n = a.c0 + (off[c + 1] - off[c]);
   b_init(sm, 1, 2);
   const uint32_t tmem = sm.tmem_base;
 
@@ -408,7 +403,7 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant
       mbar_arrive_expect_tx(smem_u32(&sm.a_ready), 2 * kTB);
       bulk_load(smem_u32(kvt), a.kv + (bh * n_tiles + kt) * 32768u, 2 * kTB, smem_u32(&sm.a_ready));
       b_copy_loop(sm, n, a.err, [&](int j, int st, uint32_t bar) {
-        const size_t tq = bh * n_tiles + dkv_step_tile(a, list, j, all_rows);
+        const size_t tq = bh * n_tiles + dkv_step_tile(a, list, j);
         const uint32_t dst = smem_u32(stage0 + st * 2 * kTB);
         mbar_arrive_expect_tx(bar, 2 * kTB + 2 * 256);
         bulk_load(dst, a.qtm + tq * kTB, kTB, bar);
@@ -530,6 +525,182 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_kernel(const __grid_constant
             for (int i = 0; i < 32; i += 4)
               dst[i / 4] = make_float4(y[i] * f, y[i + 1] * f, y[i + 2] * f, y[i + 3] * f);
           }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBTmemCols);
+  }
+}
+
+// ----------------------------- dK and dV of the conditioning key tiles, in pairs
+// Every query tile attends the conditioning key tiles (sink on), so two of
+// them share each step as one M = 128 product: rows 0-63 are key tile kt0,
+// rows 64-127 key tile kt0 + 1 (an odd last tile leaves rows 64-127 unused;
+// rows never mix in these products, and nothing reads those rows back). An
+// M = 128 MMA takes about as long as an M = 64 MMA of the same N, so a pair
+// costs about one dkv_kernel step. Same roles and barriers as dkv_kernel;
+// TMEM lane = key row (M = 128 layout). The two warps of a lane quadrant split
+// a row's 64 query columns and meet at a barrier between reading S^T, dP^T
+// and writing P^T, dS^T (bf16 pairs) over them, since the pairs of the second
+// warp's columns land in fp32 columns the first warp reads.
+constexpr size_t kDkvPairSmem = 1024 + 4 * kTB + kBStages * 2 * kTB + kBStages * 2 * 64 * sizeof(float);
+
+// 32 lanes x 16 consecutive 32-bit columns (one lane per thread)
+__device__ __forceinline__ void tmem_st32x32_16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kBThreads, 1) dkv_pair_kernel(const __grid_constant__ BArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
+    return;
+  }
+  BHead& sm = *reinterpret_cast<BHead*>(smem_raw);
+  uint8_t* const kp = smem_raw + 1024;              // K of the pair: [d half][128 rows][128 B]
+  uint8_t* const vp = kp + 2 * kTB;                 // V of the pair, same layout
+  uint8_t* const stage0 = vp + 2 * kTB;
+  float* const rowstat = reinterpret_cast<float*>(stage0 + kBStages * 2 * kTB);   // [stage][lse, D][64]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt0 = 2 * blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nk = min(2, a.n_cond - kt0);            // key tiles of this pair
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  const int n_tiles = a.L.n_tiles;
+  const int n = n_tiles;                            // every query tile attends them
+  b_init(sm, 1, 2);
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(smem_u32(&sm.a_ready), 4u * 8192u * nk);
+      for (int i = 0; i < nk; ++i) {
+        const uint8_t* src = a.kv + (bh * n_tiles + kt0 + i) * 32768u;
+        for (int dh = 0; dh < 2; ++dh) {
+          bulk_load(smem_u32(kp + dh * kTB + i * 8192), src + dh * 8192, 8192, smem_u32(&sm.a_ready));
+          bulk_load(smem_u32(vp + dh * kTB + i * 8192), src + kTB + dh * 8192, 8192, smem_u32(&sm.a_ready));
+        }
+      }
+      b_copy_loop(sm, n, a.err, [&](int j, int st, uint32_t bar) {
+        const size_t tq = bh * n_tiles + j;
+        const uint32_t dst = smem_u32(stage0 + st * 2 * kTB);
+        mbar_arrive_expect_tx(bar, 2 * kTB + 2 * 256);
+        bulk_load(dst, a.qtm + tq * kTB, kTB, bar);
+        bulk_load(dst + kTB, a.dotm + tq * kTB, kTB, bar);
+        bulk_load(smem_u32(rowstat + st * 128), a.lse + tq * kTile, 256, bar);
+        bulk_load(smem_u32(rowstat + st * 128 + 64), a.dd + tq * kTile, 256, bar);
+      });
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp >= 10) {
+    // as dkv_kernel: warp 1 S^T and dV, warp 10 dP^T and dK, M = 128
+    if (lane == 0 && (warp == 1 || warp == 10)) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, 0, 0), kIdA = idesc_bf16_f32(128, 128, 0, 1);
+      const bool is_s = warp == 1;
+      const uint64_t ad = smem_desc_sw128(smem_u32(is_s ? kp : vp), 16, 1024);
+      bool ok = b_wait(sm, sm.a_ready, 0, a.err);
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % kBStages;
+          const uint32_t bs = 128u * (j & 1);
+          if (!(ok = b_wait(sm, sm.full[st], (j / kBStages) & 1, a.err))) break;
+          tc_fence_after();
+          const uint64_t bd = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB + (is_s ? 0u : kTB)), 16, 1024);
+          const uint32_t dcol = (is_s ? kKColS : kKColP) + bs;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + dcol, ad + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2, bd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2,
+                    kIdS, kk > 0);
+          umma_commit(smem_u32(is_s ? &sm.s_full[j & 1] : &sm.p_full[j & 1]));
+        }
+        if (j >= 1) {
+          const int jp = j - 1, stp = jp % kBStages;
+          const uint32_t bp = 128u * (jp & 1);
+          if (!(ok = b_wait(sm, sm.ds_ready[jp & 1], (jp >> 1) & 1, a.err))) break;
+          tc_fence_after();
+          const uint64_t bmn = smem_desc_sw128(smem_u32(stage0 + stp * 2 * kTB + (is_s ? kTB : 0u)), 8192, 1024);
+          const uint32_t acc = is_s ? kKColDV : kKColDK, acol = (is_s ? kKColS : kKColP) + bp;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + acc, tmem + acol + kk * 8, bmn + kk * (2048 >> 4), kIdA, (jp > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&sm.free_[stp]));
+        }
+      }
+      umma_commit(smem_u32(&sm.acc_done));     // every MMA issued, also on a failed wait
+      mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+    } else if (lane == 0) {
+      umma_commit(smem_u32(&sm.acc_done));     // no MMAs: arrives at once
+      mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // thread (key row r = 32 qd + lane) of column set cs: queries 32 cs .. 32 cs + 31
+    const int qd = warp & 3, cs = (warp - 2) >> 2;
+    const int r = 32 * qd + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kBStages;
+      const uint32_t bs = 128u * (j & 1);
+      if (!(ok = b_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, a.err))) break;
+      if (!(ok = b_wait(sm, sm.p_full[j & 1], (j >> 1) & 1, a.err))) break;
+      tc_fence_after();
+      float s[32], dp[32];
+      tmem_ld32x32f(lane_addr + kKColS + bs + 32 * cs, s);
+      tmem_ld32x32f(lane_addr + kKColP + bs + 32 * cs, dp);
+      tmem_wait_ld();
+      // both column sets of this quadrant have read their scores (a bounded
+      // barrier wait, so that a warp leaving on a failed wait strands no one)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.qpair[qd]));
+      if (!(ok = b_wait(sm, sm.qpair[qd], j & 1, a.err))) break;
+      uint32_t wp[16], wd[16];
+      const float* lse = rowstat + st * 128 + 32 * cs;
+      const float* dd = rowstat + st * 128 + 64 + 32 * cs;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float p[2], ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int qi = 2 * i + e;
+          p[e] = ex2_approx(fmaf(s[qi], a.c_log2, -lse[qi]));    // padding query rows: lse = +inf, P = 0
+          ds[e] = p[e] * (dp[qi] - dd[qi]);
+        }
+        wp[i] = pack_bf16x2(p[0], p[1]);
+        wd[i] = pack_bf16x2(ds[0], ds[1]);
+      }
+      tmem_st32x32_16(lane_addr + kKColS + bs + 16 * cs, wp);     // P^T over S^T
+      tmem_st32x32_16(lane_addr + kKColP + bs + 16 * cs, wd);     // dS^T over dP^T
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.ds_ready[j & 1]));
+    }
+    if (ok && (ok = b_wait(sm, sm.acc_done, 0, a.err))) {
+      tc_fence_after();
+      const int i = r >> 6;                        // key tile kt0 + i, slot r & 63
+      const int tok = i < nk ? a.L.perm[(kt0 + i) * kTile + (r & 63)] : -1;
+      float* dst_base = cs == 0 ? a.dk : a.dv;     // set 0: dK (scaled), set 1: dV
+      const float f = cs == 0 ? a.scale : 1.0f;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float y[32];
+        tmem_ld32x32f(lane_addr + (cs == 0 ? kKColDK : kKColDV) + 32 * ch, y);
+        tmem_wait_ld();
+        if (tok >= 0) {
+          float4* dst = reinterpret_cast<float4*>(dst_base + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
+                                                  h * a.o_sh + 32 * ch);
+#pragma unroll
+          for (int k4 = 0; k4 < 32; k4 += 4)
+            dst[k4 / 4] = make_float4(y[k4] * f, y[k4 + 1] * f, y[k4 + 2] * f, y[k4 + 3] * f);
         }
       }
     }
@@ -1141,7 +1312,12 @@ vsa_status vsa_sparse_attn_bwd(const vsa_layout* L, const vsa_params* p, int32_t
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dq)", e);
   e = cudaFuncSetAttribute(dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDkvSmem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dkv)", e);
+  e = cudaFuncSetAttribute(dkv_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kDkvPairSmem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dkv pair)", e);
   dq_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kDqSmem, stream>>>(a);
+  if (p->sink != VSA_SINK_OFF && L->n_cond > 0)
+    dkv_pair_kernel<<<dim3((L->n_cond + 1) / 2, H, B), kBThreads, kDkvPairSmem, stream>>>(a);
   dkv_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kDkvSmem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: fine-branch launch", e);
