@@ -18,11 +18,14 @@
 //            flow back through the pooling (1 / tile count to every valid token).
 //
 // B200 design:
-//  * dq_kernel: one CTA per (batch, head, query tile) walking its key set; per
-//    key tile S = Q K^T and dP = dO V^T are M = 64 tcgen05 MMAs with Q and dO
-//    in TMEM and K, V bulk-copied tiles (the forward's tile-major copies), the
-//    fp32 elementwise step writes dS as bf16 over S in TMEM, and
-//    dQ += dS K accumulates in TMEM (K as the MN-major B operand).
+//  * dq_kernel: one CTA per (batch, head, query tile) walking its selection
+//    list; per key tile S = Q K^T and dP = dO V^T are M = 64 tcgen05 MMAs
+//    with Q and dO in TMEM and K, V bulk-copied tiles (the forward's
+//    tile-major copies), the fp32 elementwise step writes dS as bf16 over S
+//    in TMEM, and dQ += dS K accumulates in TMEM (K as the MN-major B
+//    operand). dq_pair_kernel runs the key tiles every query tile shares (the
+//    conditioning tiles; all tiles for dense conditioning rows) for two query
+//    tiles at a time as M = 128 products and writes dQ first; dq_kernel adds.
 //  * dkv_kernel: one CTA per (batch, head, candidate key tile) walking the
 //    query tiles that attend it (dense conditioning rows plus the transpose of
 //    the selection lists, built on the GPU by a counting sort); S^T = K Q^T
@@ -111,6 +114,7 @@ struct BArgs {
   float* dv;
   int64_t o_sb, o_ss, o_sh;
   float scale, c_log2;
+  int32_t dq_add;                        // dq_kernel adds to the dQ dq_pair_kernel wrote
   int* err;
 };
 
@@ -206,12 +210,9 @@ __device__ __forceinline__ void rows_to_tmem(const uint16_t* base, const int32_t
   tmem_st16x2_32<32>(taddr, w);
 }
 
-// Key tile of step jj of query tile qt's key set in the forward: dense rows
-// all tiles; otherwise the conditioning tiles (unless the sink is off), then
-// the selection list.
-__device__ __forceinline__ int dq_step_tile(const BArgs& a, size_t row, int jj, bool dense, int n_fixed) {
-  if (dense || jj < n_fixed) return jj;
-  const int c = a.idx[row * a.kmax + (jj - n_fixed)];
+// Key tile of step jj of query tile row's selection list.
+__device__ __forceinline__ int dq_step_tile(const BArgs& a, size_t row, int jj) {
+  const int c = a.idx[row * a.kmax + jj];
   return a.cand0 + min(max(c, 0), a.n_cand - 1);
 }
 
@@ -236,11 +237,10 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
   uint8_t* const stage0 = smem_raw + 1024;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (qt < a.c0) return;                           // dense conditioning rows: dq_pair_kernel
   const size_t bh = static_cast<size_t>(b) * a.H + h;
   const size_t row = bh * a.L.n_tiles + qt;
-  const bool dense = qt < a.c0;
-  const int n_fixed = (a.sink == VSA_SINK_OFF || dense) ? 0 : a.n_cond;
-  const int n = dense ? a.L.n_tiles : n_fixed + min(max(a.cnt[row], 1), a.kmax);
+  const int n = min(max(a.cnt[row], 1), a.kmax);   // the selection list (the shared key tiles: dq_pair_kernel)
   b_init(sm, 8, 1);
   const uint32_t tmem = sm.tmem_base;
 
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
     if (lane == 0) {
       const uint8_t* head_kv = a.kv + bh * a.L.n_tiles * 32768u;
       b_copy_loop(sm, n, a.err, [&](int j, int st, uint32_t bar) {
-        const int t = dq_step_tile(a, row, j, dense, n_fixed);
+        const int t = dq_step_tile(a, row, j);
         const uint32_t dst = smem_u32(stage0 + st * 2 * kTB);
         mbar_arrive_expect_tx(bar, 2 * kTB);
         bulk_load(dst, head_kv + static_cast<size_t>(t) * 32768u, kTB, bar);
@@ -313,11 +313,11 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
     if (lane == 0) mbar_arrive(smem_u32(&sm.a_ready));
     const float lse = a.lse[row * kTile + r];
     const float dd = a.dd[row * kTile + r];
-    unsigned long long vm_next = a.L.valid[dq_step_tile(a, row, 0, dense, n_fixed)];
+    unsigned long long vm_next = a.L.valid[dq_step_tile(a, row, 0)];
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const unsigned long long vm = vm_next;
-      if (j + 1 < n) vm_next = a.L.valid[dq_step_tile(a, row, j + 1, dense, n_fixed)];
+      if (j + 1 < n) vm_next = a.L.valid[dq_step_tile(a, row, j + 1)];
       const uint32_t bs = 128u * (j & 1);
       if (!(ok = b_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, a.err))) break;
       if (!(ok = b_wait(sm, sm.p_full[j & 1], (j >> 1) & 1, a.err))) break;
@@ -356,8 +356,17 @@ __global__ void __launch_bounds__(kBThreads, 1) dq_kernel(const __grid_constant_
         float4* dst = reinterpret_cast<float4*>(a.dq + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
                                                 h * a.o_sh + 64 * hf + 32 * ch);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          dst[i / 4] = make_float4(y[i] * a.scale, y[i + 1] * a.scale, y[i + 2] * a.scale, y[i + 3] * a.scale);
+        for (int i = 0; i < 32; i += 4) {
+          float4 v = make_float4(y[i] * a.scale, y[i + 1] * a.scale, y[i + 2] * a.scale, y[i + 3] * a.scale);
+          if (a.dq_add) {
+            const float4 u = dst[i / 4];
+            v.x += u.x;
+            v.y += u.y;
+            v.z += u.z;
+            v.w += u.w;
+          }
+          dst[i / 4] = v;
+        }
       }
     }
   }
@@ -701,6 +710,192 @@ __global__ void __launch_bounds__(kBThreads, 1) dkv_pair_kernel(const __grid_con
 #pragma unroll
           for (int k4 = 0; k4 < 32; k4 += 4)
             dst[k4 / 4] = make_float4(y[k4] * f, y[k4 + 1] * f, y[k4 + 2] * f, y[k4 + 3] * f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBTmemCols);
+  }
+}
+
+// ------------------------------- dQ of the shared key tiles, query tiles in pairs
+// Every query tile attends the conditioning key tiles (sink on), and a dense
+// conditioning row attends every tile, so two query tiles share each of those
+// steps as one M = 128 product: rows 0-63 query tile qa, rows 64-127 query
+// tile qb (missing at an odd end: its rows hold zero Q and dO and an infinite
+// log-sum, so P and dS vanish there). Pairs are formed among the dense rows
+// (all tiles) and among the other query tiles (the conditioning tiles); the
+// kernel writes dQ of those steps and dq_kernel adds the selection-list steps
+// of the non-dense tiles. Same roles and barriers as dq_kernel with TMEM lane =
+// query row; the two warps of a lane quadrant split the 64 key columns and
+// meet at a bounded barrier before writing dS (bf16 pairs) over the scores.
+constexpr size_t kDqPairSmem = 1024 + kBStages * 2 * kTB;
+
+// One row (64 tokens' worth of bf16 pairs: 64 columns) of a natural-layout
+// [B, S, H, 128] tensor into TMEM lane `taddr` (32x32b shape: one lane per
+// thread), zeros for a missing token.
+__device__ __forceinline__ void row_to_tmem32(const uint16_t* base, int tok, int64_t ss, uint32_t taddr) {
+  const uint4* src = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(tok) * ss);
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    uint32_t w[32];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      const uint4 u = tok >= 0 ? __ldg(src + 8 * half + cc) : make_uint4(0u, 0u, 0u, 0u);
+      w[4 * cc] = u.x;
+      w[4 * cc + 1] = u.y;
+      w[4 * cc + 2] = u.z;
+      w[4 * cc + 3] = u.w;
+    }
+    tmem_st32x32(taddr + 32 * half, w);
+  }
+}
+
+__global__ void __launch_bounds__(kBThreads, 1) dq_pair_kernel(const __grid_constant__ BArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicExch(a.err, VSA_ERR_UNSUPPORTED);
+    return;
+  }
+  BHead& sm = *reinterpret_cast<BHead*>(smem_raw);
+  uint8_t* const stage0 = smem_raw + 1024;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int n_tiles = a.L.n_tiles;
+  const int n_dense_pairs = (a.c0 + 1) / 2;
+  int qa, qb, n;                                   // the pair's query tiles (qb < 0: none) and steps
+  if (static_cast<int>(blockIdx.x) < n_dense_pairs) {
+    qa = 2 * blockIdx.x;
+    qb = qa + 1 < a.c0 ? qa + 1 : -1;
+    n = n_tiles;
+  } else {
+    qa = a.c0 + 2 * (blockIdx.x - n_dense_pairs);
+    qb = qa + 1 < n_tiles ? qa + 1 : -1;
+    n = a.n_cond;
+  }
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  b_init(sm, 8, 1);
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {                               // step j: key tile j
+      const uint8_t* head_kv = a.kv + bh * n_tiles * 32768u;
+      b_copy_loop(sm, n, a.err, [&](int j, int st, uint32_t bar) {
+        const uint32_t dst = smem_u32(stage0 + st * 2 * kTB);
+        mbar_arrive_expect_tx(bar, 2 * kTB);
+        bulk_load(dst, head_kv + static_cast<size_t>(j) * 32768u, kTB, bar);
+        bulk_load(dst + kTB, head_kv + static_cast<size_t>(j) * 32768u + kTB, kTB, bar);
+      });
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp >= 10) {
+    // as dq_kernel, M = 128: warp 1 S, warp 10 dP, warp 11 dQ
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, 0, 0), kIdQ = idesc_bf16_f32(128, 128, 0, 1);
+      bool ok = b_wait(sm, sm.a_ready, 0, a.err);
+      if (warp == 1 || warp == 10) {
+        const bool is_s = warp == 1;
+        for (int j = 0; ok && j < n; ++j) {
+          const int st = j % kBStages;
+          const uint32_t bs = 128u * (j & 1);
+          if (!(ok = b_wait(sm, sm.full[st], (j / kBStages) & 1, a.err))) break;
+          if (j >= 2 && !(ok = b_wait(sm, is_s ? sm.acc_a[j & 1] : sm.ds_ready[j & 1], ((j >> 1) - 1) & 1, a.err)))
+            break;
+          tc_fence_after();
+          const uint64_t bd = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB + (is_s ? 0u : kTB)), 16, 1024);
+          const uint32_t dcol = (is_s ? kQColS : kQColP) + bs, acol = is_s ? kQColQ : kQColDO;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + dcol, tmem + acol + kk * 8, bd + (kk >> 2) * (8192 >> 4) + (kk & 3) * 2, kIdS, kk > 0);
+          umma_commit(smem_u32(is_s ? &sm.s_full[j & 1] : &sm.p_full[j & 1]));
+        }
+      } else if (warp == 11) {
+        for (int j = 0; ok && j < n; ++j) {
+          const int st = j % kBStages;
+          if (!(ok = b_wait(sm, sm.ds_ready[j & 1], (j >> 1) & 1, a.err))) break;
+          tc_fence_after();
+          const uint64_t kmn = smem_desc_sw128(smem_u32(stage0 + st * 2 * kTB), 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + kQColAcc, tmem + kQColS + 128u * (j & 1) + kk * 8, kmn + kk * (2048 >> 4), kIdQ,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&sm.acc_a[j & 1]));
+          umma_commit(smem_u32(&sm.free_[st]));
+        }
+      }
+      umma_commit(smem_u32(&sm.acc_done));     // every MMA issued, also on a failed wait
+      mbar_wait(smem_u32(&sm.acc_done), 0, nullptr, kBDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // thread (query row r = 32 qd + lane) of column set cs: keys 32 cs .. 32 cs + 31
+    const int qd = warp & 3, cs = (warp - 2) >> 2;
+    const int r = 32 * qd + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const int qt = r < 64 ? qa : qb;
+    const int tok = qt >= 0 ? a.L.perm[qt * kTile + (r & 63)] : -1;
+    if (cs == 0) row_to_tmem32(a.q + b * a.sb + h * a.sh, tok, a.ss, lane_addr + kQColQ);
+    else row_to_tmem32(a.dout + b * a.d_sb + h * a.d_sh, tok, a.d_ss, lane_addr + kQColDO);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.a_ready));
+    const size_t srow = (bh * n_tiles + (qt >= 0 ? qt : 0)) * kTile + (r & 63);
+    const float lse = qt >= 0 ? a.lse[srow] : INFINITY;
+    const float dd = qt >= 0 ? a.dd[srow] : 0.f;
+    unsigned long long vm_next = a.L.valid[0];
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const unsigned long long vm = vm_next;
+      if (j + 1 < n) vm_next = a.L.valid[j + 1];
+      const uint32_t bs = 128u * (j & 1);
+      if (!(ok = b_wait(sm, sm.s_full[j & 1], (j >> 1) & 1, a.err))) break;
+      if (!(ok = b_wait(sm, sm.p_full[j & 1], (j >> 1) & 1, a.err))) break;
+      tc_fence_after();
+      float s[32], dp[32];
+      tmem_ld32x32f(lane_addr + kQColS + bs + 32 * cs, s);
+      tmem_ld32x32f(lane_addr + kQColP + bs + 32 * cs, dp);
+      tmem_wait_ld();
+      // both column sets of this quadrant have read their scores (bounded)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.qpair[qd]));
+      if (!(ok = b_wait(sm, sm.qpair[qd], j & 1, a.err))) break;
+      const uint32_t vbits = static_cast<uint32_t>(vm >> (32 * cs));
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = 2 * i + e;
+          const float p = ((vbits >> key) & 1u) ? ex2_approx(fmaf(s[key], a.c_log2, -lse)) : 0.f;
+          ds[e] = p * (dp[key] - dd);
+        }
+        w[i] = pack_bf16x2(ds[0], ds[1]);
+      }
+      tmem_st32x32_16(lane_addr + kQColS + bs + 16 * cs, w);    // dS (bf16 pairs) over S
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.ds_ready[j & 1]));
+    }
+    if (ok && (ok = b_wait(sm, sm.acc_done, 0, a.err))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 2 * cs; ch < 2 * cs + 2; ++ch) {   // dims 32 ch .. 32 ch + 31
+        float y[32];
+        tmem_ld32x32f(lane_addr + kQColAcc + 32 * ch, y);
+        tmem_wait_ld();
+        if (tok >= 0) {
+          float4* dst = reinterpret_cast<float4*>(a.dq + b * a.o_sb + static_cast<int64_t>(tok) * a.o_ss +
+                                                  h * a.o_sh + 32 * ch);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            dst[i / 4] = make_float4(y[i] * a.scale, y[i + 1] * a.scale, y[i + 2] * a.scale, y[i + 3] * a.scale);
         }
       }
     }
@@ -1308,6 +1503,10 @@ vsa_status vsa_sparse_attn_bwd(const vsa_layout* L, const vsa_params* p, int32_t
   a.scale = scale;
   a.c_log2 = scale * 1.4426950408889634f;
   a.err = static_cast<int*>(workspace);
+  a.dq_add = (p->sink != VSA_SINK_OFF && L->n_cond > 0) ? 1 : 0;
+  e = cudaFuncSetAttribute(dq_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kDqPairSmem));
+  if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dq pair)", e);
   e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDqSmem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dq)", e);
   e = cudaFuncSetAttribute(dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDkvSmem));
@@ -1315,6 +1514,8 @@ vsa_status vsa_sparse_attn_bwd(const vsa_layout* L, const vsa_params* p, int32_t
   e = cudaFuncSetAttribute(dkv_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kDkvPairSmem));
   if (e != cudaSuccess) return cuda_fail("vsa_sparse_attn_bwd: cudaFuncSetAttribute(dkv pair)", e);
+  if (a.dq_add)
+    dq_pair_kernel<<<dim3((c0 + 1) / 2 + (L->n_tiles - c0 + 1) / 2, H, B), kBThreads, kDqPairSmem, stream>>>(a);
   dq_kernel<<<dim3(L->n_tiles, H, B), kBThreads, kDqSmem, stream>>>(a);
   if (p->sink != VSA_SINK_OFF && L->n_cond > 0)
     dkv_pair_kernel<<<dim3((L->n_cond + 1) / 2, H, B), kBThreads, kDkvPairSmem, stream>>>(a);
