@@ -21,6 +21,10 @@ pytestmark = pytest.mark.gpu
 
 SMALL = W.Workload("small", B=1, H=3, cond=((W.SEG_TEXT, 96), (W.SEG_REF_IMAGE, 64)), grid=(8, 16, 16),
                    keep=0.25, seed=21)
+# eleven conditioning tiles (one partial): the shared key tiles of dq_pair_kernel
+# and dkv_pair_kernel run past their four copy stages, with an odd last pair
+PREFIX_HEAVY = W.Workload("prefix_heavy", B=1, H=2, cond=((W.SEG_TEXT, 500), (W.SEG_REF_IMAGE, 192)),
+                          grid=(8, 16, 16), keep=0.25, seed=23)
 
 
 def oracle_grads(q, k, v, g, dout, lay, p, sel):
@@ -96,6 +100,11 @@ def test_edge_backward(cuda_ok, wl):
 @pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS])
 def test_small_multitile_backward(cuda_ok, sink):
     bwd_check(SMALL, sink=sink)
+
+
+@pytest.mark.parametrize("sink", [O.SINK_EXACT_KV, O.SINK_EXACT_KV_AND_ROWS])
+def test_prefix_heavy_backward(cuda_ok, sink):
+    bwd_check(PREFIX_HEAVY, sink=sink)
 
 
 def test_backward_refuses_what_it_does_not_differentiate(cuda_ok):
