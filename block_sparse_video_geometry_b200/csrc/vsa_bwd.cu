@@ -33,17 +33,16 @@
 //    then dV += P^T dO and dK += dS^T Q with P^T, dS^T (bf16) in TMEM.
 //  * dkv_pair_kernel: the conditioning key tiles (sink on), which every query
 //    tile attends, two per CTA as M = 128 products over the same query steps.
-//  * Both are warp-specialised pipelines: a copy warp keeps four 32 KB stages
-//    in flight; the MMAs are spread over several issuing warps (each
+//  * All four are warp-specialised pipelines: a copy warp keeps four 32 KB
+//    stages in flight; the MMAs are spread over several issuing warps (each
 //    tcgen05.mma holds its thread for tens of cycles, so one thread issuing a
 //    step's 20-24 MMAs was the bound; dq: S, dP and dQ on three warps, dkv:
 //    S^T with dV and dP^T with dK on two); the products of step j + 1 and the
 //    accumulations of step j run while eight warps do the elementwise step of
-//    the other of two TMEM score buffers (two per TMEM quadrant, each half of
-//    a thread pair's 32 columns: 16 exponentials per thread and step). A
-//    product rewrites its buffer only after the accumulation that read it two
-//    steps earlier has completed (dq: acc_a) or was issued before it by the
-//    same thread (dkv).
+//    the other of two TMEM score buffers (two per TMEM lane quadrant, each
+//    half of a row's columns). A product rewrites its buffer only after the
+//    accumulation that read it two steps earlier has completed (dq: acc_a) or
+//    was issued before it by the same thread (dkv).
 //  * The coarse branch runs on CUDA cores in fp32 (like its forward):
 //    dOc and dg in one pass over the tokens, a row pass per 64 query tiles
 //    (softmax statistics, P, dS, dQbar), a column pass per 64 candidate tiles
