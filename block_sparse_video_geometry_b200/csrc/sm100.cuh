@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers with bounded waits, bulk global -> shared copies (no multicast),
+// mbarriers with bounded waits, bulk global -> shared copies (each CTA loads its own),
 // tcgen05 MMA with TMEM accumulators, TMEM load/store in the 32x32b shape (one
 // lane per thread) and the 16x32bx2 shape (the two half-warps address the same
 // 16 lanes at two column offsets), and the
