@@ -412,6 +412,10 @@ def run_ours(args):
     wl = W.WORKLOADS[args.workload].with_(seed=sharding.replica_seed(W.WORKLOADS[args.workload].seed, rank))
     if args.sink is not None:
         wl = wl.with_(sink=SINKS[args.sink])
+    if args.heads is not None:
+        if args.profile_call is None:
+            raise SystemExit("--heads only sizes --profile-call runs; the bench line keeps the workload's heads")
+        wl = wl.with_(H=args.heads)
     lay = vsa.Layout(wl.segments(), wl.seq_len)
     perm, inv, counts, kinds = lay.tables()
     bits = W.make_inputs(wl, inv // vsa.TILE)
@@ -667,6 +671,8 @@ def main():
     ap.add_argument("--extra-tokens", type=int, default=0,
                     help="extra_tokens E (0..64): the E best tokens beyond each query tile's selected tiles")
     ap.add_argument("--ref-tiles", type=int, default=48)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="with --profile-call: the workload with this many heads (a smaller launch to capture)")
     ap.add_argument("--profile-call", choices=["step", "select", "backward"], default=None,
                     help="only run warmup + steps calls of one entry point (selection incl. the token ranking, "
                          "the whole step, or the backward) for a kernel profiler; prints no bench line")
