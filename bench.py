@@ -412,9 +412,7 @@ def run_ours(args):
     wl = W.WORKLOADS[args.workload].with_(seed=sharding.replica_seed(W.WORKLOADS[args.workload].seed, rank))
     if args.sink is not None:
         wl = wl.with_(sink=SINKS[args.sink])
-    if args.heads is not None:
-        if args.profile_call is None:
-            raise SystemExit("--heads only sizes --profile-call runs; the bench line keeps the workload's heads")
+    if args.heads is not None:                   # --profile-call runs only (checked in main)
         wl = wl.with_(H=args.heads)
     lay = vsa.Layout(wl.segments(), wl.seq_len)
     perm, inv, counts, kinds = lay.tables()
@@ -682,6 +680,8 @@ def main():
                     help="skip the other configurations (5 s adaptive tau, keep 100%%, 10 s ragged)")
     ap.add_argument("--config-calls", type=int, default=10, help="timed calls per extra configuration")
     args = ap.parse_args()
+    if args.heads is not None and args.profile_call is None:
+        ap.error("--heads only sizes --profile-call runs; the bench line keeps the workload's heads")
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
